@@ -1,0 +1,419 @@
+#!/usr/bin/env python
+"""Benchmark of exact Top-k sparse decode attention on B200.
+
+One step = one decode call over one batch of synthetic input: score every
+cached key, select the top k per query head, softmax over the kept keys,
+gather P.V, tail mass (token variant, workloads 1/2/3/5), or block select +
+attention over kept blocks (workload 4).  The default workload is the
+Llama-3-8B-shaped GQA decode layer: B=8, 32 query / 8 KV heads, d=128,
+L=32768, k=2048, bf16 cache.
+
+Prints ONE JSON line (rank 0).  Timing: W untimed warm-up steps, then exactly
+K timed steps, each bracketed by CUDA events on the launching stream, with an
+L2 flush (a 256 MiB write) between steps outside the events; the sum of the
+K step times, max over ranks.  Multi-GPU (torchrun) runs one independent
+replica per GPU (the path shards by sequence with no exchange): weak scaling.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1..5] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "Top-k decode attention queries/s and achieved HBM GB/s vs B200 peak, L=32K–128K"
+UNIT = "queries/s"
+FALLBACK_HBM_GBS = 6650.0
+SPEC_HBM_GBS = 8000.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- accounting
+
+def elem_bytes(w):
+    return 2 if w.dtype == "bf16" else 4
+
+
+def visible(w, b, qp):
+    return int(w.seq_lens[b]) - w.Q + qp + 1
+
+
+def k_bytes(w):
+    """Whole K cache read once: every kv-head's rows below its sequence length."""
+    return sum(int(w.seq_lens[b]) for b in range(w.B)) * w.Hkv * w.d * elem_bytes(w)
+
+
+def alg_bytes_token(w, k):
+    """Algorithmic bytes of one step: full K read + the k kept K and V rows of
+    every query row + q, out, idx and tail."""
+    row = w.d * elem_bytes(w)
+    kept = sum(min(k, visible(w, b, qp)) for b in range(w.B) for qp in range(w.Q)) * w.Hq
+    rows = w.B * w.Q * w.Hq
+    return k_bytes(w) + kept * 2 * row + rows * w.d * (elem_bytes(w) + 4) + rows * (k * 4 + 4)
+
+
+def alg_bytes_block(w):
+    """Block keys (fp32) of every competing block + the kept blocks' K and V rows + q/out/block_idx."""
+    bs, top = w.block_size, w.top_blocks
+    total = 0
+    for b in range(w.B):
+        Lb = int(w.seq_lens[b])
+        nblk = -(-Lb // bs)
+        comp = nblk - 1
+        total += w.Hkv * comp * w.d * 4
+        kept_tokens = min(top, comp) * bs + (Lb - (nblk - 1) * bs)
+        total += w.Hq * kept_tokens * 2 * w.d * elem_bytes(w)
+    rows = w.B * w.Hq
+    return total + rows * w.d * (elem_bytes(w) + 4) + rows * (top + 1) * 4
+
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def score_traffic(source_file):
+    """dram bytes per launch of the score kernel from the committed ncu summary,
+    if it was taken from the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "score_bf16_llama3_8b_L32768.txt")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m_b = re.search(r"^dram_bytes_per_launch_full_workload:\s*([0-9.eE+]+)", text, re.M)
+    m_h = re.search(r"^kernel_source_sha256:\s*([0-9a-f]+)", text, re.M)
+    if not m_b or not m_h:
+        return None
+    src = hashlib.sha256(open(source_file, "rb").read()).hexdigest()
+    return float(m_b.group(1)) if src == m_h.group(1) else None
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index, period=0.005):
+        self.samples, self.reasons = [], 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._period = period
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._nv:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._nv:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def time_oracle(w, k, budget_s=10.0, max_reps=50):
+    """The oracle as it stands on this host's cores, whole workload repeated
+    until `budget_s` has elapsed.  Returns (queries/s, cores, sample text)."""
+    import oracle
+    rows = w.B * w.Q * w.Hq
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        if w.variant == "block":
+            oracle.block_attn(w, w.block_size, w.top_blocks)
+        else:
+            oracle.topk_attn(w, k)
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= budget_s or reps >= max_reps:
+            break
+    sample = f"whole workload ({rows} query rows) x {reps} repetitions, {dt:.1f} s"
+    return rows * reps / dt, oracle.max_threads(), sample
+
+
+# ----------------------------------------------------------------------------- runs
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and args.impl == "ours":
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def make_inputs(cfg, rank):
+    # each rank decodes its own batch (weak scaling); rank 0 draws the tested workload
+    return workloads.config_workload(cfg, seed=1000 + cfg + 7919 * rank)
+
+
+def run_ours(args, world, rank, local):
+    import exact_top_sparse_score_b200 as tka
+    from exact_top_sparse_score_b200._binding import block_attn_workspace_size, make_shape
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = make_inputs(args.config, rank)
+    q, kc, vc, lens = (w.q.to(dev), w.k_cache.to(dev), w.v_cache.to(dev), w.seq_lens.to(dev))
+    rows = w.B * w.Q * w.Hq
+    block = w.variant == "block"
+    k = w.k
+    if block:
+        bk = tka.topk_block_pool_keys(kc, lens, w.block_size)
+        ws = torch.empty(block_attn_workspace_size(make_shape(q, kc), w.block_size, w.top_blocks),
+                         dtype=torch.uint8, device=dev)
+        out = torch.empty((w.B, w.Q, w.Hq, w.d), dtype=torch.float32, device=dev)
+        bidx = torch.empty((w.B, w.Q, w.Hq, w.top_blocks + 1), dtype=torch.int32, device=dev)
+        launches_per_step = 2
+
+        def step(events=None, qq=q):
+            if events:
+                events[0].record()
+            tka.topk_block_attn_decode(qq, kc, vc, bk, lens, w.block_size, w.top_blocks, out=out,
+                                       block_idx=bidx, workspace=ws)
+            if events:
+                events[3].record()
+        alg = alg_bytes_block(w)
+        dominant_bytes = None
+    else:
+        ws = torch.empty(tka.topk_attn_workspace_size(make_shape(q, kc), k), dtype=torch.uint8, device=dev)
+        out = torch.empty((w.B, w.Q, w.Hq, w.d), dtype=torch.float32, device=dev)
+        idx = torch.empty((w.B, w.Q, w.Hq, k), dtype=torch.int32, device=dev)
+        tail = torch.empty((w.B, w.Q, w.Hq), dtype=torch.float32, device=dev)
+        launches_per_step = 3
+
+        def step(events=None, qq=q):
+            tka.topk_attn_decode(qq, kc, vc, lens, k, out=out, idx=idx, tail_mass=tail, workspace=ws,
+                                 stage_events=events)
+        alg = alg_bytes_token(w, k)
+        dominant_bytes = k_bytes(w) + q.numel() * q.element_size()
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if tka.topk_attn_device_status() != 0:
+        raise RuntimeError("device status raised during warm-up")
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for i in range(K):
+            flush.zero_()
+            step(evs[i])
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    stage_ms = None if block else [[e[j].elapsed_time(e[j + 1]) for e in evs] for j in range(3)]
+    total_ms = sum(step_ms)
+
+    e2e_ms = None
+    h2d = d2h = 0
+    if not args.no_e2e:
+        # public API with host buffers: H2D of the step's queries and lengths
+        # from pinned memory, D2H of every result, all inside the events
+        q_host = w.q.pin_memory()
+        lens_host = w.seq_lens.pin_memory()
+        q_step = torch.empty_like(q)
+        lens_step = torch.empty_like(lens)
+        outs = [out, bidx] if block else [out, idx, tail]
+        hosts = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+        h2d = q_host.numel() * q_host.element_size() + lens_host.numel() * 4
+        d2h = sum(t.numel() * t.element_size() for t in outs)
+        e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+        for i in range(K):
+            flush.zero_()
+            e2e_ev[i][0].record()
+            q_step.copy_(q_host, non_blocking=True)
+            lens_step.copy_(lens_host, non_blocking=True)
+            if block:
+                tka.topk_block_attn_decode(q_step, kc, vc, bk, lens_step, w.block_size, w.top_blocks, out=out,
+                                           block_idx=bidx, workspace=ws)
+            else:
+                tka.topk_attn_decode(q_step, kc, vc, lens_step, k, out=out, idx=idx, tail_mass=tail, workspace=ws)
+            for h, t in zip(hosts, outs):
+                h.copy_(t, non_blocking=True)
+            e2e_ev[i][1].record()
+        torch.cuda.synchronize()
+        e2e_ms = sum(e[0].elapsed_time(e[1]) for e in e2e_ev)
+    if tka.topk_attn_device_status() != 0:
+        raise RuntimeError("device status raised during timing")
+
+    vals = torch.tensor([total_ms, e2e_ms or 0.0] + ([sum(s) for s in stage_ms] if stage_ms else [0.0] * 3),
+                        dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(vals, op=torch.distributed.ReduceOp.MAX)
+    total_ms, e2e_ms_max = float(vals[0]), float(vals[1])
+    stage_tot = [float(x) for x in vals[2:]]
+
+    if rank != 0:
+        return None
+    ms = total_ms / K
+    peak, peak_src = measured_hbm_peak()
+    res = {
+        "metric": METRIC,
+        "value": world * rows / (ms / 1e3),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.dtype,
+        "data": "synthetic (seeded numpy PCG64, rounded once to the cache dtype)",
+        "config": {
+            "workload": w.name, "B": w.B, "Q": w.Q, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "L_max": w.L_max,
+            "k": k, "block_size": w.block_size, "top_blocks": w.top_blocks,
+            "seq_lens": "full" if int(w.seq_lens.min()) == w.L_max else [int(x) for x in w.seq_lens],
+            "accumulate": "fp32", "parallelism": f"replica x{world} (independent sequences per GPU)",
+            "l2": "flushed between timed steps (256 MiB write outside the timed events)",
+        },
+        "us_per_step": ms * 1e3,
+        "tokens_per_s": world * w.B * w.Q / (ms / 1e3),
+        "alg_bytes_per_step": alg,
+        "alg_gbs": alg / (ms / 1e3) / 1e9,
+        "alg_frac_of_spec_8tbs": alg / (ms / 1e3) / 1e9 / SPEC_HBM_GBS,
+        "alg_frac_of_measured_hbm": alg / (ms / 1e3) / 1e9 / peak,
+        "gpu_launches": launches_per_step * K,
+        "clocks": clocks.summary(),
+    }
+    if stage_ms:
+        res["stage_us"] = {n: stage_tot[j] / K * 1e3 for j, n in enumerate(["score", "select", "gather"])}
+        score_s = stage_tot[0] / K / 1e3
+        achieved = dominant_bytes / score_s / 1e9
+        traffic = score_traffic(os.path.join(ROOT, "exact_top_sparse_score_b200", "csrc", "score.cu"))
+        res["roofline"] = {"kernel": "score", "bound": "hbm", "achieved": achieved, "peak": peak,
+                           "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
+                           else "fallback 6.65 TB/s", "unit": "GB/s", "frac": achieved / peak,
+                           "traffic": traffic, "alg_bytes_per_launch": dominant_bytes}
+    if e2e_ms is not None:
+        e2e_step = e2e_ms_max / K
+        res["e2e"] = {"value": world * rows / (e2e_step / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                      "d2h_bytes_per_step": d2h, "ms_per_step": e2e_step}
+    if world == 1 and not args.no_cpu_baseline:
+        v, cores, sample = time_oracle(w, k)
+        res["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+    return res
+
+
+def run_reference(args, rank):
+    """The fp64 CPU oracle as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return None
+    import oracle
+    w = make_inputs(args.config, 0)
+    rows = w.B * w.Q * w.Hq
+    k = w.k
+
+    def step():
+        if w.variant == "block":
+            oracle.block_attn(w, w.block_size, w.top_blocks)
+        else:
+            oracle.topk_attn(w, k)
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    ms = dt / args.steps * 1e3
+    value = rows / (ms / 1e3)
+    cores = oracle.max_threads()
+    sample = f"whole workload ({rows} query rows) per step"
+    return {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded numpy PCG64)",
+        "config": {"workload": w.name, "B": w.B, "Q": w.Q, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "L_max": w.L_max,
+                   "k": k, "block_size": w.block_size, "top_blocks": w.top_blocks},
+        "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    world, rank, local = dist_setup(args)
+    try:
+        res = run_reference(args, rank) if args.impl == "reference" else run_ours(args, world, rank, local)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if torch.distributed.is_initialized():
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

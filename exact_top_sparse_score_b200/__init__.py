@@ -1,0 +1,24 @@
+"""Exact Top-k sparse decode attention on B200 (sm_100a).
+
+The compute lives in ``libtopk_attn.so`` (hand-written CUDA behind a C ABI,
+declared in ``include/topk_attn.h``).  This package is a thin ctypes binding:
+it checks tensors, allocates outputs with torch when the caller passes none,
+and forwards pointers and the current CUDA stream.  There is no CPU path:
+every call fails if the library is missing or a tensor is not on a CUDA
+device.
+"""
+from ._binding import (  # noqa: F401
+    TKA_BF16,
+    TKA_F32,
+    DEV_BAD_SEQ_LEN,
+    DEV_INTERNAL,
+    TopkAttnError,
+    block_attn_workspace_size,
+    library_path,
+    load_library,
+    topk_attn_decode,
+    topk_attn_device_status,
+    topk_attn_workspace_size,
+    topk_block_attn_decode,
+    topk_block_pool_keys,
+)

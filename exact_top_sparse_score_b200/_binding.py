@@ -1,0 +1,219 @@
+"""ctypes binding of the C ABI in include/topk_attn.h (argument marshalling only)."""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "libtopk_attn.so"
+
+TKA_F32, TKA_BF16 = 0, 1
+DEV_BAD_SEQ_LEN, DEV_INTERNAL = 0x1, 0x2
+_STATUS = {0: "TKA_OK", 1: "TKA_ERR_INVALID_ARG", 2: "TKA_ERR_UNSUPPORTED", 3: "TKA_ERR_WORKSPACE",
+           4: "TKA_ERR_CUDA"}
+
+
+class TopkAttnError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} returned {_STATUS.get(code, code)}")
+        self.code = code
+
+
+class tka_shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("Q", ctypes.c_int32), ("Hq", ctypes.c_int32),
+                ("Hkv", ctypes.c_int32), ("d", ctypes.c_int32), ("L_max", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
+_lib = None
+_vp, _sz, _i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32
+_shape_p = ctypes.POINTER(tka_shape)
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, _LIB_NAME)
+
+
+def load_library() -> ctypes.CDLL:
+    """Loads the in-tree CUDA library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        path = library_path()
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: build it with `python -m exact_top_sparse_score_b200.build` "
+                               "(there is no fallback implementation)")
+        lib = ctypes.CDLL(path)
+        lib.topk_attn_workspace_size.argtypes = [_shape_p, _i32]
+        lib.topk_attn_workspace_size.restype = _sz
+        lib.topk_attn_decode.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp]
+        lib.topk_attn_decode.restype = ctypes.c_int
+        lib.topk_attn_decode_staged.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp,
+                                                ctypes.POINTER(_vp)]
+        lib.topk_attn_decode_staged.restype = ctypes.c_int
+        lib.topk_block_pool_keys.argtypes = [_shape_p, _vp, _vp, _i32, _vp, _vp]
+        lib.topk_block_pool_keys.restype = ctypes.c_int
+        lib.topk_block_attn_workspace_size.argtypes = [_shape_p, _i32, _i32]
+        lib.topk_block_attn_workspace_size.restype = _sz
+        lib.topk_block_attn_decode.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _vp,
+                                               _sz, _vp]
+        lib.topk_block_attn_decode.restype = ctypes.c_int
+        lib.topk_attn_device_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_uint32)]
+        lib.topk_attn_device_status.restype = ctypes.c_int
+        lib.topk_attn_status_string.argtypes = [ctypes.c_int]
+        lib.topk_attn_status_string.restype = ctypes.c_char_p
+        _lib = lib
+    return _lib
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return TKA_BF16
+    if t.dtype == torch.float32:
+        return TKA_F32
+    raise TypeError(f"unsupported cache dtype {t.dtype}")
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _check_cuda(**tensors):
+    for name, t in tensors.items():
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def make_shape(q: torch.Tensor, k_cache: torch.Tensor, scale: float = 0.0) -> tka_shape:
+    """Shape struct from q [B,Q,Hq,d] and a cache [B,Hkv,L_max,d]."""
+    if q.dim() != 4 or k_cache.dim() != 4:
+        raise ValueError("q must be [B,Q,Hq,d] and the caches [B,Hkv,L_max,d]")
+    B, Q, Hq, d = q.shape
+    Bk, Hkv, L_max, dk = k_cache.shape
+    if Bk != B or dk != d:
+        raise ValueError("q and cache shapes disagree")
+    if q.dtype != k_cache.dtype:
+        raise TypeError("q must have the cache dtype")
+    return tka_shape(B, Q, Hq, Hkv, d, L_max, _dtype_code(k_cache), float(scale))
+
+
+def topk_attn_workspace_size(shape: tka_shape, k: int) -> int:
+    return int(load_library().topk_attn_workspace_size(ctypes.byref(shape), k))
+
+
+def block_attn_workspace_size(shape: tka_shape, block_size: int, top_blocks: int) -> int:
+    return int(load_library().topk_block_attn_workspace_size(ctypes.byref(shape), block_size, top_blocks))
+
+
+def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]) -> torch.Tensor:
+    if workspace is None:
+        return torch.empty(nbytes, dtype=torch.uint8, device=device)
+    if workspace.numel() * workspace.element_size() < nbytes:
+        raise ValueError(f"workspace needs {nbytes} bytes")
+    return workspace
+
+
+def topk_attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, seq_lens: torch.Tensor,
+                     k: int, *, scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                     idx: Optional[torch.Tensor] = None, tail_mass: Optional[torch.Tensor] = None,
+                     workspace: Optional[torch.Tensor] = None, want_tail: bool = True,
+                     stream=None, stage_events=None) -> Tuple[torch.Tensor, torch.Tensor, Optional[torch.Tensor]]:
+    """Exact Top-k decode attention; returns (out fp32 [B,Q,Hq,d], idx int32 [B,Q,Hq,k], tail fp32 [B,Q,Hq]).
+
+    stage_events: optional four torch.cuda.Event objects recorded before score,
+    before select, before gather and after gather (topk_attn_decode_staged)."""
+    lib = load_library()
+    shape = make_shape(q, k_cache, scale)
+    B, Q, Hq, d = q.shape
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, Q, Hq, d), dtype=torch.float32, device=dev)
+    if idx is None:
+        idx = torch.empty((B, Q, Hq, k), dtype=torch.int32, device=dev)
+    if tail_mass is None and want_tail:
+        tail_mass = torch.empty((B, Q, Hq), dtype=torch.float32, device=dev)
+    if seq_lens.dtype != torch.int32:
+        raise TypeError("seq_lens must be int32")
+    _check_cuda(q=q, k_cache=k_cache, v_cache=v_cache, seq_lens=seq_lens, out=out, idx=idx, tail_mass=tail_mass,
+                workspace=workspace)
+    nbytes = topk_attn_workspace_size(shape, k)
+    if nbytes == 0:
+        raise TopkAttnError("topk_attn_workspace_size", 2)
+    ws = _workspace(nbytes, dev, workspace)
+    args = (ctypes.byref(shape), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seq_lens.data_ptr(), k,
+            out.data_ptr(), idx.data_ptr(), _ptr(tail_mass), ws.data_ptr(), nbytes, _stream(stream))
+    if stage_events is None:
+        rc = lib.topk_attn_decode(*args)
+    else:
+        evs = (_vp * 4)(*[e.cuda_event for e in stage_events])
+        rc = lib.topk_attn_decode_staged(*args, evs)
+    if rc:
+        raise TopkAttnError("topk_attn_decode", rc)
+    return out, idx, tail_mass
+
+
+def topk_block_pool_keys(k_cache: torch.Tensor, seq_lens: torch.Tensor, block_size: int, *,
+                         block_keys: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Mean-pooled block keys fp32 [B, Hkv, ceil(L_max/block_size), d]."""
+    lib = load_library()
+    B, Hkv, L_max, d = k_cache.shape
+    nblk = -(-L_max // block_size)
+    if block_keys is None:
+        block_keys = torch.empty((B, Hkv, nblk, d), dtype=torch.float32, device=k_cache.device)
+    _check_cuda(k_cache=k_cache, seq_lens=seq_lens, block_keys=block_keys)
+    shape = tka_shape(B, 1, Hkv, Hkv, d, L_max, _dtype_code(k_cache), 0.0)
+    rc = lib.topk_block_pool_keys(ctypes.byref(shape), k_cache.data_ptr(), seq_lens.data_ptr(), block_size,
+                                  block_keys.data_ptr(), _stream(stream))
+    if rc:
+        raise TopkAttnError("topk_block_pool_keys", rc)
+    return block_keys
+
+
+def topk_block_attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                           block_keys: torch.Tensor, seq_lens: torch.Tensor, block_size: int, top_blocks: int, *,
+                           scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                           block_idx: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                           stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """MoBA block-sparse decode attention; returns (out fp32 [B,1,Hq,d], block_idx int32 [B,1,Hq,top+1])."""
+    lib = load_library()
+    shape = make_shape(q, k_cache, scale)
+    B, Q, Hq, d = q.shape
+    if out is None:
+        out = torch.empty((B, Q, Hq, d), dtype=torch.float32, device=q.device)
+    if block_idx is None:
+        block_idx = torch.empty((B, Q, Hq, top_blocks + 1), dtype=torch.int32, device=q.device)
+    _check_cuda(q=q, k_cache=k_cache, v_cache=v_cache, block_keys=block_keys, seq_lens=seq_lens, out=out,
+                block_idx=block_idx, workspace=workspace)
+    nbytes = block_attn_workspace_size(shape, block_size, top_blocks)
+    if nbytes == 0:
+        raise TopkAttnError("topk_block_attn_workspace_size", 2)
+    ws = _workspace(nbytes, q.device, workspace)
+    rc = lib.topk_block_attn_decode(ctypes.byref(shape), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                    block_keys.data_ptr(), seq_lens.data_ptr(), block_size, top_blocks,
+                                    out.data_ptr(), block_idx.data_ptr(), ws.data_ptr(), nbytes, _stream(stream))
+    if rc:
+        raise TopkAttnError("topk_block_attn_decode", rc)
+    return out, block_idx
+
+
+def topk_attn_device_status(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device status bits."""
+    bits = ctypes.c_uint32(0)
+    rc = load_library().topk_attn_device_status(_stream(stream), ctypes.byref(bits))
+    if rc:
+        raise TopkAttnError("topk_attn_device_status", rc)
+    return int(bits.value)

@@ -1,0 +1,329 @@
+// C ABI entry points: argument checks, workspace layout and the launch
+// sequence of each operation.  Nothing here allocates or synchronises on the
+// compute path; every launch goes onto the caller's stream.
+#include <math.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace tka {
+namespace {
+
+__device__ unsigned int g_status = 0u;
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxK = 8192;
+constexpr int kMaxQ = 64;
+constexpr int kMaxRowsPerKvHead = 256;  // Q * G
+constexpr int kMaxLen = 1 << 24;
+constexpr int kMinKeysPerSplit = 64;
+
+struct DeviceInfo {
+    bool ready = false;
+    int num_sms = 0;
+    unsigned *status = nullptr;  // device address of g_status
+};
+DeviceInfo g_dev[kMaxDevices];
+
+// SM count and status-word address of the current device (looked up once).
+cudaError_t device_info(DeviceInfo **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    DeviceInfo &d = g_dev[dev];
+    if (!d.ready) {
+        e = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        e = cudaGetSymbolAddress(reinterpret_cast<void **>(&d.status), g_status);
+        if (e != cudaSuccess) return e;
+        d.ready = true;
+    }
+    *out = &d;
+    return cudaSuccess;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+cudaError_t record(const tka_event_t *events, int i, cudaStream_t s) {
+    if (!events || !events[i]) return cudaSuccess;
+    return cudaEventRecord(reinterpret_cast<cudaEvent_t>(events[i]), s);
+}
+
+float resolve_scale(const tka_shape *s) { return s->scale > 0.f ? s->scale : 1.f / sqrtf((float)s->d); }
+
+// Shape checks shared by both variants.
+tka_status check_shape(const tka_shape *s) {
+    if (!s) return TKA_ERR_INVALID_ARG;
+    if (s->B < 1 || s->Q < 1 || s->Hq < 1 || s->Hkv < 1 || s->d < 1 || s->L_max < 1) return TKA_ERR_INVALID_ARG;
+    if (s->Hq % s->Hkv) return TKA_ERR_INVALID_ARG;
+    if (!(s->scale >= 0.f) || isinf(s->scale)) return TKA_ERR_INVALID_ARG;
+    if (s->Q > s->L_max) return TKA_ERR_INVALID_ARG;
+    if (s->d != kHeadDim) return TKA_ERR_UNSUPPORTED;
+    if (s->dtype != TKA_F32 && s->dtype != TKA_BF16) return TKA_ERR_UNSUPPORTED;
+    if (s->Q > kMaxQ || s->L_max > kMaxLen) return TKA_ERR_UNSUPPORTED;
+    if ((long long)s->Q * (s->Hq / s->Hkv) > kMaxRowsPerKvHead) return TKA_ERR_UNSUPPORTED;
+    if ((long long)s->B * s->Hkv > 65535 || (long long)s->B * s->Q * s->Hq > 65535) return TKA_ERR_UNSUPPORTED;
+    return TKA_OK;
+}
+
+// Workspace of topk_attn_decode, in order, each region 256-byte aligned:
+//   scores   fp32 [rows, ld]          ld = L_max rounded up to 64
+//   weights  fp32 [rows, k]           e^{s - m} of the kept positions
+//   stats    float4 [rows]            {m, Z_k, Z_tail, 0}
+//   partial  fp32 [rows, max_splits, 128]
+//   counters uint32 [rows]
+struct TokenLayout {
+    size_t scores, weights, stats, partial, counters, total;
+    int ld, max_splits;
+};
+
+TokenLayout token_layout(const tka_shape *s, int k) {
+    TokenLayout L;
+    const size_t rows = (size_t)s->B * s->Q * s->Hq;
+    L.ld = (int)align_up((size_t)s->L_max, 64);
+    L.max_splits = (k + kMinKeysPerSplit - 1) / kMinKeysPerSplit;
+    size_t off = 0;
+    L.scores = off;
+    off = align_up(off + rows * L.ld * sizeof(float), 256);
+    L.weights = off;
+    off = align_up(off + rows * (size_t)k * sizeof(float), 256);
+    L.stats = off;
+    off = align_up(off + rows * sizeof(float4), 256);
+    L.partial = off;
+    off = align_up(off + rows * (size_t)L.max_splits * kHeadDim * sizeof(float), 256);
+    L.counters = off;
+    off = align_up(off + rows * sizeof(unsigned), 256);
+    L.total = off;
+    return L;
+}
+
+// Workspace of topk_block_attn_decode:
+//   block_idx int32 [rows, top+1]  (used when the caller passes none)
+//   part_ml   float4 [rows, top+1]
+//   part_acc  fp32 [rows, top+1, 128]
+//   counters  uint32 [rows]
+struct BlockLayout {
+    size_t block_idx, part_ml, part_acc, counters, total;
+};
+
+BlockLayout block_layout(const tka_shape *s, int top_blocks) {
+    BlockLayout L;
+    const size_t rows = (size_t)s->B * s->Hq, slots = (size_t)top_blocks + 1;
+    size_t off = 0;
+    L.block_idx = off;
+    off = align_up(off + rows * slots * sizeof(int32_t), 256);
+    L.part_ml = off;
+    off = align_up(off + rows * slots * sizeof(float4), 256);
+    L.part_acc = off;
+    off = align_up(off + rows * slots * kHeadDim * sizeof(float), 256);
+    L.counters = off;
+    off = align_up(off + rows * sizeof(unsigned), 256);
+    L.total = off;
+    return L;
+}
+
+tka_status check_block_args(const tka_shape *s, int block_size, int top_blocks) {
+    tka_status st = check_shape(s);
+    if (st != TKA_OK) return st;
+    if (block_size < 1 || top_blocks < 0) return TKA_ERR_INVALID_ARG;
+    if (block_size != 16 && block_size != 32 && block_size != 64 && block_size != 128) return TKA_ERR_UNSUPPORTED;
+    if (s->Q != 1 || top_blocks > 255) return TKA_ERR_UNSUPPORTED;
+    if ((s->L_max + block_size - 1) / block_size > 8192) return TKA_ERR_UNSUPPORTED;
+    return TKA_OK;
+}
+
+}  // namespace
+}  // namespace tka
+
+using namespace tka;
+
+extern "C" {
+
+size_t topk_attn_workspace_size(const tka_shape *shape, int32_t k) {
+    if (check_shape(shape) != TKA_OK || k < 1 || k > kMaxK) return 0;
+    return token_layout(shape, k).total;
+}
+
+tka_status topk_attn_decode_staged(const tka_shape *shape, const void *q, const void *k_cache,
+                                   const void *v_cache, const int32_t *seq_lens, int32_t k, float *out,
+                                   int32_t *idx, float *tail_mass, void *workspace, size_t workspace_bytes,
+                                   tka_stream_t stream, const tka_event_t events[4]) {
+    tka_status st = check_shape(shape);
+    if (st != TKA_OK) return st;
+    if (k < 1) return TKA_ERR_INVALID_ARG;
+    if (k > kMaxK) return TKA_ERR_UNSUPPORTED;
+    if (!q || !k_cache || !v_cache || !seq_lens || !out || !idx) return TKA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
+        !aligned(idx, 4) || !aligned(seq_lens, 4) || (tail_mass && !aligned(tail_mass, 4)))
+        return TKA_ERR_INVALID_ARG;
+    const TokenLayout L = token_layout(shape, k);
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < L.total) return TKA_ERR_WORKSPACE;
+    DeviceInfo *dev = nullptr;
+    if (device_info(&dev) != cudaSuccess) return TKA_ERR_CUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    char *ws = static_cast<char *>(workspace);
+    const int G = shape->Hq / shape->Hkv;
+    const int rows = shape->B * shape->Q * shape->Hq;
+
+    ScoreParams sp;
+    sp.status = dev->status;
+    sp.q = q;
+    sp.k = k_cache;
+    sp.seq_lens = seq_lens;
+    sp.scores = reinterpret_cast<float *>(ws + L.scores);
+    sp.B = shape->B; sp.Q = shape->Q; sp.Hq = shape->Hq; sp.Hkv = shape->Hkv; sp.G = G;
+    sp.L_max = shape->L_max; sp.ld = L.ld; sp.dtype = shape->dtype;
+    sp.scale = resolve_scale(shape);
+    if (record(events, 0, s) != cudaSuccess) return TKA_ERR_CUDA;
+    if (launch_score(sp, dev->num_sms, s) != cudaSuccess) return TKA_ERR_CUDA;
+    if (record(events, 1, s) != cudaSuccess) return TKA_ERR_CUDA;
+
+    SelectParams se;
+    se.status = dev->status;
+    se.scores = sp.scores;
+    se.seq_lens = seq_lens;
+    se.B = shape->B; se.Q = shape->Q; se.Hq = shape->Hq; se.L_max = shape->L_max; se.ld = L.ld; se.k = k;
+    se.idx = idx;
+    se.w = reinterpret_cast<float *>(ws + L.weights);
+    se.stats = reinterpret_cast<float4 *>(ws + L.stats);
+    se.tail = tail_mass;
+    se.counters = reinterpret_cast<unsigned *>(ws + L.counters);
+    if (launch_select(se, s) != cudaSuccess) return TKA_ERR_CUDA;
+    if (record(events, 2, s) != cudaSuccess) return TKA_ERR_CUDA;
+
+    GatherParams gp;
+    gp.status = dev->status;
+    gp.v = v_cache;
+    gp.seq_lens = seq_lens;
+    gp.B = shape->B; gp.Q = shape->Q; gp.Hq = shape->Hq; gp.Hkv = shape->Hkv; gp.G = G;
+    gp.L_max = shape->L_max; gp.k = k; gp.dtype = shape->dtype;
+    gp.idx = idx;
+    gp.w = se.w;
+    gp.stats = se.stats;
+    gp.partial = reinterpret_cast<float *>(ws + L.partial);
+    gp.counters = se.counters;
+    gp.out = out;
+    // about 8 CTAs per SM in total, never fewer than kMinKeysPerSplit keys per CTA
+    int splits = (dev->num_sms * 8 + rows - 1) / rows;
+    if (splits > L.max_splits) splits = L.max_splits;
+    if (splits < 1) splits = 1;
+    gp.per_split = (k + splits - 1) / splits;
+    gp.splits = (k + gp.per_split - 1) / gp.per_split;
+    if (launch_gather(gp, s) != cudaSuccess) return TKA_ERR_CUDA;
+    if (record(events, 3, s) != cudaSuccess) return TKA_ERR_CUDA;
+    return TKA_OK;
+}
+
+tka_status topk_attn_decode(const tka_shape *shape, const void *q, const void *k_cache, const void *v_cache,
+                            const int32_t *seq_lens, int32_t k, float *out, int32_t *idx, float *tail_mass,
+                            void *workspace, size_t workspace_bytes, tka_stream_t stream) {
+    return topk_attn_decode_staged(shape, q, k_cache, v_cache, seq_lens, k, out, idx, tail_mass, workspace,
+                                   workspace_bytes, stream, nullptr);
+}
+
+tka_status topk_block_pool_keys(const tka_shape *shape, const void *k_cache, const int32_t *seq_lens,
+                                int32_t block_size, float *block_keys, tka_stream_t stream) {
+    if (!shape) return TKA_ERR_INVALID_ARG;
+    if (shape->B < 1 || shape->Hkv < 1 || shape->L_max < 1 || block_size < 1) return TKA_ERR_INVALID_ARG;
+    if (shape->d != kHeadDim) return TKA_ERR_UNSUPPORTED;
+    if (shape->dtype != TKA_F32 && shape->dtype != TKA_BF16) return TKA_ERR_UNSUPPORTED;
+    if (shape->L_max > kMaxLen || (long long)shape->B * shape->Hkv > 65535) return TKA_ERR_UNSUPPORTED;
+    if (!k_cache || !seq_lens || !block_keys) return TKA_ERR_INVALID_ARG;
+    if (!aligned(k_cache, 16) || !aligned(block_keys, 16) || !aligned(seq_lens, 4)) return TKA_ERR_INVALID_ARG;
+    const int nblk_max = (shape->L_max + block_size - 1) / block_size;
+    if (nblk_max > (1 << 20)) return TKA_ERR_UNSUPPORTED;
+    DeviceInfo *dev = nullptr;
+    if (device_info(&dev) != cudaSuccess) return TKA_ERR_CUDA;
+    BlockPoolParams p;
+    p.status = dev->status;
+    p.k = k_cache;
+    p.seq_lens = seq_lens;
+    p.block_keys = block_keys;
+    p.B = shape->B; p.Hkv = shape->Hkv; p.L_max = shape->L_max; p.block_size = block_size;
+    p.nblk_max = nblk_max; p.dtype = shape->dtype;
+    if (launch_block_pool(p, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return TKA_ERR_CUDA;
+    return TKA_OK;
+}
+
+size_t topk_block_attn_workspace_size(const tka_shape *shape, int32_t block_size, int32_t top_blocks) {
+    if (check_block_args(shape, block_size, top_blocks) != TKA_OK) return 0;
+    return block_layout(shape, top_blocks).total;
+}
+
+tka_status topk_block_attn_decode(const tka_shape *shape, const void *q, const void *k_cache, const void *v_cache,
+                                  const float *block_keys, const int32_t *seq_lens, int32_t block_size,
+                                  int32_t top_blocks, float *out, int32_t *block_idx, void *workspace,
+                                  size_t workspace_bytes, tka_stream_t stream) {
+    tka_status st = check_block_args(shape, block_size, top_blocks);
+    if (st != TKA_OK) return st;
+    if (!q || !k_cache || !v_cache || !block_keys || !seq_lens || !out) return TKA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(block_keys, 16) ||
+        !aligned(out, 16) || !aligned(seq_lens, 4) || (block_idx && !aligned(block_idx, 4)))
+        return TKA_ERR_INVALID_ARG;
+    const BlockLayout L = block_layout(shape, top_blocks);
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < L.total) return TKA_ERR_WORKSPACE;
+    DeviceInfo *dev = nullptr;
+    if (device_info(&dev) != cudaSuccess) return TKA_ERR_CUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    char *ws = static_cast<char *>(workspace);
+    const int G = shape->Hq / shape->Hkv;
+    const int nblk_max = (shape->L_max + block_size - 1) / block_size;
+    int32_t *bidx = block_idx ? block_idx : reinterpret_cast<int32_t *>(ws + L.block_idx);
+    unsigned *counters = reinterpret_cast<unsigned *>(ws + L.counters);
+
+    BlockSelectParams sp;
+    sp.status = dev->status;
+    sp.q = q;
+    sp.block_keys = block_keys;
+    sp.seq_lens = seq_lens;
+    sp.B = shape->B; sp.Hq = shape->Hq; sp.Hkv = shape->Hkv; sp.G = G; sp.L_max = shape->L_max;
+    sp.block_size = block_size; sp.nblk_max = nblk_max; sp.top_blocks = top_blocks; sp.dtype = shape->dtype;
+    sp.scale = resolve_scale(shape);
+    sp.block_idx = bidx;
+    sp.counters = counters;
+    if (launch_block_select(sp, s) != cudaSuccess) return TKA_ERR_CUDA;
+
+    BlockAttnParams ap;
+    ap.status = dev->status;
+    ap.q = q; ap.k = k_cache; ap.v = v_cache;
+    ap.seq_lens = seq_lens;
+    ap.block_idx = bidx;
+    ap.B = shape->B; ap.Hq = shape->Hq; ap.Hkv = shape->Hkv; ap.G = G; ap.L_max = shape->L_max;
+    ap.block_size = block_size; ap.top_blocks = top_blocks; ap.dtype = shape->dtype;
+    ap.scale = sp.scale;
+    ap.part_ml = reinterpret_cast<float4 *>(ws + L.part_ml);
+    ap.part_acc = reinterpret_cast<float *>(ws + L.part_acc);
+    ap.counters = counters;
+    ap.out = out;
+    if (launch_block_attn(ap, s) != cudaSuccess) return TKA_ERR_CUDA;
+    return TKA_OK;
+}
+
+tka_status topk_attn_device_status(tka_stream_t stream, uint32_t *bits) {
+    if (!bits) return TKA_ERR_INVALID_ARG;
+    DeviceInfo *dev = nullptr;
+    if (device_info(&dev) != cudaSuccess) return TKA_ERR_CUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    unsigned v = 0u;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return TKA_ERR_CUDA;
+    if (cudaMemcpy(&v, dev->status, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return TKA_ERR_CUDA;
+    if (cudaMemset(dev->status, 0, sizeof v) != cudaSuccess) return TKA_ERR_CUDA;
+    *bits = v;
+    return TKA_OK;
+}
+
+const char *topk_attn_status_string(tka_status status) {
+    switch (status) {
+        case TKA_OK: return "TKA_OK";
+        case TKA_ERR_INVALID_ARG: return "TKA_ERR_INVALID_ARG";
+        case TKA_ERR_UNSUPPORTED: return "TKA_ERR_UNSUPPORTED";
+        case TKA_ERR_WORKSPACE: return "TKA_ERR_WORKSPACE";
+        case TKA_ERR_CUDA: return "TKA_ERR_CUDA";
+    }
+    return "unknown tka_status";
+}
+
+}  // extern "C"

@@ -1,0 +1,75 @@
+// Device helpers shared by the Top-k decode-attention kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/topk_attn.h"
+
+namespace tka {
+
+constexpr int kHeadDim = 128;
+
+// Kernels report problems they can only see on the device (TKA_DEV_* bits) by
+// OR-ing them into the library's per-device status word, whose address every
+// launch receives.
+__device__ __forceinline__ void raise_status(unsigned int *status, unsigned int bits) { atomicOr(status, bits); }
+
+// Rows are (b, qpos, h) in that order: row = (b * Q + qpos) * Hq + h.
+struct RowGeom {
+    int B, Q, Hq, Hkv, G, L_max;
+};
+
+// Visible keys of query position qpos in a chunk of Q queries ending at the
+// sequence's last position.
+__device__ __forceinline__ int visible_keys(int seq_len, int Q, int qpos) { return seq_len - Q + qpos + 1; }
+
+__device__ __forceinline__ bool seq_len_ok(int seq_len, int Q, int L_max) { return seq_len >= Q && seq_len <= L_max; }
+
+// Order-preserving map from fp32 to uint32: a > b (as floats, no NaN) iff
+// key(a) > key(b); -0.0 and +0.0 get distinct adjacent keys.
+__device__ __forceinline__ uint32_t order_key(float f) {
+    uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float bf16lo_to_f32(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi_to_f32(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+template <typename T>
+__device__ __forceinline__ T warp_sum(T v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// Block-wide sum/max of one value per thread (blockDim.x multiple of 32,
+// <= 1024).  `red` is >= 32 floats of shared memory; contains a barrier.
+__device__ __forceinline__ float block_sum(float v, float *red) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    v = warp_sum(v);
+    __syncthreads();
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    float t = lane < nw ? red[lane] : 0.f;
+    return warp_sum(t);
+}
+
+__device__ __forceinline__ float block_max(float v, float *red) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    v = warp_max(v);
+    __syncthreads();
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    float t = lane < nw ? red[lane] : -INFINITY;
+    return warp_max(t);
+}
+
+}  // namespace tka

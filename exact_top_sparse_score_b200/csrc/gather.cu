@@ -1,0 +1,153 @@
+// Attention step over the kept positions: out = sum_{i in S} (e^{s_i - m} / Z_k) V[i].
+//
+// "Sparse attention layers first read the KV entries corresponding to
+// positions selected by the Indexer" ("Sparse Attention in LLM Inference:
+// Practical Trade-Offs", section "Changes in Caching Strategy"): only the k
+// kept V rows are read, by position index.  The weights e^{s_i - m} and Z_k
+// come from the select step, so no K row is read again.
+//
+// Grid (splits, rows): each CTA gathers a contiguous slice of a row's kept
+// positions.  A V row is 256 bytes in bf16, read by 16 lanes with one 16-byte
+// load each (two rows per warp instruction); four rows per lane are in flight.
+// The slices of a row are summed by whichever CTA of the row finishes last
+// (an atomic ticket, no waiting), in slice order, so the result does not
+// depend on scheduling.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace tka {
+
+namespace {
+
+constexpr int kGatherThreads = 128;
+
+template <typename T>
+__global__ void __launch_bounds__(kGatherThreads) gather_pv(GatherParams p) {
+    constexpr int kPer = 16 / sizeof(T);              // elements per lane
+    constexpr int kLanesPerRow = kHeadDim / kPer;     // 16 (bf16) or 32 (fp32)
+    constexpr int kRowsPerWarp = 32 / kLanesPerRow;   // 2 or 1
+    constexpr int kSlots = (kGatherThreads / 32) * kRowsPerWarp;
+    __shared__ float red[kGatherThreads / 32][kHeadDim];
+    __shared__ unsigned s_ticket;
+
+    const int row = blockIdx.y, split = blockIdx.x;
+    const int b = row / (p.Q * p.Hq), qpos = (row / p.Hq) % p.Q, h = row % p.Hq;
+    const int seq_len = p.seq_lens[b];
+    if (!seq_len_ok(seq_len, p.Q, p.L_max)) return;  // the select step raised the status
+    const int vis = visible_keys(seq_len, p.Q, qpos);
+    const int kept = p.k < vis ? p.k : vis;
+    const int lo = split * p.per_split;
+    const int hi = min(kept, lo + p.per_split);
+
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int slot = warp * kRowsPerWarp + lane / kLanesPerRow;
+    const int c = lane % kLanesPerRow;  // this lane's 16-byte piece of a V row
+    const T *vbase = reinterpret_cast<const T *>(p.v) + ((size_t)b * p.Hkv + h / p.G) * p.L_max * kHeadDim +
+                     c * kPer;
+    const int32_t *idx = p.idx + (size_t)row * p.k;
+    const float *wv = p.w + (size_t)row * p.k;
+
+    float acc[kPer];
+#pragma unroll
+    for (int e = 0; e < kPer; e++) acc[e] = 0.f;
+    bool bad = false;
+
+    int j = lo + slot;
+    for (; j + 3 * kSlots < hi; j += 4 * kSlots) {
+        uint4 v[4];
+        float wt[4];
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+            int pos = __ldg(idx + j + u * kSlots);
+            wt[u] = __ldg(wv + j + u * kSlots);
+            if ((unsigned)pos >= (unsigned)vis) {  // never taken unless the select step is wrong
+                bad = true;
+                pos = 0;
+                wt[u] = 0.f;
+            }
+            v[u] = __ldg(reinterpret_cast<const uint4 *>(vbase + (size_t)pos * kHeadDim));
+        }
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+            const uint32_t wd[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+            if constexpr (sizeof(T) == 2) {
+#pragma unroll
+                for (int e = 0; e < 4; e++) {
+                    acc[2 * e] = fmaf(wt[u], bf16lo_to_f32(wd[e]), acc[2 * e]);
+                    acc[2 * e + 1] = fmaf(wt[u], bf16hi_to_f32(wd[e]), acc[2 * e + 1]);
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; e++) acc[e] = fmaf(wt[u], __uint_as_float(wd[e]), acc[e]);
+            }
+        }
+    }
+    for (; j < hi; j += kSlots) {
+        int pos = __ldg(idx + j);
+        float wt = __ldg(wv + j);
+        if ((unsigned)pos >= (unsigned)vis) {
+            bad = true;
+            pos = 0;
+            wt = 0.f;
+        }
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(vbase + (size_t)pos * kHeadDim));
+        const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+        if constexpr (sizeof(T) == 2) {
+#pragma unroll
+            for (int e = 0; e < 4; e++) {
+                acc[2 * e] = fmaf(wt, bf16lo_to_f32(wd[e]), acc[2 * e]);
+                acc[2 * e + 1] = fmaf(wt, bf16hi_to_f32(wd[e]), acc[2 * e + 1]);
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 4; e++) acc[e] = fmaf(wt, __uint_as_float(wd[e]), acc[e]);
+        }
+    }
+    if (bad) raise_status(p.status, TKA_DEV_INTERNAL);
+    // sum the rows of a warp, then the warps of the CTA
+    if constexpr (kRowsPerWarp == 2) {
+#pragma unroll
+        for (int e = 0; e < kPer; e++) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
+    }
+    if (lane < kLanesPerRow) {
+#pragma unroll
+        for (int e = 0; e < kPer; e++) red[warp][c * kPer + e] = acc[e];
+    }
+    __syncthreads();
+    const int d = threadIdx.x;  // one output dim per thread (128 threads)
+    float sum = 0.f;
+#pragma unroll
+    for (int w = 0; w < kGatherThreads / 32; w++) sum += red[w][d];
+    const float inv_zk = 1.f / p.stats[row].y;
+    float *out = p.out + (size_t)row * kHeadDim;
+    if (p.splits == 1) {
+        out[d] = sum * inv_zk;
+        return;
+    }
+    float *part = p.partial + (size_t)row * p.splits * kHeadDim;
+    part[(size_t)split * kHeadDim + d] = sum;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_ticket = atomicAdd(&p.counters[row], 1u);
+    __syncthreads();
+    if (s_ticket != (unsigned)p.splits - 1) return;
+    __threadfence();
+    float total = 0.f;
+    for (int sp = 0; sp < p.splits; sp++) total += __ldcg(part + (size_t)sp * kHeadDim + d);
+    out[d] = total * inv_zk;
+    if (threadIdx.x == 0) p.counters[row] = 0u;
+}
+
+}  // namespace
+
+cudaError_t launch_gather(const GatherParams &p, cudaStream_t stream) {
+    const int rows = p.B * p.Q * p.Hq;
+    const dim3 grid(p.splits, rows);
+    if (p.dtype == TKA_BF16)
+        gather_pv<__nv_bfloat16><<<grid, kGatherThreads, 0, stream>>>(p);
+    else
+        gather_pv<float><<<grid, kGatherThreads, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace tka

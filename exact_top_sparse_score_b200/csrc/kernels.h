@@ -1,0 +1,84 @@
+// Launch interfaces of the Top-k decode-attention kernels (internal).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace tka {
+
+struct ScoreParams {
+    unsigned *status;         // device status word (TKA_DEV_* bits)
+    const void *q;            // [B, Q, Hq, 128]
+    const void *k;            // [B, Hkv, L_max, 128]
+    const int32_t *seq_lens;  // [B]
+    float *scores;            // [B*Q*Hq, ld]
+    int B, Q, Hq, Hkv, G, L_max, ld, dtype;
+    float scale;
+};
+
+struct SelectParams {
+    unsigned *status;         // device status word (TKA_DEV_* bits)
+    const float *scores;      // [rows, ld]
+    const int32_t *seq_lens;
+    int B, Q, Hq, L_max, ld, k;
+    int32_t *idx;             // [rows, k] ascending, -1 padded
+    float *w;                 // [rows, k] e^{s_i - m} of the kept positions
+    float4 *stats;            // [rows] {m, Z_k, Z_tail, 0}
+    float *tail;              // [rows] or null
+    unsigned *counters;       // [rows], zeroed here for the combine step
+};
+
+struct GatherParams {
+    unsigned *status;         // device status word (TKA_DEV_* bits)
+    const void *v;            // [B, Hkv, L_max, 128]
+    const int32_t *seq_lens;
+    int B, Q, Hq, Hkv, G, L_max, k, dtype;
+    const int32_t *idx;       // [rows, k]
+    const float *w;           // [rows, k]
+    const float4 *stats;      // [rows]
+    float *partial;           // [rows, splits, 128]
+    unsigned *counters;       // [rows]
+    float *out;               // [rows, 128]
+    int splits, per_split;
+};
+
+struct BlockPoolParams {
+    unsigned *status;         // device status word (TKA_DEV_* bits)
+    const void *k;
+    const int32_t *seq_lens;
+    float *block_keys;        // [B, Hkv, nblk_max, 128]
+    int B, Hkv, L_max, block_size, nblk_max, dtype;
+};
+
+struct BlockSelectParams {
+    unsigned *status;         // device status word (TKA_DEV_* bits)
+    const void *q;            // [B, 1, Hq, 128]
+    const float *block_keys;  // [B, Hkv, nblk_max, 128]
+    const int32_t *seq_lens;
+    int B, Hq, Hkv, G, L_max, block_size, nblk_max, top_blocks, dtype;
+    float scale;
+    int32_t *block_idx;       // [B*Hq, top_blocks + 1] (workspace or caller's)
+    unsigned *counters;       // [B*Hq], zeroed here for the attention step
+};
+
+struct BlockAttnParams {
+    unsigned *status;         // device status word (TKA_DEV_* bits)
+    const void *q, *k, *v;
+    const int32_t *seq_lens;
+    const int32_t *block_idx; // [rows, top_blocks + 1]
+    int B, Hq, Hkv, G, L_max, block_size, top_blocks, dtype;
+    float scale;
+    float4 *part_ml;          // [rows, top_blocks + 1] {m, l}
+    float *part_acc;          // [rows, top_blocks + 1, 128]
+    unsigned *counters;       // [rows]
+    float *out;               // [rows, 128]
+};
+
+cudaError_t launch_score(const ScoreParams &p, int num_sms, cudaStream_t stream);
+cudaError_t launch_select(const SelectParams &p, cudaStream_t stream);
+cudaError_t launch_gather(const GatherParams &p, cudaStream_t stream);
+cudaError_t launch_block_pool(const BlockPoolParams &p, cudaStream_t stream);
+cudaError_t launch_block_select(const BlockSelectParams &p, cudaStream_t stream);
+cudaError_t launch_block_attn(const BlockAttnParams &p, cudaStream_t stream);
+
+}  // namespace tka

@@ -1,0 +1,146 @@
+/*
+ * topk_attn.h -- C ABI of the B200 exact Top-k sparse decode-attention library.
+ *
+ * The operation ("A Preliminary Study on the Promises and Challenges of Native
+ * Top-k Sparse Attention", abstract: exact Top-k decoding keeps only the keys
+ * most similar to the query; "Sparse Attention in LLM Inference: Practical
+ * Trade-Offs", section "The Role of the Indexer": score every historical
+ * position, keep the Top-K, attend only to those):
+ *
+ *   for every query row (b, qpos, h), with G = Hq / Hkv and kv-head h / G,
+ *     vis   = seq_lens[b] - Q + qpos + 1                   (causal visibility)
+ *     s_i   = scale * <q[b,qpos,h,:], K[b,h/G,i,:]>        for i < vis
+ *     S     = the min(k, vis) positions with the highest s_i, ties to the lower i
+ *     out   = sum_{i in S} softmax_S(s)_i * V[b,h/G,i,:]
+ *     tail  = sum_{i not in S} softmax(s)_i                (discarded softmax mass;
+ *             "A Mathematical Theory of Top-k Sparse Attention via Total
+ *             Variation Distance", abstract: equals TV(P, P_hat))
+ *
+ * and a block-sparse variant (MoBA, "Sparse Attention Landscape", section
+ * "Block Sparse Attention"): blocks of `block_size` keys are scored by
+ * <q, mean of the block's keys>, the best `top_blocks` blocks other than the
+ * last are kept together with the last (current) block, and dense softmax
+ * attention runs over the kept blocks' keys.
+ *
+ * Conventions shared by every entry point:
+ *   - Every data pointer is DEVICE memory owned by the caller.  The library
+ *     never allocates, frees or synchronises inside a compute call; it only
+ *     enqueues kernels on `stream` (a cudaStream_t; NULL = legacy default).
+ *   - Layouts are row-major and contiguous:
+ *       q         [B, Q, Hq, d]        dtype of the cache
+ *       k_cache   [B, Hkv, L_max, d]   bf16 or fp32
+ *       v_cache   [B, Hkv, L_max, d]   same dtype as k_cache
+ *       seq_lens  int32 [B]            valid keys per sequence, Q <= seq_lens[b] <= L_max
+ *       out       fp32 [B, Q, Hq, d]
+ *       idx       int32 [B, Q, Hq, k]  kept positions, ascending, -1 padded when vis < k
+ *       tail_mass fp32 [B, Q, Hq]
+ *     q, k_cache, v_cache and out must be 16-byte aligned, the workspace
+ *     256-byte aligned.
+ *     Cache rows at positions >= seq_lens[b] are never read.
+ *   - Arguments are checked on the host before anything is launched; a bad
+ *     argument returns an error code and launches nothing.  seq_lens lives on
+ *     the device, so its values are checked by the kernels: a sequence whose
+ *     length is out of range is skipped (its outputs are left untouched) and
+ *     TKA_DEV_BAD_SEQ_LEN is raised in the device status word, readable with
+ *     topk_attn_device_status().
+ *   - Supported: d = 128, dtype bf16 or fp32, Hq % Hkv == 0, 1 <= k <= 8192,
+ *     Q <= 64.  Anything else returns TKA_ERR_UNSUPPORTED.
+ */
+#ifndef TOPK_ATTN_H
+#define TOPK_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    TKA_OK = 0,
+    TKA_ERR_INVALID_ARG = 1, /* null pointer, misaligned pointer, non-positive size */
+    TKA_ERR_UNSUPPORTED = 2, /* valid but outside the supported set above */
+    TKA_ERR_WORKSPACE = 3,   /* workspace pointer missing or smaller than required */
+    TKA_ERR_CUDA = 4         /* a launch or CUDA runtime call failed */
+} tka_status;
+
+typedef enum { TKA_F32 = 0, TKA_BF16 = 1 } tka_dtype;
+
+/* Bits of the device status word (OR-ed by kernels, cleared by reading). */
+#define TKA_DEV_BAD_SEQ_LEN 0x1u /* a seq_lens value was out of range; that sequence was skipped */
+#define TKA_DEV_INTERNAL 0x2u    /* an internal consistency check failed (a library bug) */
+
+/* cudaStream_t without pulling in the CUDA headers. */
+typedef struct CUstream_st *tka_stream_t;
+
+typedef struct {
+    int32_t B;      /* sequences */
+    int32_t Q;      /* query positions per sequence (1 for plain decode) */
+    int32_t Hq;     /* query heads */
+    int32_t Hkv;    /* key/value heads; Hq % Hkv == 0 */
+    int32_t d;      /* head dimension (128) */
+    int32_t L_max;  /* cache capacity per sequence */
+    int32_t dtype;  /* tka_dtype of q, k_cache and v_cache */
+    float scale;    /* score scale; 0 means 1/sqrt(d) */
+} tka_shape;
+
+/* Bytes of scratch topk_attn_decode needs for this shape and k (0 on a bad
+ * shape).  The caller allocates it once and may reuse it for every call with
+ * the same or a smaller shape; calls sharing one workspace must not overlap. */
+size_t topk_attn_workspace_size(const tka_shape *shape, int32_t k);
+
+/* Exact Top-k decode attention for all B*Q*Hq query rows (see top of file).
+ * idx is required; tail_mass may be NULL. */
+tka_status topk_attn_decode(const tka_shape *shape, const void *q, const void *k_cache,
+                            const void *v_cache, const int32_t *seq_lens, int32_t k, float *out,
+                            int32_t *idx, float *tail_mass, void *workspace, size_t workspace_bytes,
+                            tka_stream_t stream);
+
+/* Same as topk_attn_decode, and additionally records the caller's CUDA events
+ * (cudaEvent_t, created by the caller) on `stream` around the three kernels:
+ * events[0] before the score kernel, events[1] between score and select,
+ * events[2] between select and gather, events[3] after gather.  Used to time
+ * each step inside a benchmark without changing what runs. */
+typedef struct CUevent_st *tka_event_t;
+tka_status topk_attn_decode_staged(const tka_shape *shape, const void *q, const void *k_cache,
+                                   const void *v_cache, const int32_t *seq_lens, int32_t k, float *out,
+                                   int32_t *idx, float *tail_mass, void *workspace, size_t workspace_bytes,
+                                   tka_stream_t stream, const tka_event_t events[4]);
+
+/* MoBA block keys: block_keys[b, h, j, :] = mean of K[b, h, i, :] over the keys
+ * of block j below seq_lens[b] (a partial last block is averaged over the keys
+ * it holds; blocks past the end are written as zero).  block_keys is fp32
+ * [B, Hkv, ceil(L_max / block_size), d].  Only shape->B, Hkv, d, L_max and
+ * dtype are used.  Called when blocks change, not once per decode step. */
+tka_status topk_block_pool_keys(const tka_shape *shape, const void *k_cache, const int32_t *seq_lens,
+                                int32_t block_size, float *block_keys, tka_stream_t stream);
+
+/* Bytes of scratch topk_block_attn_decode needs (0 on a bad shape). */
+size_t topk_block_attn_workspace_size(const tka_shape *shape, int32_t block_size, int32_t top_blocks);
+
+/* Block-sparse (MoBA) decode attention, one query position per sequence
+ * (shape->Q == 1).  With nblk = ceil(seq_lens[b] / block_size), the blocks
+ * j < nblk - 1 compete on r_j = scale * <q, block_keys[b, h/G, j, :]>; the
+ * best top_blocks of them (ties to the lower j) and block nblk - 1 are kept,
+ * and out is dense softmax attention over their keys below seq_lens[b].
+ * block_idx (nullable) is int32 [B, 1, Hq, top_blocks + 1], ascending, -1
+ * padded.  Supported: block_size in {16, 32, 64, 128}, 0 <= top_blocks <= 255,
+ * ceil(L_max / block_size) <= 8192. */
+tka_status topk_block_attn_decode(const tka_shape *shape, const void *q, const void *k_cache,
+                                  const void *v_cache, const float *block_keys,
+                                  const int32_t *seq_lens, int32_t block_size, int32_t top_blocks,
+                                  float *out, int32_t *block_idx, void *workspace,
+                                  size_t workspace_bytes, tka_stream_t stream);
+
+/* Synchronises `stream`, returns the device status word of the current device
+ * (TKA_DEV_* bits raised by kernels since the last read) in *bits and clears it. */
+tka_status topk_attn_device_status(tka_stream_t stream, uint32_t *bits);
+
+/* Human-readable name of a status code. */
+const char *topk_attn_status_string(tka_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TOPK_ATTN_H */

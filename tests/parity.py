@@ -1,0 +1,128 @@
+"""Comparison of the CUDA path with the fp64 oracle.
+
+Agreement required:
+  * kept index sets equal, except for positions whose oracle score lies within
+    BAND = 1e-3 of the oracle's k-th (smallest kept) score: near-ties that fp32
+    scoring may order either way.  Rows whose sets differ inside the band are
+    checked for validity instead: their out and tail must match an fp64
+    evaluation over the GPU's own kept set.
+  * out within 2e-2 absolute or 1e-2 relative for bf16 inputs, 1e-4 for fp32;
+  * tail mass within 1e-3 absolute.
+"""
+import math
+
+import numpy as np
+import torch
+
+import oracle
+
+BAND = 1e-3
+TAIL_TOL = 1e-3
+
+
+def out_tol(dtype):
+    return (2e-2, 1e-2) if dtype == "bf16" else (1e-4, 1e-4)
+
+
+def to_device(w, device="cuda:0"):
+    return (w.q.to(device), w.k_cache.to(device), w.v_cache.to(device), w.seq_lens.to(device))
+
+
+def _close(got, want, atol, rtol):
+    return np.abs(got - want) <= atol + rtol * np.abs(want)
+
+
+def _vis(w, b, qp):
+    return int(w.seq_lens[b]) - w.Q + qp + 1
+
+
+def _set_eval(w, s, sel, b, h):
+    """fp64 out and tail over a given kept set (validity check of a tie-band row)."""
+    m = s.max()
+    e = np.exp(s - m)
+    zk = e[sel].sum()
+    V = w.v_cache[b, h // w.G].double().numpy()[sel]
+    return (e[sel, None] * V).sum(0) / zk, 1.0 - zk / e.sum()
+
+
+def check_token(w, k, out, idx, tail, ref, scale=0.0, rows_checked=None):
+    """Asserts parity of topk_attn_decode outputs with oracle.topk_attn output `ref`.
+
+    rows_checked: optional list of (b, qpos, h) to restrict to (sampled full-size checks;
+    `ref` then holds only those rows, in that order)."""
+    out = out.detach().cpu().double().numpy()
+    idx = idx.detach().cpu().numpy()
+    tail = tail.detach().cpu().double().numpy() if tail is not None else None
+    atol, rtol = out_tol(w.dtype)
+    rows = rows_checked or [(b, qp, h) for b in range(w.B) for qp in range(w.Q) for h in range(w.Hq)]
+    n_band = 0
+    for r_i, (b, qp, h) in enumerate(rows):
+        g = idx[b, qp, h]
+        if rows_checked:
+            o, ro, rt, kth = ref["idx"][r_i], ref["out"][r_i], ref["tail"][r_i], ref["kth"][r_i]
+        else:
+            o, ro, rt, kth = ref["idx"][b, qp, h], ref["out"][b, qp, h], ref["tail"][b, qp, h], ref["kth"][b, qp, h]
+        vis = _vis(w, b, qp)
+        kk = min(k, vis)
+        where = f"row (b={b}, q={qp}, h={h})"
+        assert np.all(g[kk:] == -1), f"{where}: padding"
+        gs = g[:kk]
+        assert np.all(gs >= 0) and np.all(gs < vis), f"{where}: position out of range"
+        assert np.all(np.diff(gs) > 0), f"{where}: not strictly ascending"
+        if np.array_equal(gs, o[:kk]):
+            ok = _close(out[b, qp, h], ro, atol, rtol)
+            assert ok.all(), f"{where}: out max |diff| {np.abs(out[b, qp, h] - ro).max():.3e}"
+            if tail is not None:
+                assert abs(tail[b, qp, h] - rt) <= TAIL_TOL, f"{where}: tail {tail[b, qp, h]} vs {rt}"
+            continue
+        n_band += 1
+        s = oracle.row_scores(w, b, qp, h, scale)
+        diff = np.setxor1d(gs, o[:kk])
+        assert np.all(np.abs(s[diff] - kth) <= BAND), \
+            f"{where}: set differs outside the tie band (max {np.abs(s[diff] - kth).max():.3e})"
+        vo, vt = _set_eval(w, s, gs, b, h)
+        assert _close(out[b, qp, h], vo, atol, rtol).all(), f"{where}: out invalid for its own set"
+        if tail is not None:
+            assert abs(tail[b, qp, h] - vt) <= TAIL_TOL, f"{where}: tail invalid for its own set"
+    return n_band
+
+
+def oracle_block_scores(w, bk, b, h, scale=0.0):
+    sc = scale if scale > 0 else 1.0 / math.sqrt(w.d)
+    return bk[b, h // w.G] @ w.q[b, 0, h].double().numpy() * sc
+
+
+def check_block(w, block_size, top_blocks, out, bidx, ref, scale=0.0):
+    out = out.detach().cpu().double().numpy()
+    bidx = bidx.detach().cpu().numpy()
+    atol, rtol = out_tol(w.dtype)
+    bk = None
+    n_band = 0
+    for b in range(w.B):
+        Lb = int(w.seq_lens[b])
+        nblk = -(-Lb // block_size)
+        nk = min(top_blocks, nblk - 1) + 1
+        for h in range(w.Hq):
+            where = f"row (b={b}, h={h})"
+            g, o = bidx[b, 0, h], ref["block_idx"][b, 0, h]
+            assert np.all(g[nk:] == -1), f"{where}: padding"
+            gs = g[:nk]
+            assert np.all(np.diff(gs) > 0) and gs[-1] == nblk - 1 and gs[0] >= 0, f"{where}: block list"
+            if np.array_equal(gs, o[:nk]):
+                ok = _close(out[b, 0, h], ref["out"][b, 0, h], atol, rtol)
+                assert ok.all(), f"{where}: out max |diff| {np.abs(out[b, 0, h] - ref['out'][b, 0, h]).max():.3e}"
+                continue
+            n_band += 1
+            if bk is None:
+                bk = oracle.block_pool(w, block_size)
+            r = oracle_block_scores(w, bk, b, h, scale)
+            diff = np.setxor1d(gs, o[:nk])
+            assert np.all(np.abs(r[diff] - ref["kth"][b, 0, h]) <= BAND), f"{where}: block set outside tie band"
+            # validity: dense attention over the GPU's kept blocks
+            s = oracle.row_scores(w, b, 0, h, scale)
+            sel = np.concatenate([np.arange(j * block_size, min(j * block_size + block_size, Lb)) for j in gs])
+            e = np.exp(s[sel] - s[sel].max())
+            V = w.v_cache[b, h // w.G].double().numpy()[sel]
+            want = (e[:, None] * V).sum(0) / e.sum()
+            assert _close(out[b, 0, h], want, atol, rtol).all(), f"{where}: out invalid for its own blocks"
+    return n_band

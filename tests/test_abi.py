@@ -1,0 +1,108 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry point
+that include/topk_attn.h declares, sizes workspaces, and rejects bad
+arguments on the host before launching anything (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_top_sparse_score_b200 import _binding as bd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "topk_attn.h")
+
+OK, INVALID, UNSUPPORTED, WORKSPACE = 0, 1, 2, 3
+FAKE = 1 << 20  # a non-null, 256-byte aligned address that is never dereferenced on error paths
+
+
+def declared_functions():
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    return sorted(set(re.findall(r"\b(topk_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from exact_top_sparse_score_b200.build import build
+    build()
+    return bd.load_library()
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ["topk_attn_decode", "topk_attn_workspace_size", "topk_block_attn_decode",
+              "topk_block_pool_keys", "topk_block_attn_workspace_size", "topk_attn_device_status",
+              "topk_attn_status_string"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    assert lib.topk_attn_status_string(0) == b"TKA_OK"
+    assert lib.topk_attn_status_string(3) == b"TKA_ERR_WORKSPACE"
+
+
+def shape(B=2, Q=1, Hq=8, Hkv=2, d=128, L=1000, dtype=1, scale=0.0):
+    return bd.tka_shape(B, Q, Hq, Hkv, d, L, dtype, scale)
+
+
+def test_workspace_size_layout(lib):
+    s = shape(B=8, Q=1, Hq=32, Hkv=8, L=32768)
+    n = bd.topk_attn_workspace_size(s, 2048)
+    rows = 8 * 32
+    # scores + weights + stats + partial (32 splits of 64 keys) + counters
+    want = rows * 32768 * 4 + rows * 2048 * 4 + rows * 16 + rows * 32 * 128 * 4 + 1024
+    assert n == want
+    assert bd.topk_attn_workspace_size(shape(L=1001), 7) % 256 == 0
+
+
+@pytest.mark.parametrize("kw,k", [(dict(d=64), 8), (dict(dtype=5), 8), (dict(Q=65, L=100), 8),
+                                  (dict(Hq=8, Hkv=3), 8), (dict(B=0), 8), (dict(), 0), (dict(), 8193),
+                                  (dict(scale=-1.0), 8), (dict(Q=5, L=4), 2)])
+def test_workspace_size_zero_on_bad_shape(lib, kw, k):
+    assert bd.topk_attn_workspace_size(shape(**kw), k) == 0
+
+
+def call_decode(lib, s, k=8, q=FAKE, kc=FAKE, vc=FAKE, lens=FAKE, out=FAKE, idx=FAKE, tail=FAKE, ws=FAKE,
+                nbytes=None):
+    if nbytes is None:
+        nbytes = bd.topk_attn_workspace_size(s, k) if bd.topk_attn_workspace_size(s, k) else 1 << 40
+    return lib.topk_attn_decode(ctypes.byref(s), q, kc, vc, lens, k, out, idx, tail, ws, nbytes, None)
+
+
+def test_decode_rejects_bad_arguments_before_launch(lib):
+    s = shape()
+    assert call_decode(lib, s, k=0) == INVALID
+    assert call_decode(lib, s, k=9000) == UNSUPPORTED
+    assert call_decode(lib, s, q=None) == INVALID
+    assert call_decode(lib, s, idx=None) == INVALID
+    assert call_decode(lib, s, kc=FAKE + 8) == INVALID          # misaligned
+    assert call_decode(lib, s, ws=None) == WORKSPACE
+    assert call_decode(lib, s, ws=FAKE + 16) == WORKSPACE       # workspace not 256-byte aligned
+    assert call_decode(lib, s, nbytes=bd.topk_attn_workspace_size(s, 8) - 1) == WORKSPACE
+    assert call_decode(lib, shape(d=64)) == UNSUPPORTED
+    assert call_decode(lib, shape(Hkv=3)) == INVALID
+    assert call_decode(lib, shape(dtype=2)) == UNSUPPORTED
+    assert lib.topk_attn_decode(None, FAKE, FAKE, FAKE, FAKE, 8, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == INVALID
+
+
+def test_block_decode_rejects_bad_arguments_before_launch(lib):
+    def call(s, bs=64, top=16, bk=FAKE, nbytes=None):
+        if nbytes is None:
+            nbytes = bd.block_attn_workspace_size(s, bs, top) or (1 << 40)
+        return lib.topk_block_attn_decode(ctypes.byref(s), FAKE, FAKE, FAKE, bk, FAKE, bs, top, FAKE, FAKE,
+                                          FAKE, nbytes, None)
+    s = shape(L=65536)
+    assert call(s, bs=48) == UNSUPPORTED
+    assert call(s, top=-1) == INVALID
+    assert call(s, top=256) == UNSUPPORTED
+    assert call(shape(Q=2, L=65536)) == UNSUPPORTED
+    assert call(shape(L=65536 * 4), bs=16) == UNSUPPORTED          # 16384 blocks > 8192
+    assert call(s, bk=None) == INVALID
+    assert call(s, nbytes=16) == WORKSPACE
+    assert lib.topk_block_pool_keys(ctypes.byref(s), FAKE, FAKE, 0, FAKE, None) == INVALID
+    assert lib.topk_block_pool_keys(ctypes.byref(shape(d=96)), FAKE, FAKE, 64, FAKE, None) == UNSUPPORTED

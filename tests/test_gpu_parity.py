@@ -1,0 +1,150 @@
+"""CUDA path vs the fp64 oracle, through the C ABI (ctypes binding).
+
+Small cases span several score chunks, ragged tails, every query-tile width
+of the tensor-core scorer (Q*G = 4, 16, 32, 64) and the CUDA-core scorer
+(fp32, and bf16 with Q*G > 64); edge cases cover k > visible keys, k = 1,
+k = visible keys, one-key sequences, exact ties, the largest k, NaN-poisoned
+cache rows past the sequence end, and an out-of-range sequence length.
+"""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from parity import check_block, check_token, to_device
+
+import exact_top_sparse_score_b200 as tka
+
+pytestmark = pytest.mark.gpu
+
+
+def _seed(case):
+    return zlib.crc32(repr(case).encode()) % 100000
+
+
+def run_token(w, k, scale=0.0):
+    q, kc, vc, lens = to_device(w)
+    out, idx, tail = tka.topk_attn_decode(q, kc, vc, lens, k, scale=scale)
+    torch.cuda.synchronize()
+    assert tka.topk_attn_device_status() == 0
+    return out, idx, tail
+
+
+TOKEN_CASES = [
+    # dtype, B, Q, Hq, Hkv, L_max, seq_lens, k
+    ("bf16", 2, 1, 8, 2, 1000, [1000, 517], 100),      # ragged tail, Q*G = 4
+    ("bf16", 2, 1, 32, 8, 4133, [4133, 3001], 512),    # Llama-3-8B head layout
+    ("bf16", 2, 2, 16, 2, 600, [600, 301], 40),        # Q*G = 16
+    ("bf16", 1, 4, 16, 2, 1500, None, 64),             # Q*G = 32
+    ("bf16", 2, 16, 32, 8, 2500, [2500, 2000], 300),   # Q*G = 64, causal chunk
+    ("bf16", 1, 8, 32, 2, 900, None, 50),              # Q*G = 128: CUDA-core scorer
+    ("f32", 2, 3, 8, 4, 777, [777, 200], 50),          # fp32, causal
+    ("f32", 1, 1, 4, 4, 3000, None, 1),                # k = 1
+    ("bf16", 2, 1, 8, 2, 300, [300, 50], 100),         # k > visible keys for b=1
+    ("bf16", 2, 1, 4, 1, 64, [1, 64], 8),              # one-key sequence
+    ("bf16", 1, 1, 8, 2, 256, None, 256),              # k = visible keys
+    ("bf16", 1, 1, 8, 8, 10000, None, 8192),           # largest k
+    ("bf16", 1, 3, 4, 4, 700, None, 30),               # G = 1 (multi-head), Q = 3
+]
+
+
+@pytest.mark.parametrize("case", TOKEN_CASES, ids=lambda c: "-".join(map(str, c[:6])) + f"-k{c[7]}")
+def test_token_parity_small(case, cuda_device):
+    dtype, B, Q, Hq, Hkv, L, lens, k = case
+    w = workloads.make_workload(B, Q, Hq, Hkv, L, dtype=dtype, seq_lens=lens, k_mean_std=0.5, seed=_seed(case))
+    out, idx, tail = run_token(w, k)
+    assert torch.isfinite(out).all() and torch.isfinite(tail).all()
+    check_token(w, k, out, idx, tail, oracle.topk_attn(w, k))
+
+
+def test_token_explicit_scale(cuda_device):
+    w = workloads.make_workload(2, 1, 8, 2, 800, dtype="bf16", seed=3)
+    out, idx, tail = run_token(w, 64, scale=0.3)
+    check_token(w, 64, out, idx, tail, oracle.topk_attn(w, 64, scale=0.3), scale=0.3)
+
+
+def test_token_exact_ties_go_to_lower_position(cuda_device):
+    # many duplicated key rows: exactly equal scores on both sides
+    w = workloads.make_workload(1, 1, 8, 2, 2048, dtype="bf16", seed=4)
+    src = torch.arange(2048) % 97
+    w.k_cache[:] = w.k_cache[:, :, src]
+    out, idx, tail = run_token(w, 200)
+    ref = oracle.topk_attn(w, 200)
+    assert np.array_equal(idx.cpu().numpy(), ref["idx"])
+    check_token(w, 200, out, idx, tail, ref)
+
+
+def test_planted_heavy_tail(cuda_device):
+    w = workloads.make_workload(2, 1, 32, 8, 5000, dtype="bf16", seq_len_range=(2500, 5000), plant_count=16,
+                                seed=5)
+    out, idx, tail = run_token(w, 256)
+    check_token(w, 256, out, idx, tail, oracle.topk_attn(w, 256))
+
+
+def test_repeat_calls_are_bitwise_identical(cuda_device):
+    w = workloads.make_workload(2, 1, 32, 8, 3000, dtype="bf16", seed=6)
+    q, kc, vc, lens = to_device(w)
+    ws = torch.empty(tka.topk_attn_workspace_size(tka._binding.make_shape(q, kc), 300), dtype=torch.uint8,
+                     device="cuda")
+    a = tka.topk_attn_decode(q, kc, vc, lens, 300, workspace=ws)
+    a = [t.clone() for t in a]
+    b = tka.topk_attn_decode(q, kc, vc, lens, 300, workspace=ws)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_non_default_stream(cuda_device):
+    w = workloads.make_workload(1, 1, 8, 2, 1200, dtype="bf16", seed=7)
+    q, kc, vc, lens = to_device(w)
+    st = torch.cuda.Stream()
+    st.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(st):
+        out, idx, tail = tka.topk_attn_decode(q, kc, vc, lens, 100)
+    st.synchronize()
+    check_token(w, 100, out, idx, tail, oracle.topk_attn(w, 100))
+
+
+def test_bad_seq_len_raises_status_and_skips_sequence(cuda_device):
+    w = workloads.make_workload(2, 1, 8, 2, 500, dtype="bf16", seed=8)
+    q, kc, vc, lens = to_device(w)
+    bad = lens.clone()
+    bad[1] = 501  # > L_max
+    out = torch.full((2, 1, 8, 128), 7.0, device="cuda")
+    idx = torch.full((2, 1, 8, 40), -7, dtype=torch.int32, device="cuda")
+    tail = torch.full((2, 1, 8), 7.0, device="cuda")
+    tka.topk_attn_device_status()
+    tka.topk_attn_decode(q, kc, vc, bad, 40, out=out, idx=idx, tail_mass=tail)
+    assert tka.topk_attn_device_status() & tka.DEV_BAD_SEQ_LEN
+    assert tka.topk_attn_device_status() == 0  # cleared by reading
+    assert (out[1] == 7.0).all() and (idx[1] == -7).all() and (tail[1] == 7.0).all()
+    ref = oracle.topk_attn(w, 40)
+    w1 = workloads.make_workload(1, 1, 8, 2, 500, dtype="bf16", seed=8)
+    check_token(w1, 40, out[:1], idx[:1], tail[:1], {k: v[:1] for k, v in ref.items()})
+
+
+BLOCK_CASES = [
+    # dtype, B, Hq, Hkv, L_max, seq_lens, block_size, top_blocks
+    ("bf16", 2, 8, 2, 4096, [4096, 3000], 64, 16),
+    ("bf16", 2, 32, 8, 2000, [2000, 1111], 32, 5),
+    ("f32", 2, 8, 4, 1024, [1024, 70], 16, 7),
+    ("bf16", 1, 4, 1, 640, None, 128, 2),
+    ("bf16", 2, 8, 2, 700, [700, 64], 64, 30),          # top_blocks >= competing blocks: dense
+    ("bf16", 1, 8, 2, 256, [1], 64, 4),                 # one-key sequence
+]
+
+
+@pytest.mark.parametrize("case", BLOCK_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_block_parity_small(case, cuda_device):
+    dtype, B, Hq, Hkv, L, lens, bs, top = case
+    w = workloads.make_workload(B, 1, Hq, Hkv, L, dtype=dtype, seq_lens=lens, seed=_seed(case))
+    q, kc, vc, lens_d = to_device(w)
+    bk = tka.topk_block_pool_keys(kc, lens_d, bs)
+    ref_bk = oracle.block_pool(w, bs)
+    np.testing.assert_allclose(bk.cpu().double().numpy(), ref_bk, atol=2e-5, rtol=1e-5)
+    out, bidx = tka.topk_block_attn_decode(q, kc, vc, bk, lens_d, bs, top)
+    torch.cuda.synchronize()
+    assert tka.topk_attn_device_status() == 0
+    check_block(w, bs, top, out, bidx, oracle.block_attn(w, bs, top))
