@@ -260,6 +260,9 @@ def run_ours(args, world, rank, local):
 
     K = args.steps
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    for e in (x for row in evs for x in row):
+        e.record()  # torch creates the CUDA event on its first record
+    torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()

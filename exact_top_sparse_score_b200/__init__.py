@@ -12,6 +12,7 @@ from ._binding import (  # noqa: F401
     TKA_F32,
     DEV_BAD_SEQ_LEN,
     DEV_INTERNAL,
+    DEV_TIMEOUT,
     TopkAttnError,
     block_attn_workspace_size,
     library_path,

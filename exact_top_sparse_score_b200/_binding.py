@@ -11,7 +11,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_NAME = "libtopk_attn.so"
 
 TKA_F32, TKA_BF16 = 0, 1
-DEV_BAD_SEQ_LEN, DEV_INTERNAL = 0x1, 0x2
+DEV_BAD_SEQ_LEN, DEV_INTERNAL, DEV_TIMEOUT = 0x1, 0x2, 0x4
 _STATUS = {0: "TKA_OK", 1: "TKA_ERR_INVALID_ARG", 2: "TKA_ERR_UNSUPPORTED", 3: "TKA_ERR_WORKSPACE",
            4: "TKA_ERR_CUDA"}
 
@@ -90,6 +90,16 @@ def _check_cuda(**tensors):
             raise ValueError(f"{name} must be contiguous")
 
 
+def _check_out(name: str, t: Optional[torch.Tensor], dtype: torch.dtype, shape: tuple):
+    """Caller-supplied output buffers must match what the kernels write."""
+    if t is None:
+        return
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
 def _stream(stream) -> int:
     if stream is None:
         return torch.cuda.current_stream().cuda_stream
@@ -119,12 +129,25 @@ def block_attn_workspace_size(shape: tka_shape, block_size: int, top_blocks: int
     return int(load_library().topk_block_attn_workspace_size(ctypes.byref(shape), block_size, top_blocks))
 
 
-def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]) -> torch.Tensor:
-    if workspace is None:
-        return torch.empty(nbytes, dtype=torch.uint8, device=device)
-    if workspace.numel() * workspace.element_size() < nbytes:
-        raise ValueError(f"workspace needs {nbytes} bytes")
-    return workspace
+# Workspaces the binding allocates itself, one per (device, stream), grown on
+# demand and kept for the life of the process: a call's kernels may still be
+# running when the call returns, so its scratch must not go back to the
+# allocator at that point.  Calls on one stream run in order, so they can
+# share one buffer.
+_cached_ws = {}
+
+
+def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor], stream_handle: int) -> torch.Tensor:
+    if workspace is not None:
+        if workspace.numel() * workspace.element_size() < nbytes:
+            raise ValueError(f"workspace needs {nbytes} bytes")
+        return workspace
+    key = (torch.device(device).index, stream_handle)
+    ws = _cached_ws.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        _cached_ws[key] = ws
+    return ws
 
 
 def topk_attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, seq_lens: torch.Tensor,
@@ -146,16 +169,24 @@ def topk_attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tens
         idx = torch.empty((B, Q, Hq, k), dtype=torch.int32, device=dev)
     if tail_mass is None and want_tail:
         tail_mass = torch.empty((B, Q, Hq), dtype=torch.float32, device=dev)
-    if seq_lens.dtype != torch.int32:
-        raise TypeError("seq_lens must be int32")
+    if seq_lens.dtype != torch.int32 or tuple(seq_lens.shape) != (B,):
+        raise TypeError("seq_lens must be int32 [B]")
+    if v_cache.dtype != k_cache.dtype or v_cache.shape != k_cache.shape:
+        raise TypeError("v_cache must match k_cache in dtype and shape")
+    _check_out("out", out, torch.float32, (B, Q, Hq, d))
+    _check_out("idx", idx, torch.int32, (B, Q, Hq, k))
+    _check_out("tail_mass", tail_mass, torch.float32, (B, Q, Hq))
+    if workspace is not None and workspace.dtype != torch.uint8:
+        raise TypeError("workspace must be a uint8 tensor")
     _check_cuda(q=q, k_cache=k_cache, v_cache=v_cache, seq_lens=seq_lens, out=out, idx=idx, tail_mass=tail_mass,
                 workspace=workspace)
     nbytes = topk_attn_workspace_size(shape, k)
     if nbytes == 0:
         raise TopkAttnError("topk_attn_workspace_size", 2)
-    ws = _workspace(nbytes, dev, workspace)
+    sh = _stream(stream)
+    ws = _workspace(nbytes, dev, workspace, sh)
     args = (ctypes.byref(shape), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seq_lens.data_ptr(), k,
-            out.data_ptr(), idx.data_ptr(), _ptr(tail_mass), ws.data_ptr(), nbytes, _stream(stream))
+            out.data_ptr(), idx.data_ptr(), _ptr(tail_mass), ws.data_ptr(), nbytes, sh)
     if stage_events is None:
         rc = lib.topk_attn_decode(*args)
     else:
@@ -174,6 +205,9 @@ def topk_block_pool_keys(k_cache: torch.Tensor, seq_lens: torch.Tensor, block_si
     nblk = -(-L_max // block_size)
     if block_keys is None:
         block_keys = torch.empty((B, Hkv, nblk, d), dtype=torch.float32, device=k_cache.device)
+    if seq_lens.dtype != torch.int32 or tuple(seq_lens.shape) != (B,):
+        raise TypeError("seq_lens must be int32 [B]")
+    _check_out("block_keys", block_keys, torch.float32, (B, Hkv, nblk, d))
     _check_cuda(k_cache=k_cache, seq_lens=seq_lens, block_keys=block_keys)
     shape = tka_shape(B, 1, Hkv, Hkv, d, L_max, _dtype_code(k_cache), 0.0)
     rc = lib.topk_block_pool_keys(ctypes.byref(shape), k_cache.data_ptr(), seq_lens.data_ptr(), block_size,
@@ -196,15 +230,25 @@ def topk_block_attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torc
         out = torch.empty((B, Q, Hq, d), dtype=torch.float32, device=q.device)
     if block_idx is None:
         block_idx = torch.empty((B, Q, Hq, top_blocks + 1), dtype=torch.int32, device=q.device)
+    if seq_lens.dtype != torch.int32 or tuple(seq_lens.shape) != (B,):
+        raise TypeError("seq_lens must be int32 [B]")
+    if v_cache.dtype != k_cache.dtype or v_cache.shape != k_cache.shape:
+        raise TypeError("v_cache must match k_cache in dtype and shape")
+    _check_out("out", out, torch.float32, (B, Q, Hq, d))
+    _check_out("block_idx", block_idx, torch.int32, (B, Q, Hq, top_blocks + 1))
+    _check_out("block_keys", block_keys, torch.float32, (B, k_cache.shape[1], -(-k_cache.shape[2] // block_size), d))
+    if workspace is not None and workspace.dtype != torch.uint8:
+        raise TypeError("workspace must be a uint8 tensor")
     _check_cuda(q=q, k_cache=k_cache, v_cache=v_cache, block_keys=block_keys, seq_lens=seq_lens, out=out,
                 block_idx=block_idx, workspace=workspace)
     nbytes = block_attn_workspace_size(shape, block_size, top_blocks)
     if nbytes == 0:
         raise TopkAttnError("topk_block_attn_workspace_size", 2)
-    ws = _workspace(nbytes, q.device, workspace)
+    sh = _stream(stream)
+    ws = _workspace(nbytes, q.device, workspace, sh)
     rc = lib.topk_block_attn_decode(ctypes.byref(shape), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
                                     block_keys.data_ptr(), seq_lens.data_ptr(), block_size, top_blocks,
-                                    out.data_ptr(), block_idx.data_ptr(), ws.data_ptr(), nbytes, _stream(stream))
+                                    out.data_ptr(), block_idx.data_ptr(), ws.data_ptr(), nbytes, sh)
     if rc:
         raise TopkAttnError("topk_block_attn_decode", rc)
     return out, block_idx

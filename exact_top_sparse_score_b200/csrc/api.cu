@@ -75,9 +75,12 @@ tka_status check_shape(const tka_shape *s) {
 //   stats    float4 [rows]            {m, Z_k, Z_tail, 0}
 //   partial  fp32 [rows, max_splits, 128]
 //   counters uint32 [rows]
+//   rowhist  uint32 [rows, 2048] + rowmax uint32 [rows]   (bf16 with Q*G <= 8: the
+//            tensor-core scorer's radix histogram and row maximum, zeroed per call)
 struct TokenLayout {
-    size_t scores, weights, stats, partial, counters, total;
+    size_t scores, weights, stats, partial, counters, rowhist, rowmax, total;
     int ld, max_splits;
+    bool hist;
 };
 
 TokenLayout token_layout(const tka_shape *s, int k) {
@@ -96,6 +99,10 @@ TokenLayout token_layout(const tka_shape *s, int k) {
     off = align_up(off + rows * (size_t)L.max_splits * kHeadDim * sizeof(float), 256);
     L.counters = off;
     off = align_up(off + rows * sizeof(unsigned), 256);
+    L.hist = s->dtype == TKA_BF16 && score_tc_builds_hist(s->Q * (s->Hq / s->Hkv));
+    L.rowhist = off;
+    L.rowmax = off + rows * 2048 * sizeof(unsigned);
+    if (L.hist) off = align_up(L.rowmax + rows * sizeof(unsigned), 256);
     L.total = off;
     return L;
 }
@@ -168,22 +175,44 @@ tka_status topk_attn_decode_staged(const tka_shape *shape, const void *q, const 
     const int G = shape->Hq / shape->Hkv;
     const int rows = shape->B * shape->Q * shape->Hq;
 
-    ScoreParams sp;
-    sp.status = dev->status;
-    sp.q = q;
-    sp.k = k_cache;
-    sp.seq_lens = seq_lens;
-    sp.scores = reinterpret_cast<float *>(ws + L.scores);
-    sp.B = shape->B; sp.Q = shape->Q; sp.Hq = shape->Hq; sp.Hkv = shape->Hkv; sp.G = G;
-    sp.L_max = shape->L_max; sp.ld = L.ld; sp.dtype = shape->dtype;
-    sp.scale = resolve_scale(shape);
+    float *scores = reinterpret_cast<float *>(ws + L.scores);
+    const int NQ = shape->Q * G;
+    // the tensor map addresses cache rows with int32 coordinates
+    const bool tc = score_tc_supported(shape->dtype, NQ) &&
+                    (long long)shape->B * shape->Hkv * shape->L_max < (1LL << 31);
+    const bool hist = tc && L.hist;
     if (record(events, 0, s) != cudaSuccess) return TKA_ERR_CUDA;
-    if (launch_score(sp, dev->num_sms, s) != cudaSuccess) return TKA_ERR_CUDA;
+    if (tc) {
+        if (hist && cudaMemsetAsync(ws + L.rowhist, 0, L.total - L.rowhist, s) != cudaSuccess) return TKA_ERR_CUDA;
+        ScoreTcParams tp;
+        tp.status = dev->status;
+        tp.seq_lens = seq_lens;
+        tp.scores = scores;
+        tp.rowhist = hist ? reinterpret_cast<unsigned *>(ws + L.rowhist) : nullptr;
+        tp.rowmax = hist ? reinterpret_cast<unsigned *>(ws + L.rowmax) : nullptr;
+        tp.B = shape->B; tp.Q = shape->Q; tp.Hq = shape->Hq; tp.Hkv = shape->Hkv; tp.G = G;
+        tp.L_max = shape->L_max; tp.ld = L.ld; tp.NQ = NQ;
+        tp.scale = resolve_scale(shape);
+        if (launch_score_tc(tp, q, k_cache, dev->num_sms, s) != cudaSuccess) return TKA_ERR_CUDA;
+    } else {
+        ScoreParams sp;
+        sp.status = dev->status;
+        sp.q = q;
+        sp.k = k_cache;
+        sp.seq_lens = seq_lens;
+        sp.scores = scores;
+        sp.B = shape->B; sp.Q = shape->Q; sp.Hq = shape->Hq; sp.Hkv = shape->Hkv; sp.G = G;
+        sp.L_max = shape->L_max; sp.ld = L.ld; sp.dtype = shape->dtype;
+        sp.scale = resolve_scale(shape);
+        if (launch_score(sp, dev->num_sms, s) != cudaSuccess) return TKA_ERR_CUDA;
+    }
     if (record(events, 1, s) != cudaSuccess) return TKA_ERR_CUDA;
 
     SelectParams se;
     se.status = dev->status;
-    se.scores = sp.scores;
+    se.scores = scores;
+    se.rowhist = hist ? reinterpret_cast<const unsigned *>(ws + L.rowhist) : nullptr;
+    se.rowmax = hist ? reinterpret_cast<const unsigned *>(ws + L.rowmax) : nullptr;
     se.seq_lens = seq_lens;
     se.B = shape->B; se.Q = shape->Q; se.Hq = shape->Hq; se.L_max = shape->L_max; se.ld = L.ld; se.k = k;
     se.idx = idx;

@@ -1,0 +1,384 @@
+// Score step on the 5th-generation tensor cores (bf16 cache).
+//
+// s[row, i] = scale * <q_row, K[b, kvh, i, :]> for every key below the
+// sequence length, all Q*G query rows of a kv-head at once: a
+// [128 keys x 128 dims] x [128 dims x N rows] product per tile of 128 keys,
+// i.e. the relevance scan of the whole cache ("Sparse Attention in LLM
+// Inference: Practical Trade-Offs", sections "The Role of the Indexer" and
+// "The Overhead of the Indexer") with the exact logit as the score.
+//
+// Persistent kernel, one CTA per SM.  The valid tiles (b, kv-head, 128-key
+// block below seq_lens[b]) are numbered in order and each CTA takes one
+// contiguous, equal share, so every CTA streams a contiguous run of the cache
+// and sees at most a few kv-heads.  Warp roles:
+//   warp 0      TMA producer: K tiles (two 64-dim boxes, 128-byte swizzle) into
+//               a ring of shared-memory stages; the kv-head's query rows into
+//               one of two query buffers whenever the kv-head changes.
+//   warp 1      MMA issuer: allocates TMEM, issues 8 tcgen05.mma (K = 16 each)
+//               per tile into one of two TMEM accumulators, commits to the
+//               stage's "empty" and the accumulator's "full" barriers.
+//   warps 2-5   epilogue: TMEM -> registers (one key per thread, N query
+//               columns), scale, coalesced score stores (32 consecutive keys
+//               per warp per row), and optionally the per-row radix
+//               histogram of the top 11 order-key bits and the row maximum
+//               that the select step starts from.
+// Every barrier wait is bounded; a wait that gives up raises TKA_DEV_TIMEOUT,
+// makes the other roles stop, drains the copies and MMAs in flight, frees
+// TMEM and returns.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace tka {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kTileKeys = 128;
+constexpr int kKBlockBytes = kTileKeys * 128;  // 64 bf16 dims x 128 keys
+constexpr int kTileBytes = 2 * kKBlockBytes;   // 128 dims
+constexpr int kThreads = 192;
+constexpr int kHistBins = 2048;
+
+__host__ __device__ constexpr int stages_for(int N) { return N <= 64 ? 4 : 3; }
+__host__ __device__ constexpr int tmem_cols_for(int N) { return 2 * N < 32 ? 32 : 2 * N; }
+
+__device__ __forceinline__ int tiles_of(const ScoreTcParams &p, int b) {
+    const int L = p.seq_lens[b];
+    if (!seq_len_ok(L, p.Q, p.L_max)) return 0;
+    return (L + kTileKeys - 1) / kTileKeys;
+}
+
+// Walks this CTA's share of the valid tiles in (bh, tile) order.
+struct TileWalk {
+    int bh, t, ntb, count;
+    __device__ void init(const ScoreTcParams &p) {
+        long long total = 0;
+        for (int b = 0; b < p.B; b++) total += (long long)p.Hkv * tiles_of(p, b);
+        const long long lo = total * blockIdx.x / gridDim.x, hi = total * (blockIdx.x + 1) / gridDim.x;
+        count = (int)(hi - lo);
+        long long cum = 0;
+        bh = 0;
+        t = 0;
+        ntb = 0;
+        if (count == 0) return;
+        for (int b = 0; b < p.B; b++) {
+            const int nt = tiles_of(p, b);
+            const long long here = (long long)p.Hkv * nt;
+            if (lo < cum + here) {
+                const long long off = lo - cum;
+                bh = b * p.Hkv + (int)(off / nt);
+                t = (int)(off % nt);
+                ntb = nt;
+                return;
+            }
+            cum += here;
+        }
+    }
+    __device__ bool seg_first(int i) const { return i == 0 || t == 0; }
+    __device__ bool seg_last(int i) const { return i == count - 1 || t + 1 == ntb; }
+    __device__ void next(const ScoreTcParams &p) {
+        if (++t < ntb) return;
+        t = 0;
+        do {
+            ++bh;
+            ntb = bh < p.B * p.Hkv ? tiles_of(p, bh / p.Hkv) : 1;
+        } while (ntb == 0);
+    }
+};
+
+template <int N, bool HIST>
+__global__ void __launch_bounds__(kThreads, 1)
+    score_tc(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap, ScoreTcParams p) {
+    constexpr int S = stages_for(N);
+    constexpr uint32_t kCols = tmem_cols_for(N);
+    constexpr int kQBuf = N * 256;  // two 64-dim blocks of N rows x 128 B
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *stages = base;
+    uint8_t *qbuf = stages + S * kTileBytes;
+    uint32_t *hist = reinterpret_cast<uint32_t *>(qbuf + 2 * kQBuf);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(hist + (HIST ? p.NQ * kHistBins : 0));
+    uint64_t *full = bars, *empty = bars + S, *qfull = bars + 2 * S, *qempty = qfull + 2, *tfull = qempty + 2,
+             *tempty = tfull + 2, *drain = tempty + 2, *hready = drain + 1, *hclear = drain + 2;
+    uint32_t *misc = reinterpret_cast<uint32_t *>(drain + 3);
+    // misc: [0] TMEM base, [1] abort flag, [2] K tiles issued, [3] query loads issued, [4..12) row max keys
+    volatile int *abort = reinterpret_cast<volatile int *>(&misc[1]);
+    uint32_t *smax = misc + 4;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; s++) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int j = 0; j < 2; j++) {
+            mbar_init(&qfull[j], 1);
+            mbar_init(&qempty[j], 1);
+            mbar_init(&tfull[j], 1);
+            mbar_init(&tempty[j], 128);
+        }
+        mbar_init(drain, 1);
+        mbar_init(hready, 128);
+        mbar_init(hclear, 128);
+        misc[1] = 0;
+        misc[2] = 0;
+        misc[3] = 0;
+        fence_barrier_init();
+    }
+    if (HIST) {
+        for (int i = threadIdx.x; i < p.NQ * kHistBins; i += kThreads) hist[i] = 0u;
+        if (threadIdx.x < 8) smax[threadIdx.x] = 0u;
+    }
+    if (warp == 1) tmem_alloc(&misc[0], kCols);
+    if (threadIdx.x == 0) {
+        prefetch_tensormap(&kmap);
+        prefetch_tensormap(&qmap);
+        if (blockIdx.x == 0)
+            for (int b = 0; b < p.B; b++)
+                if (!seq_len_ok(p.seq_lens[b], p.Q, p.L_max)) raise_status(p.status, TKA_DEV_BAD_SEQ_LEN);
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc[0];
+
+    TileWalk w;
+    w.init(p);
+    bool ok = true;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int seg = 0;
+            for (int i = 0; i < w.count && ok; i++) {
+                const int b = w.bh / p.Hkv, kvh = w.bh - b * p.Hkv;
+                if (w.seg_first(i)) {
+                    const int qb = seg & 1;
+                    if (seg >= 2) ok = mbar_wait(&qempty[qb], ((seg >> 1) - 1) & 1, abort);
+                    if (!ok) break;
+                    uint8_t *dst = qbuf + qb * kQBuf;
+                    mbar_arrive_expect_tx(&qfull[qb], 2u * 128u * p.NQ);
+                    tma_load_3d(dst, &qmap, &qfull[qb], 0, kvh * p.G, b * p.Q);
+                    tma_load_3d(dst + N * 128, &qmap, &qfull[qb], 64, kvh * p.G, b * p.Q);
+                    misc[3] = seg + 1;
+                }
+                const int s = i % S;
+                if (i >= S) ok = mbar_wait(&empty[s], ((i / S) - 1) & 1, abort);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&full[s], kTileBytes);
+                const int row0 = w.bh * p.L_max + w.t * kTileKeys;
+                tma_load_2d(stages + s * kTileBytes, &kmap, &full[s], 0, row0);
+                tma_load_2d(stages + s * kTileBytes + kKBlockBytes, &kmap, &full[s], 64, row0);
+                misc[2] = i + 1;
+                if (w.seg_last(i)) seg++;
+                w.next(p);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(128, N);
+            int seg = 0;
+            for (int i = 0; i < w.count && ok; i++) {
+                const int qb = seg & 1;
+                if (w.seg_first(i)) ok = mbar_wait(&qfull[qb], (seg >> 1) & 1, abort);
+                const int s = i % S, buf = i & 1;
+                if (ok) ok = mbar_wait(&full[s], (i / S) & 1, abort);
+                if (ok && i >= 2) ok = mbar_wait(&tempty[buf], ((i >> 1) - 1) & 1, abort);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t a0 = smem_addr(stages + s * kTileBytes), b0 = smem_addr(qbuf + qb * kQBuf);
+#pragma unroll
+                for (int k = 0; k < 8; k++) {
+                    const uint64_t ad = smem_desc_sw128(a0 + (k >> 2) * kKBlockBytes + (k & 3) * 32);
+                    const uint64_t bd = smem_desc_sw128(b0 + (k >> 2) * (N * 128) + (k & 3) * 32);
+                    mma_bf16(tmem + buf * N, ad, bd, idesc, k > 0 ? 1u : 0u);
+                }
+                mma_commit(&empty[s]);
+                mma_commit(&tfull[buf]);
+                if (w.seg_last(i)) {
+                    mma_commit(&qempty[qb]);
+                    seg++;
+                }
+                w.next(p);
+            }
+            // every MMA issued above has completed once this arrives (waited
+            // for even after an abort: TMEM is freed below)
+            mma_commit(drain);
+            int no_abort = 0;
+            if (!mbar_wait(drain, 0, reinterpret_cast<volatile int *>(&no_abort))) ok = false;
+        }
+    } else {
+        const int et = threadIdx.x - 64;   // 0..127
+        const int quarter = warp & 3;      // TMEM lanes [32*quarter, +32)
+        const uint32_t tlane = (uint32_t)(quarter * 32) << 16;
+        const float scale = p.scale;
+        int seg = 0;
+        for (int i = 0; i < w.count && ok; i++) {
+            const int b = w.bh / p.Hkv, kvh = w.bh - b * p.Hkv;
+            const int seq_len = p.seq_lens[b];
+            const int buf = i & 1;
+            ok = mbar_wait(&tfull[buf], (i >> 1) & 1, abort);
+            if (!ok) break;
+            tc_fence_after();
+            const int key = w.t * kTileKeys + quarter * 32 + lane;
+            const bool valid = key < seq_len;
+#pragma unroll
+            for (int c = 0; c < N / 16; c++) {
+                if (c * 16 >= p.NQ) break;
+                uint32_t r[16];
+                tmem_ld16(tmem + tlane + buf * N + c * 16, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; j++) {
+                    const int n = c * 16 + j;
+                    if (n >= p.NQ) break;
+                    const float sc = __uint_as_float(r[j]) * scale;
+                    const int qpos = n / p.G, gi = n - qpos * p.G;
+                    const size_t row = ((size_t)b * p.Q + qpos) * p.Hq + (size_t)kvh * p.G + gi;
+                    // keys a causal query position cannot see are neither stored nor counted
+                    const bool vis = valid && key < seq_len - p.Q + qpos + 1;
+                    if (vis) p.scores[row * p.ld + key] = sc;
+                    if (HIST) {
+                        const uint32_t okey = vis ? order_key(sc) : 0u;
+                        if (vis) atomicAdd(&hist[n * kHistBins + (okey >> 21)], 1u);
+                        uint32_t m = okey;
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+                        if (lane == 0) atomicMax(&smax[n], m);
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&tempty[buf]);
+            if (HIST && w.seg_last(i)) {
+                // all four epilogue warps have counted this kv-head's keys
+                mbar_arrive(hready);
+                ok = mbar_wait(hready, seg & 1, abort);
+                if (!ok) break;
+                for (int e = et; e < p.NQ * kHistBins; e += 128) {
+                    const uint32_t h = hist[e];
+                    if (h) {
+                        const int n = e / kHistBins, bin = e - n * kHistBins;
+                        const int qpos = n / p.G, gi = n - qpos * p.G;
+                        const size_t row = ((size_t)b * p.Q + qpos) * p.Hq + (size_t)kvh * p.G + gi;
+                        atomicAdd(&p.rowhist[row * kHistBins + bin], h);
+                        hist[e] = 0u;
+                    }
+                }
+                if (et < p.NQ) {
+                    const int qpos = et / p.G, gi = et - qpos * p.G;
+                    const size_t row = ((size_t)b * p.Q + qpos) * p.Hq + (size_t)kvh * p.G + gi;
+                    atomicMax(&p.rowmax[row], smax[et]);
+                    smax[et] = 0u;
+                }
+                // every bin is flushed and cleared before the next kv-head's counts
+                mbar_arrive(hclear);
+                ok = mbar_wait(hclear, seg & 1, abort);
+                seg++;
+            }
+            w.next(p);
+        }
+    }
+
+    if (!ok) {
+        *abort = 1;
+        raise_status(p.status, TKA_DEV_TIMEOUT);
+    }
+    __syncthreads();
+    if (*abort && threadIdx.x == 0) {
+        // let every copy still in flight land before the shared memory goes away
+        const int issued = (int)misc[2], qissued = (int)misc[3];
+        for (int s = 0; s < S && s < issued; s++) {
+            const int last = issued - 1 - ((issued - 1 - s) % S);
+            int dummy = 0;
+            mbar_wait(&full[s], (last / S) & 1, reinterpret_cast<volatile int *>(&dummy));
+        }
+        for (int j = 0; j < 2 && j < qissued; j++) {
+            const int last = qissued - 1 - ((qissued - 1 - j) % 2);
+            int dummy = 0;
+            mbar_wait(&qfull[j], (last >> 1) & 1, reinterpret_cast<volatile int *>(&dummy));
+        }
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kCols);
+    }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+template <int N, bool HIST>
+size_t smem_bytes(int NQ) {
+    constexpr int S = stages_for(N);
+    return 1024 + (size_t)S * kTileBytes + 2 * (size_t)N * 256 + (HIST ? (size_t)NQ * kHistBins * 4 : 0) +
+           (2 * S + 11) * 8 + 64;
+}
+
+template <int N, bool HIST>
+cudaError_t launch_n(const CUtensorMap &km, const CUtensorMap &qm, const ScoreTcParams &p, int num_sms,
+                     cudaStream_t stream) {
+    const size_t smem = smem_bytes<N, HIST>(p.NQ);
+    cudaError_t e = cudaFuncSetAttribute(score_tc<N, HIST>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    score_tc<N, HIST><<<num_sms, kThreads, smem, stream>>>(km, qm, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool score_tc_supported(int dtype, int NQ) { return dtype == TKA_BF16 && NQ <= 128 && encode_fn() != nullptr; }
+bool score_tc_builds_hist(int NQ) { return NQ <= 8; }
+
+cudaError_t launch_score_tc(const ScoreTcParams &p, const void *q, const void *k_cache, int num_sms,
+                            cudaStream_t stream) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    CUtensorMap km, qm;
+    {
+        // K cache as rows of 128 bf16: [B*Hkv*L_max, 128]; boxes of 128 rows x 64 dims
+        const cuuint64_t dims[2] = {128, (cuuint64_t)p.B * p.Hkv * p.L_max};
+        const cuuint64_t strides[1] = {256};
+        const cuuint32_t box[2] = {64, kTileKeys};
+        const cuuint32_t es[2] = {1, 1};
+        if (enc(&km, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(k_cache), dims, strides, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    {
+        // queries as [B*Q, Hq, 128]; one box = the G heads of a kv-head at all Q positions
+        const cuuint64_t dims[3] = {128, (cuuint64_t)p.Hq, (cuuint64_t)p.B * p.Q};
+        const cuuint64_t strides[2] = {256, (cuuint64_t)p.Hq * 256};
+        const cuuint32_t box[3] = {64, (cuuint32_t)p.G, (cuuint32_t)p.Q};
+        const cuuint32_t es[3] = {1, 1, 1};
+        if (enc(&qm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(q), dims, strides, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    const int NQ = p.NQ;
+    if (NQ <= 8) return launch_n<16, true>(km, qm, p, num_sms, stream);
+    if (NQ <= 16) return launch_n<16, false>(km, qm, p, num_sms, stream);
+    if (NQ <= 32) return launch_n<32, false>(km, qm, p, num_sms, stream);
+    if (NQ <= 64) return launch_n<64, false>(km, qm, p, num_sms, stream);
+    return launch_n<128, false>(km, qm, p, num_sms, stream);
+}
+
+}  // namespace tka

@@ -7,16 +7,22 @@
 // the discarded mass is the Top-k tail mass of "A Mathematical Theory of
 // Top-k Sparse Attention via Total Variation Distance" (abstract).
 //
-// One CTA per row.  Scores are mapped to order-preserving uint32 keys and the
-// k-th largest key is found exactly by a three-level radix select (11 + 11 +
-// 10 bits), each level one histogram pass over the row (the row is read from
-// L2: the score workspace of a decode step is small enough to stay resident).
-// A final pass walks the row in position order and compacts the kept
-// positions with block-wide prefix sums, so the output is ascending and a tie
-// at the threshold key is resolved by position.  The same pass computes
-// Z_k = sum_kept e^{s-m} and Z_tail = sum_dropped e^{s-m}, so the tail mass
-// Z_tail / (Z_k + Z_tail) is formed from the dropped terms directly rather
-// than as a difference.
+// One CTA per row.  Scores are compared as order-preserving uint32 keys, so
+// the k-th largest is found exactly by radix selection on the key bits.  Two
+// ways in:
+//   * histogram given (the tensor-core scorer built, per row, the histogram
+//     of the top 11 key bits and the row maximum): the bin holding the k-th
+//     key is read off the histogram, then ONE pass over the row compacts, in
+//     position order, the keys of higher bins (certainly kept) and collects
+//     the keys of that bin as candidates in shared memory.  The candidates are
+//     resolved exactly in shared memory (radix on the low 21 bits, ties to the
+//     lower position) and the two ascending lists are merged.  If the bin holds
+//     more candidates than fit, the row falls back to the path below.
+//   * no histogram: three histogram passes (11 + 11 + 10 bits) find the k-th
+//     key, and a fourth pass compacts the kept positions in order.
+// Either way the pass that writes the output also forms Z_k = sum_kept
+// e^{s-m} and Z_tail = sum_dropped e^{s-m}; the tail mass is
+// Z_tail / (Z_k + Z_tail), formed from the dropped terms directly.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -25,6 +31,11 @@ namespace tka {
 namespace {
 
 constexpr int kSelectThreads = 512;
+constexpr int kCandCap = 4096;
+
+__device__ __forceinline__ float key_to_float(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
 
 // Exclusive prefix sum of one value per thread over the block; *total gets
 // the block sum.  `tmp` holds >= 32 words of shared memory.
@@ -105,71 +116,99 @@ __device__ __forceinline__ void visit_row(const float *s, int n, F &&f) {
     for (int j = 4 * n4 + threadIdx.x; j < n; j += stride) f(j, __ldcg(s + j));
 }
 
-__global__ void __launch_bounds__(kSelectThreads) select_topk(SelectParams p) {
-    __shared__ uint32_t hist[2048];
-    __shared__ uint32_t tmp[32];
-    __shared__ float red[32];
-    __shared__ uint32_t s_bin, s_above;
-
-    const int row = blockIdx.x;
-    const int b = row / (p.Q * p.Hq), qpos = (row / p.Hq) % p.Q;
-    const int seq_len = p.seq_lens[b];
-    if (!seq_len_ok(seq_len, p.Q, p.L_max)) {
-        if (threadIdx.x == 0) raise_status(p.status, TKA_DEV_BAD_SEQ_LEN);
-        return;
+// Loads 4 consecutive positions i0..i0+3 (zeros past n).
+__device__ __forceinline__ void load4(const float *s, int i0, int n, float (&x)[4]) {
+    if (i0 + 3 < n) {
+        const float4 v = __ldcg(reinterpret_cast<const float4 *>(s + i0));
+        x[0] = v.x;
+        x[1] = v.y;
+        x[2] = v.z;
+        x[3] = v.w;
+    } else {
+#pragma unroll
+        for (int j = 0; j < 4; j++) x[j] = i0 + j < n ? __ldcg(s + i0 + j) : 0.f;
     }
-    const int vis = visible_keys(seq_len, p.Q, qpos);
+}
+
+struct SelectSmem {
+    uint32_t *hist;  // [2048]
+    uint32_t *tmp;   // [32]
+    float *red;      // [32]
+    uint32_t *scal;  // [2]: bin, above
+};
+
+// Writes stats, tail and counter of a finished row.
+__device__ __forceinline__ void finish_row(const SelectParams &p, int row, float m, float zk, float zt,
+                                           uint32_t written, uint32_t kept, const SelectSmem &sm) {
+    zk = block_sum(zk, sm.red);
+    __syncthreads();
+    zt = block_sum(zt, sm.red);
+    if (threadIdx.x == 0) {
+        if (written != kept) raise_status(p.status, TKA_DEV_INTERNAL);
+        p.stats[row] = make_float4(m, zk, zt, 0.f);
+        if (p.tail) p.tail[row] = zt / (zk + zt);
+        p.counters[row] = 0u;
+    }
+}
+
+// k >= visible keys: every position is kept, in order.
+__device__ void select_all(const SelectParams &p, int row, int vis, float m, const SelectSmem &sm) {
+    const float *s = p.scores + (size_t)row * p.ld;
+    int32_t *idx = p.idx + (size_t)row * p.k;
+    float *wv = p.w + (size_t)row * p.k;
+    float zk = 0.f;
+    visit_row(s, vis, [&](int i, float x) {
+        const float e = __expf(x - m);
+        idx[i] = i;
+        wv[i] = e;
+        zk += e;
+    });
+    for (int j = vis + threadIdx.x; j < p.k; j += blockDim.x) idx[j] = -1;
+    finish_row(p, row, m, zk, 0.f, vis, vis, sm);
+}
+
+// Three histogram passes and an ordered compaction pass (no histogram given,
+// or too many candidates in the boundary bin).
+__device__ void select_multipass(const SelectParams &p, int row, int vis, const SelectSmem &sm) {
     const float *s = p.scores + (size_t)row * p.ld;
     const int k = p.k;
-    const bool take_all = k >= vis;
-
+    uint32_t *hist = sm.hist;
     for (int i = threadIdx.x; i < 2048; i += blockDim.x) hist[i] = 0u;
     __syncthreads();
-
-    // pass 1: row max and histogram of the top 11 key bits
     float m = -INFINITY;
     visit_row(s, vis, [&](int, float x) {
         m = fmaxf(m, x);
-        if (!take_all) atomicAdd(&hist[order_key(x) >> 21], 1u);
+        atomicAdd(&hist[order_key(x) >> 21], 1u);
     });
-    m = block_max(m, red);
+    m = block_max(m, sm.red);
+    __syncthreads();
+    find_bin(hist, 2048, (uint32_t)k, sm.tmp, &sm.scal[0], &sm.scal[1]);
+    const uint32_t b1 = sm.scal[0];
+    uint32_t above = sm.scal[1];
+    for (int i = threadIdx.x; i < 2048; i += blockDim.x) hist[i] = 0u;
+    __syncthreads();
+    visit_row(s, vis, [&](int, float x) {
+        const uint32_t key = order_key(x);
+        if ((key >> 21) == b1) atomicAdd(&hist[(key >> 10) & 0x7ffu], 1u);
+    });
+    __syncthreads();
+    find_bin(hist, 2048, (uint32_t)k - above, sm.tmp, &sm.scal[0], &sm.scal[1]);
+    const uint32_t b2 = sm.scal[0];
+    above += sm.scal[1];
+    const uint32_t pre = (b1 << 11) | b2;
+    for (int i = threadIdx.x; i < 2048; i += blockDim.x) hist[i] = 0u;
+    __syncthreads();
+    visit_row(s, vis, [&](int, float x) {
+        const uint32_t key = order_key(x);
+        if ((key >> 10) == pre) atomicAdd(&hist[key & 0x3ffu], 1u);
+    });
+    __syncthreads();
+    find_bin(hist, 1024, (uint32_t)k - above, sm.tmp, &sm.scal[0], &sm.scal[1]);
+    const uint32_t b3 = sm.scal[0];
+    above += sm.scal[1];
+    const uint32_t T = (pre << 10) | b3, n_eq = hist[b3], r_eq = (uint32_t)k - above;
+    const bool rank_ties = n_eq != r_eq;
 
-    uint32_t T = 0u, n_eq = 0u, r_eq = 0u;  // threshold key, its multiplicity, how many of those to keep
-    if (!take_all) {
-        __syncthreads();
-        find_bin(hist, 2048, (uint32_t)k, tmp, &s_bin, &s_above);
-        const uint32_t b1 = s_bin;
-        uint32_t above = s_above;
-        for (int i = threadIdx.x; i < 2048; i += blockDim.x) hist[i] = 0u;
-        __syncthreads();
-        // pass 2: next 11 bits among keys in bin b1
-        visit_row(s, vis, [&](int, float x) {
-            const uint32_t key = order_key(x);
-            if ((key >> 21) == b1) atomicAdd(&hist[(key >> 10) & 0x7ffu], 1u);
-        });
-        __syncthreads();
-        find_bin(hist, 2048, (uint32_t)k - above, tmp, &s_bin, &s_above);
-        const uint32_t b2 = s_bin;
-        above += s_above;
-        const uint32_t pre = (b1 << 11) | b2;
-        for (int i = threadIdx.x; i < 2048; i += blockDim.x) hist[i] = 0u;
-        __syncthreads();
-        // pass 3: last 10 bits among keys matching the 22-bit prefix
-        visit_row(s, vis, [&](int, float x) {
-            const uint32_t key = order_key(x);
-            if ((key >> 10) == pre) atomicAdd(&hist[key & 0x3ffu], 1u);
-        });
-        __syncthreads();
-        find_bin(hist, 1024, (uint32_t)k - above, tmp, &s_bin, &s_above);
-        const uint32_t b3 = s_bin;
-        above += s_above;
-        T = (pre << 10) | b3;
-        n_eq = hist[b3];
-        r_eq = (uint32_t)k - above;
-    }
-    const bool rank_ties = !take_all && n_eq != r_eq;
-
-    // pass 4: ordered compaction, 4 consecutive positions per thread per tile
     int32_t *idx = p.idx + (size_t)row * k;
     float *wv = p.w + (size_t)row * k;
     uint32_t base_sel = 0u, base_eq = 0u;
@@ -177,13 +216,7 @@ __global__ void __launch_bounds__(kSelectThreads) select_topk(SelectParams p) {
     for (int tile = 0; tile < vis; tile += 4 * blockDim.x) {
         const int i0 = tile + 4 * threadIdx.x;
         float x[4];
-        if (i0 + 3 < vis) {
-            const float4 v = __ldcg(reinterpret_cast<const float4 *>(s + i0));
-            x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
-        } else {
-#pragma unroll
-            for (int j = 0; j < 4; j++) x[j] = i0 + j < vis ? __ldcg(s + i0 + j) : 0.f;
-        }
+        load4(s, i0, vis, x);
         uint32_t key[4], n_eq_t = 0u;
 #pragma unroll
         for (int j = 0; j < 4; j++) {
@@ -191,29 +224,24 @@ __global__ void __launch_bounds__(kSelectThreads) select_topk(SelectParams p) {
             if (i0 + j < vis && key[j] == T) n_eq_t++;
         }
         uint32_t eq_total = 0u, eq_rank = base_eq;
-        if (rank_ties) eq_rank += block_excl_scan(n_eq_t, tmp, &eq_total);
+        if (rank_ties) eq_rank += block_excl_scan(n_eq_t, sm.tmp, &eq_total);
         bool sel[4];
         uint32_t n_sel_t = 0u;
 #pragma unroll
         for (int j = 0; j < 4; j++) {
             bool v = i0 + j < vis;
-            if (v && !take_all) {
-                if (key[j] == T)
-                    v = !rank_ties || (eq_rank++ < r_eq);
-                else
-                    v = key[j] > T;
-            }
+            if (v) v = key[j] == T ? (!rank_ties || eq_rank++ < r_eq) : key[j] > T;
             sel[j] = v;
             n_sel_t += v;
         }
         uint32_t sel_total;
-        uint32_t pos = base_sel + block_excl_scan(n_sel_t, tmp, &sel_total);
+        uint32_t pos = base_sel + block_excl_scan(n_sel_t, sm.tmp, &sel_total);
 #pragma unroll
         for (int j = 0; j < 4; j++) {
             if (i0 + j >= vis) continue;
             const float e = __expf(x[j] - m);
             if (sel[j]) {
-                if (pos < (uint32_t)k) {  // always true unless the select above is wrong
+                if (pos < (uint32_t)k) {  // always true unless the search above is wrong
                     idx[pos] = i0 + j;
                     wv[pos] = e;
                 }
@@ -226,24 +254,202 @@ __global__ void __launch_bounds__(kSelectThreads) select_topk(SelectParams p) {
         base_sel += sel_total;
         base_eq += eq_total;
     }
-    const int kept = take_all ? vis : k;
-    for (int j = kept + threadIdx.x; j < k; j += blockDim.x) idx[j] = -1;
-    zk = block_sum(zk, red);
-    __syncthreads();
-    zt = block_sum(zt, red);
-    if (threadIdx.x == 0) {
-        if (base_sel != (uint32_t)kept) raise_status(p.status, TKA_DEV_INTERNAL);
-        p.stats[row] = make_float4(m, zk, zt, 0.f);
-        if (p.tail) p.tail[row] = zt / (zk + zt);
-        p.counters[row] = 0u;
+    finish_row(p, row, m, zk, zt, base_sel, (uint32_t)k, sm);
+}
+
+// Number of elements of the ascending array a[0..n) that are < x.
+__device__ __forceinline__ int lower_bound(const int32_t *a, int n, int32_t x) {
+    int lo = 0, hi = n;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (a[mid] < x)
+            lo = mid + 1;
+        else
+            hi = mid;
     }
+    return lo;
+}
+
+__global__ void __launch_bounds__(kSelectThreads) select_topk(SelectParams p) {
+    extern __shared__ uint32_t dyn[];
+    SelectSmem sm;
+    sm.hist = dyn;
+    sm.tmp = dyn + 2048;
+    sm.red = reinterpret_cast<float *>(dyn + 2048 + 32);
+    sm.scal = dyn + 2048 + 64;
+    int32_t *a_idx = reinterpret_cast<int32_t *>(dyn + 2048 + 64 + 8);  // [k]
+    float *a_w = reinterpret_cast<float *>(a_idx + p.k);                 // [k]
+    uint32_t *c_key = reinterpret_cast<uint32_t *>(a_w + p.k);           // [kCandCap]
+    int32_t *c_idx = reinterpret_cast<int32_t *>(c_key + kCandCap);      // [kCandCap]
+
+    const int row = blockIdx.x;
+    const int b = row / (p.Q * p.Hq), qpos = (row / p.Hq) % p.Q;
+    const int seq_len = p.seq_lens[b];
+    if (!seq_len_ok(seq_len, p.Q, p.L_max)) {
+        if (threadIdx.x == 0) raise_status(p.status, TKA_DEV_BAD_SEQ_LEN);
+        return;
+    }
+    const int vis = visible_keys(seq_len, p.Q, qpos);
+    const int k = p.k;
+    const float *s = p.scores + (size_t)row * p.ld;
+
+    if (!p.rowhist) {
+        if (k >= vis) {
+            float m = -INFINITY;
+            visit_row(s, vis, [&](int, float x) { m = fmaxf(m, x); });
+            m = block_max(m, sm.red);
+            select_all(p, row, vis, m, sm);
+        } else {
+            select_multipass(p, row, vis, sm);
+        }
+        return;
+    }
+
+    const float m = key_to_float(p.rowmax[row]);
+    if (k >= vis) {
+        select_all(p, row, vis, m, sm);
+        return;
+    }
+    for (int i = threadIdx.x; i < 2048; i += blockDim.x) sm.hist[i] = p.rowhist[(size_t)row * 2048 + i];
+    __syncthreads();
+    find_bin(sm.hist, 2048, (uint32_t)k, sm.tmp, &sm.scal[0], &sm.scal[1]);
+    const uint32_t b1 = sm.scal[0], above = sm.scal[1], ncand = sm.hist[b1];
+    if (ncand > (uint32_t)kCandCap) {
+        __syncthreads();
+        select_multipass(p, row, vis, sm);
+        return;
+    }
+
+    // one pass: keys of higher bins go to list A, keys of bin b1 to the candidates
+    uint32_t base_a = 0u, base_c = 0u;
+    float zk = 0.f, zt = 0.f;
+    for (int tile = 0; tile < vis; tile += 4 * blockDim.x) {
+        const int i0 = tile + 4 * threadIdx.x;
+        float x[4];
+        load4(s, i0, vis, x);
+        uint32_t key[4], cnt = 0u;
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            key[j] = order_key(x[j]);
+            if (i0 + j < vis) cnt += (key[j] >> 21) > b1 ? 1u : ((key[j] >> 21) == b1 ? 0x10000u : 0u);
+        }
+        uint32_t tot;
+        const uint32_t ex = block_excl_scan(cnt, sm.tmp, &tot);
+        uint32_t pa = base_a + (ex & 0xffffu), pc = base_c + (ex >> 16);
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            if (i0 + j >= vis) continue;
+            const uint32_t bin = key[j] >> 21;
+            if (bin > b1) {
+                const float e = __expf(x[j] - m);
+                if (pa < above) {  // always true unless the histogram is wrong
+                    a_idx[pa] = i0 + j;
+                    a_w[pa] = e;
+                }
+                pa++;
+                zk += e;
+            } else if (bin == b1) {
+                if (pc < ncand) {
+                    c_key[pc] = key[j];
+                    c_idx[pc] = i0 + j;
+                }
+                pc++;
+            } else {
+                zt += __expf(x[j] - m);
+            }
+        }
+        base_a += tot & 0xffffu;
+        base_c += tot >> 16;
+    }
+    if (base_a != above || base_c != ncand) {
+        // the histogram does not describe these scores (a library bug); recompute safely
+        if (threadIdx.x == 0) raise_status(p.status, TKA_DEV_INTERNAL);
+        __syncthreads();
+        select_multipass(p, row, vis, sm);
+        return;
+    }
+    __syncthreads();
+
+    // resolve the boundary bin: r of its ncand keys are kept
+    const uint32_t r = (uint32_t)k - above;
+    uint32_t *hist = sm.hist;
+    for (int i = threadIdx.x; i < 2048; i += blockDim.x) hist[i] = 0u;
+    __syncthreads();
+    for (uint32_t c = threadIdx.x; c < ncand; c += blockDim.x) atomicAdd(&hist[(c_key[c] >> 10) & 0x7ffu], 1u);
+    __syncthreads();
+    find_bin(hist, 2048, r, sm.tmp, &sm.scal[0], &sm.scal[1]);
+    const uint32_t b2 = sm.scal[0];
+    uint32_t gt = sm.scal[1];
+    const uint32_t pre = (b1 << 11) | b2;
+    for (int i = threadIdx.x; i < 2048; i += blockDim.x) hist[i] = 0u;
+    __syncthreads();
+    for (uint32_t c = threadIdx.x; c < ncand; c += blockDim.x)
+        if ((c_key[c] >> 10) == pre) atomicAdd(&hist[c_key[c] & 0x3ffu], 1u);
+    __syncthreads();
+    find_bin(hist, 1024, r - gt, sm.tmp, &sm.scal[0], &sm.scal[1]);
+    const uint32_t b3 = sm.scal[0];
+    gt += sm.scal[1];
+    const uint32_t T = (pre << 10) | b3, n_eq = hist[b3], r_eq = r - gt;
+    const bool rank_ties = n_eq != r_eq;
+
+    // compact the chosen candidates in place (candidates are in position order)
+    uint32_t base_b = 0u, base_eq = 0u;
+    for (uint32_t c0 = 0; c0 < ncand; c0 += blockDim.x) {
+        const uint32_t c = c0 + threadIdx.x;
+        const bool have = c < ncand;
+        const uint32_t key = have ? c_key[c] : 0u;
+        const int32_t pos = have ? c_idx[c] : 0;
+        uint32_t eq_total = 0u, eq_rank = base_eq;
+        if (rank_ties) eq_rank += block_excl_scan(have && key == T ? 1u : 0u, sm.tmp, &eq_total);
+        const bool chosen = have && (key == T ? (!rank_ties || eq_rank < r_eq) : key > T);
+        uint32_t tot;
+        const uint32_t dst = base_b + block_excl_scan(chosen ? 1u : 0u, sm.tmp, &tot);  // ends with a barrier
+        if (have) {
+            const float e = __expf(key_to_float(key) - m);
+            if (chosen) {
+                c_idx[dst] = pos;
+                reinterpret_cast<float *>(c_key)[dst] = e;
+                zk += e;
+            } else {
+                zt += e;
+            }
+        }
+        __syncthreads();
+        base_b += tot;
+        base_eq += eq_total;
+    }
+    // merge the two ascending lists into the output
+    int32_t *idx = p.idx + (size_t)row * k;
+    float *wv = p.w + (size_t)row * k;
+    const float *b_w = reinterpret_cast<const float *>(c_key);
+    const int na = (int)above, nb = (int)base_b;
+    for (int i = threadIdx.x; i < na; i += blockDim.x) {
+        const int pos = i + lower_bound(c_idx, nb, a_idx[i]);
+        idx[pos] = a_idx[i];
+        wv[pos] = a_w[i];
+    }
+    for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+        const int pos = i + lower_bound(a_idx, na, c_idx[i]);
+        idx[pos] = c_idx[i];
+        wv[pos] = b_w[i];
+    }
+    finish_row(p, row, m, zk, zt, above + base_b, (uint32_t)k, sm);
 }
 
 }  // namespace
 
+size_t select_smem_bytes(int k) {
+    return (size_t)(2048 + 64 + 8) * 4 + (size_t)k * 8 + (size_t)kCandCap * 8;
+}
+
 cudaError_t launch_select(const SelectParams &p, cudaStream_t stream) {
     const int rows = p.B * p.Q * p.Hq;
-    select_topk<<<rows, kSelectThreads, 0, stream>>>(p);
+    const size_t smem = select_smem_bytes(p.k);
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(select_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    select_topk<<<rows, kSelectThreads, smem, stream>>>(p);
     return cudaGetLastError();
 }
 

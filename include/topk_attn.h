@@ -69,6 +69,7 @@ typedef enum { TKA_F32 = 0, TKA_BF16 = 1 } tka_dtype;
 /* Bits of the device status word (OR-ed by kernels, cleared by reading). */
 #define TKA_DEV_BAD_SEQ_LEN 0x1u /* a seq_lens value was out of range; that sequence was skipped */
 #define TKA_DEV_INTERNAL 0x2u    /* an internal consistency check failed (a library bug) */
+#define TKA_DEV_TIMEOUT 0x4u     /* a bounded wait inside a kernel gave up; results are incomplete */
 
 /* cudaStream_t without pulling in the CUDA headers. */
 typedef struct CUstream_st *tka_stream_t;

@@ -55,7 +55,8 @@ def test_workspace_size_layout(lib):
     n = bd.topk_attn_workspace_size(s, 2048)
     rows = 8 * 32
     # scores + weights + stats + partial (32 splits of 64 keys) + counters
-    want = rows * 32768 * 4 + rows * 2048 * 4 + rows * 16 + rows * 32 * 128 * 4 + 1024
+    # + the scorer's per-row radix histogram (2048 bins) and row maximum
+    want = rows * 32768 * 4 + rows * 2048 * 4 + rows * 16 + rows * 32 * 128 * 4 + 1024 + rows * 2048 * 4 + rows * 4
     assert n == want
     assert bd.topk_attn_workspace_size(shape(L=1001), 7) % 256 == 0
 
@@ -106,3 +107,19 @@ def test_block_decode_rejects_bad_arguments_before_launch(lib):
     assert call(s, nbytes=16) == WORKSPACE
     assert lib.topk_block_pool_keys(ctypes.byref(s), FAKE, FAKE, 0, FAKE, None) == INVALID
     assert lib.topk_block_pool_keys(ctypes.byref(shape(d=96)), FAKE, FAKE, 64, FAKE, None) == UNSUPPORTED
+
+
+def test_binding_rejects_mismatched_output_buffers(lib):
+    import torch
+    import exact_top_sparse_score_b200 as tka
+    q = torch.zeros(1, 1, 4, 128, dtype=torch.bfloat16)
+    kc = torch.zeros(1, 2, 64, 128, dtype=torch.bfloat16)
+    lens = torch.full((1,), 64, dtype=torch.int32)
+    with pytest.raises(TypeError):   # fp64 outputs would be misread: the kernels write fp32
+        tka.topk_attn_decode(q, kc, kc, lens, 8, out=torch.zeros(1, 1, 4, 128, dtype=torch.float64))
+    with pytest.raises(TypeError):
+        tka.topk_attn_decode(q, kc, kc, lens, 8, idx=torch.zeros(1, 1, 4, 8, dtype=torch.int64))
+    with pytest.raises(ValueError):
+        tka.topk_attn_decode(q, kc, kc, lens, 8, tail_mass=torch.zeros(1, 1, 3, dtype=torch.float32))
+    with pytest.raises(ValueError):  # host tensors: there is no CPU path
+        tka.topk_attn_decode(q, kc, kc, lens, 8)

@@ -112,9 +112,9 @@ def test_bad_seq_len_raises_status_and_skips_sequence(cuda_device):
     q, kc, vc, lens = to_device(w)
     bad = lens.clone()
     bad[1] = 501  # > L_max
-    out = torch.full((2, 1, 8, 128), 7.0, device="cuda")
+    out = torch.full((2, 1, 8, 128), 7.0, dtype=torch.float32, device="cuda")
     idx = torch.full((2, 1, 8, 40), -7, dtype=torch.int32, device="cuda")
-    tail = torch.full((2, 1, 8), 7.0, device="cuda")
+    tail = torch.full((2, 1, 8), 7.0, dtype=torch.float32, device="cuda")
     tka.topk_attn_device_status()
     tka.topk_attn_decode(q, kc, vc, bad, 40, out=out, idx=idx, tail_mass=tail)
     assert tka.topk_attn_device_status() & tka.DEV_BAD_SEQ_LEN

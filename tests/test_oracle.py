@@ -26,8 +26,6 @@ import torch
 import oracle
 import workloads
 
-torch.set_default_dtype(torch.float64)
-
 
 def _f64(t):
     return t.to(torch.float64)
