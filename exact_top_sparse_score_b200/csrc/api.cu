@@ -75,12 +75,9 @@ tka_status check_shape(const tka_shape *s) {
 //   stats    float4 [rows]            {m, Z_k, Z_tail, 0}
 //   partial  fp32 [rows, max_splits, 128]
 //   counters uint32 [rows]
-//   rowhist  uint32 [rows, 2048] + rowmax uint32 [rows]   (bf16 with Q*G <= 8: the
-//            tensor-core scorer's radix histogram and row maximum, zeroed per call)
 struct TokenLayout {
-    size_t scores, weights, stats, partial, counters, rowhist, rowmax, total;
+    size_t scores, weights, stats, partial, counters, total;
     int ld, max_splits;
-    bool hist;
 };
 
 TokenLayout token_layout(const tka_shape *s, int k) {
@@ -99,10 +96,6 @@ TokenLayout token_layout(const tka_shape *s, int k) {
     off = align_up(off + rows * (size_t)L.max_splits * kHeadDim * sizeof(float), 256);
     L.counters = off;
     off = align_up(off + rows * sizeof(unsigned), 256);
-    L.hist = s->dtype == TKA_BF16 && score_tc_builds_hist(s->Q * (s->Hq / s->Hkv));
-    L.rowhist = off;
-    L.rowmax = off + rows * 2048 * sizeof(unsigned);
-    if (L.hist) off = align_up(L.rowmax + rows * sizeof(unsigned), 256);
     L.total = off;
     return L;
 }
@@ -180,16 +173,12 @@ tka_status topk_attn_decode_staged(const tka_shape *shape, const void *q, const 
     // the tensor map addresses cache rows with int32 coordinates
     const bool tc = score_tc_supported(shape->dtype, NQ) &&
                     (long long)shape->B * shape->Hkv * shape->L_max < (1LL << 31);
-    const bool hist = tc && L.hist;
     if (record(events, 0, s) != cudaSuccess) return TKA_ERR_CUDA;
     if (tc) {
-        if (hist && cudaMemsetAsync(ws + L.rowhist, 0, L.total - L.rowhist, s) != cudaSuccess) return TKA_ERR_CUDA;
         ScoreTcParams tp;
         tp.status = dev->status;
         tp.seq_lens = seq_lens;
         tp.scores = scores;
-        tp.rowhist = hist ? reinterpret_cast<unsigned *>(ws + L.rowhist) : nullptr;
-        tp.rowmax = hist ? reinterpret_cast<unsigned *>(ws + L.rowmax) : nullptr;
         tp.B = shape->B; tp.Q = shape->Q; tp.Hq = shape->Hq; tp.Hkv = shape->Hkv; tp.G = G;
         tp.L_max = shape->L_max; tp.ld = L.ld; tp.NQ = NQ;
         tp.scale = resolve_scale(shape);
@@ -211,8 +200,6 @@ tka_status topk_attn_decode_staged(const tka_shape *shape, const void *q, const 
     SelectParams se;
     se.status = dev->status;
     se.scores = scores;
-    se.rowhist = hist ? reinterpret_cast<const unsigned *>(ws + L.rowhist) : nullptr;
-    se.rowmax = hist ? reinterpret_cast<const unsigned *>(ws + L.rowmax) : nullptr;
     se.seq_lens = seq_lens;
     se.B = shape->B; se.Q = shape->Q; se.Hq = shape->Hq; se.L_max = shape->L_max; se.ld = L.ld; se.k = k;
     se.idx = idx;

@@ -7,11 +7,12 @@
 // come from the select step, so no K row is read again.
 //
 // Grid (splits, rows): each CTA gathers a contiguous slice of a row's kept
-// positions.  A V row is 256 bytes in bf16, read by 16 lanes with one 16-byte
-// load each (two rows per warp instruction); four rows per lane are in flight.
-// The slices of a row are summed by whichever CTA of the row finishes last
-// (an atomic ticket, no waiting), in slice order, so the result does not
-// depend on scheduling.
+// positions.  The slice's positions and weights are first staged in shared
+// memory (coalesced), so the V loads that follow depend on nothing in
+// flight: a V row is 256 bytes in bf16, read by 16 lanes with one 16-byte
+// load each, and every lane keeps 8 rows in flight.  The slices of a row are
+// summed by whichever CTA of the row finishes last (an atomic ticket, no
+// waiting), in slice order, so the result does not depend on scheduling.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -19,15 +20,43 @@ namespace tka {
 
 namespace {
 
-constexpr int kGatherThreads = 128;
+constexpr int kGatherThreads = 256;
+constexpr int kChunk = 512;  // positions staged in shared memory at a time
+constexpr int kUnroll = 8;
+
+__device__ __forceinline__ uint4 ldg_stream(const void *p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+template <typename T>
+__device__ __forceinline__ void fma_row(float (&acc)[16 / sizeof(T)], float wt, const uint4 &v) {
+    const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+    if constexpr (sizeof(T) == 2) {
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+            acc[2 * e] = fmaf(wt, bf16lo_to_f32(wd[e]), acc[2 * e]);
+            acc[2 * e + 1] = fmaf(wt, bf16hi_to_f32(wd[e]), acc[2 * e + 1]);
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < 4; e++) acc[e] = fmaf(wt, __uint_as_float(wd[e]), acc[e]);
+    }
+}
 
 template <typename T>
 __global__ void __launch_bounds__(kGatherThreads) gather_pv(GatherParams p) {
     constexpr int kPer = 16 / sizeof(T);              // elements per lane
     constexpr int kLanesPerRow = kHeadDim / kPer;     // 16 (bf16) or 32 (fp32)
     constexpr int kRowsPerWarp = 32 / kLanesPerRow;   // 2 or 1
-    constexpr int kSlots = (kGatherThreads / 32) * kRowsPerWarp;
-    __shared__ float red[kGatherThreads / 32][kHeadDim];
+    constexpr int kWarps = kGatherThreads / 32;
+    constexpr int kSlots = kWarps * kRowsPerWarp;
+    __shared__ int32_t s_idx[kChunk];
+    __shared__ float s_w[kChunk];
+    __shared__ float red[kWarps][kHeadDim];
     __shared__ unsigned s_ticket;
 
     const int row = blockIdx.y, split = blockIdx.x;
@@ -44,64 +73,38 @@ __global__ void __launch_bounds__(kGatherThreads) gather_pv(GatherParams p) {
     const int c = lane % kLanesPerRow;  // this lane's 16-byte piece of a V row
     const T *vbase = reinterpret_cast<const T *>(p.v) + ((size_t)b * p.Hkv + h / p.G) * p.L_max * kHeadDim +
                      c * kPer;
-    const int32_t *idx = p.idx + (size_t)row * p.k;
-    const float *wv = p.w + (size_t)row * p.k;
+    const int32_t *gidx = p.idx + (size_t)row * p.k;
+    const float *gw = p.w + (size_t)row * p.k;
 
     float acc[kPer];
 #pragma unroll
     for (int e = 0; e < kPer; e++) acc[e] = 0.f;
     bool bad = false;
 
-    int j = lo + slot;
-    for (; j + 3 * kSlots < hi; j += 4 * kSlots) {
-        uint4 v[4];
-        float wt[4];
-#pragma unroll
-        for (int u = 0; u < 4; u++) {
-            int pos = __ldg(idx + j + u * kSlots);
-            wt[u] = __ldg(wv + j + u * kSlots);
+    for (int c0 = lo; c0 < hi; c0 += kChunk) {
+        const int n = min(kChunk, hi - c0);
+        __syncthreads();
+        for (int j = threadIdx.x; j < n; j += kGatherThreads) {
+            int pos = __ldg(gidx + c0 + j);
+            float wt = __ldg(gw + c0 + j);
             if ((unsigned)pos >= (unsigned)vis) {  // never taken unless the select step is wrong
                 bad = true;
                 pos = 0;
-                wt[u] = 0.f;
+                wt = 0.f;
             }
-            v[u] = __ldg(reinterpret_cast<const uint4 *>(vbase + (size_t)pos * kHeadDim));
+            s_idx[j] = pos;
+            s_w[j] = wt;
         }
+        __syncthreads();
+        int j = slot;
+        for (; j + (kUnroll - 1) * kSlots < n; j += kUnroll * kSlots) {
+            uint4 v[kUnroll];
 #pragma unroll
-        for (int u = 0; u < 4; u++) {
-            const uint32_t wd[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-            if constexpr (sizeof(T) == 2) {
+            for (int u = 0; u < kUnroll; u++) v[u] = ldg_stream(vbase + (size_t)s_idx[j + u * kSlots] * kHeadDim);
 #pragma unroll
-                for (int e = 0; e < 4; e++) {
-                    acc[2 * e] = fmaf(wt[u], bf16lo_to_f32(wd[e]), acc[2 * e]);
-                    acc[2 * e + 1] = fmaf(wt[u], bf16hi_to_f32(wd[e]), acc[2 * e + 1]);
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < 4; e++) acc[e] = fmaf(wt[u], __uint_as_float(wd[e]), acc[e]);
-            }
+            for (int u = 0; u < kUnroll; u++) fma_row<T>(acc, s_w[j + u * kSlots], v[u]);
         }
-    }
-    for (; j < hi; j += kSlots) {
-        int pos = __ldg(idx + j);
-        float wt = __ldg(wv + j);
-        if ((unsigned)pos >= (unsigned)vis) {
-            bad = true;
-            pos = 0;
-            wt = 0.f;
-        }
-        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(vbase + (size_t)pos * kHeadDim));
-        const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
-        if constexpr (sizeof(T) == 2) {
-#pragma unroll
-            for (int e = 0; e < 4; e++) {
-                acc[2 * e] = fmaf(wt, bf16lo_to_f32(wd[e]), acc[2 * e]);
-                acc[2 * e + 1] = fmaf(wt, bf16hi_to_f32(wd[e]), acc[2 * e + 1]);
-            }
-        } else {
-#pragma unroll
-            for (int e = 0; e < 4; e++) acc[e] = fmaf(wt, __uint_as_float(wd[e]), acc[e]);
-        }
+        for (; j < n; j += kSlots) fma_row<T>(acc, s_w[j], ldg_stream(vbase + (size_t)s_idx[j] * kHeadDim));
     }
     if (bad) raise_status(p.status, TKA_DEV_INTERNAL);
     // sum the rows of a warp, then the warps of the CTA
@@ -114,10 +117,11 @@ __global__ void __launch_bounds__(kGatherThreads) gather_pv(GatherParams p) {
         for (int e = 0; e < kPer; e++) red[warp][c * kPer + e] = acc[e];
     }
     __syncthreads();
-    const int d = threadIdx.x;  // one output dim per thread (128 threads)
+    if (threadIdx.x >= kHeadDim) return;
+    const int d = threadIdx.x;  // one output dim per thread
     float sum = 0.f;
 #pragma unroll
-    for (int w = 0; w < kGatherThreads / 32; w++) sum += red[w][d];
+    for (int w = 0; w < kWarps; w++) sum += red[w][d];
     const float inv_zk = 1.f / p.stats[row].y;
     float *out = p.out + (size_t)row * kHeadDim;
     if (p.splits == 1) {
@@ -127,9 +131,9 @@ __global__ void __launch_bounds__(kGatherThreads) gather_pv(GatherParams p) {
     float *part = p.partial + (size_t)row * p.splits * kHeadDim;
     part[(size_t)split * kHeadDim + d] = sum;
     __threadfence();
-    __syncthreads();
+    asm volatile("bar.sync 1, %0;\n" ::"r"(kHeadDim));  // the 128 threads that wrote a partial
     if (threadIdx.x == 0) s_ticket = atomicAdd(&p.counters[row], 1u);
-    __syncthreads();
+    asm volatile("bar.sync 1, %0;\n" ::"r"(kHeadDim));
     if (s_ticket != (unsigned)p.splits - 1) return;
     __threadfence();
     float total = 0.f;

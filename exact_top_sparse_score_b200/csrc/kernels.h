@@ -20,8 +20,6 @@ struct ScoreTcParams {
     unsigned *status;         // device status word (TKA_DEV_* bits)
     const int32_t *seq_lens;  // [B]
     float *scores;            // [B*Q*Hq, ld]
-    unsigned *rowhist;        // [rows, 2048] histogram of order_key >> 21 (Q*G <= 8 only), zeroed by the caller
-    unsigned *rowmax;         // [rows] max order key (Q*G <= 8 only), zeroed by the caller
     int B, Q, Hq, Hkv, G, L_max, ld, NQ;
     float scale;
 };
@@ -29,8 +27,6 @@ struct ScoreTcParams {
 struct SelectParams {
     unsigned *status;         // device status word (TKA_DEV_* bits)
     const float *scores;      // [rows, ld]
-    const unsigned *rowhist;  // [rows, 2048] or null (then the select builds its own)
-    const unsigned *rowmax;   // [rows] max order key, with rowhist
     const int32_t *seq_lens;
     int B, Q, Hq, L_max, ld, k;
     int32_t *idx;             // [rows, k] ascending, -1 padded
@@ -88,7 +84,6 @@ struct BlockAttnParams {
 
 cudaError_t launch_score(const ScoreParams &p, int num_sms, cudaStream_t stream);
 bool score_tc_supported(int dtype, int NQ);
-bool score_tc_builds_hist(int NQ);
 cudaError_t launch_score_tc(const ScoreTcParams &p, const void *q, const void *k_cache, int num_sms,
                             cudaStream_t stream);
 cudaError_t launch_select(const SelectParams &p, cudaStream_t stream);

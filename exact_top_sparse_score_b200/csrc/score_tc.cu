@@ -19,9 +19,10 @@
 //               stage's "empty" and the accumulator's "full" barriers.
 //   warps 2-5   epilogue: TMEM -> registers (one key per thread, N query
 //               columns), scale, coalesced score stores (32 consecutive keys
-//               per warp per row), and optionally the per-row radix
-//               histogram of the top 11 order-key bits and the row maximum
-//               that the select step starts from.
+//               per warp per row; row addresses advance incrementally, no
+//               division in the loop).
+// K is read exactly once, so its TMA loads carry an L2 evict-first policy:
+// the scores written here stay in L2 for the select step.
 // Every barrier wait is bounded; a wait that gives up raises TKA_DEV_TIMEOUT,
 // makes the other roles stop, drains the copies and MMAs in flight, frees
 // TMEM and returns.
@@ -41,7 +42,6 @@ constexpr int kTileKeys = 128;
 constexpr int kKBlockBytes = kTileKeys * 128;  // 64 bf16 dims x 128 keys
 constexpr int kTileBytes = 2 * kKBlockBytes;   // 128 dims
 constexpr int kThreads = 192;
-constexpr int kHistBins = 2048;
 
 __host__ __device__ constexpr int stages_for(int N) { return N <= 64 ? 4 : 3; }
 __host__ __device__ constexpr int tmem_cols_for(int N) { return 2 * N < 32 ? 32 : 2 * N; }
@@ -90,7 +90,7 @@ struct TileWalk {
     }
 };
 
-template <int N, bool HIST>
+template <int N>
 __global__ void __launch_bounds__(kThreads, 1)
     score_tc(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap, ScoreTcParams p) {
     constexpr int S = stages_for(N);
@@ -100,14 +100,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *stages = base;
     uint8_t *qbuf = stages + S * kTileBytes;
-    uint32_t *hist = reinterpret_cast<uint32_t *>(qbuf + 2 * kQBuf);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(hist + (HIST ? p.NQ * kHistBins : 0));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(qbuf + 2 * kQBuf);
     uint64_t *full = bars, *empty = bars + S, *qfull = bars + 2 * S, *qempty = qfull + 2, *tfull = qempty + 2,
-             *tempty = tfull + 2, *drain = tempty + 2, *hready = drain + 1, *hclear = drain + 2;
-    uint32_t *misc = reinterpret_cast<uint32_t *>(drain + 3);
-    // misc: [0] TMEM base, [1] abort flag, [2] K tiles issued, [3] query loads issued, [4..12) row max keys
+             *tempty = tfull + 2, *drain = tempty + 2;
+    uint32_t *misc = reinterpret_cast<uint32_t *>(drain + 1);
+    // misc: [0] TMEM base, [1] abort flag, [2] K tiles issued, [3] query loads issued
     volatile int *abort = reinterpret_cast<volatile int *>(&misc[1]);
-    uint32_t *smax = misc + 4;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -122,16 +120,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&tempty[j], 128);
         }
         mbar_init(drain, 1);
-        mbar_init(hready, 128);
-        mbar_init(hclear, 128);
         misc[1] = 0;
         misc[2] = 0;
         misc[3] = 0;
         fence_barrier_init();
-    }
-    if (HIST) {
-        for (int i = threadIdx.x; i < p.NQ * kHistBins; i += kThreads) hist[i] = 0u;
-        if (threadIdx.x < 8) smax[threadIdx.x] = 0u;
     }
     if (warp == 1) tmem_alloc(&misc[0], kCols);
     if (threadIdx.x == 0) {
@@ -151,6 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0) {
         if (lane == 0) {
+            const uint64_t evict_first = policy_evict_first();
             int seg = 0;
             for (int i = 0; i < w.count && ok; i++) {
                 const int b = w.bh / p.Hkv, kvh = w.bh - b * p.Hkv;
@@ -169,8 +162,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 mbar_arrive_expect_tx(&full[s], kTileBytes);
                 const int row0 = w.bh * p.L_max + w.t * kTileKeys;
-                tma_load_2d(stages + s * kTileBytes, &kmap, &full[s], 0, row0);
-                tma_load_2d(stages + s * kTileBytes + kKBlockBytes, &kmap, &full[s], 64, row0);
+                tma_load_2d_hint(stages + s * kTileBytes, &kmap, &full[s], 0, row0, evict_first);
+                tma_load_2d_hint(stages + s * kTileBytes + kKBlockBytes, &kmap, &full[s], 64, row0, evict_first);
                 misc[2] = i + 1;
                 if (w.seg_last(i)) seg++;
                 w.next(p);
@@ -210,11 +203,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!mbar_wait(drain, 0, reinterpret_cast<volatile int *>(&no_abort))) ok = false;
         }
     } else {
-        const int et = threadIdx.x - 64;   // 0..127
         const int quarter = warp & 3;      // TMEM lanes [32*quarter, +32)
         const uint32_t tlane = (uint32_t)(quarter * 32) << 16;
         const float scale = p.scale;
-        int seg = 0;
         for (int i = 0; i < w.count && ok; i++) {
             const int b = w.bh / p.Hkv, kvh = w.bh - b * p.Hkv;
             const int seq_len = p.seq_lens[b];
@@ -223,7 +214,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             tc_fence_after();
             const int key = w.t * kTileKeys + quarter * 32 + lane;
-            const bool valid = key < seq_len;
+            // column n = qpos * G + gi is query row (b, qpos, kvh*G + gi); walk it without division
+            float *dst = p.scores + (((size_t)b * p.Q) * p.Hq + (size_t)kvh * p.G) * p.ld + key;
+            int qpos = 0, gi = 0, vis = seq_len - p.Q + 1;
 #pragma unroll
             for (int c = 0; c < N / 16; c++) {
                 if (c * 16 >= p.NQ) break;
@@ -232,52 +225,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 16; j++) {
-                    const int n = c * 16 + j;
-                    if (n >= p.NQ) break;
-                    const float sc = __uint_as_float(r[j]) * scale;
-                    const int qpos = n / p.G, gi = n - qpos * p.G;
-                    const size_t row = ((size_t)b * p.Q + qpos) * p.Hq + (size_t)kvh * p.G + gi;
-                    // keys a causal query position cannot see are neither stored nor counted
-                    const bool vis = valid && key < seq_len - p.Q + qpos + 1;
-                    if (vis) p.scores[row * p.ld + key] = sc;
-                    if (HIST) {
-                        const uint32_t okey = vis ? order_key(sc) : 0u;
-                        if (vis) atomicAdd(&hist[n * kHistBins + (okey >> 21)], 1u);
-                        uint32_t m = okey;
-#pragma unroll
-                        for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-                        if (lane == 0) atomicMax(&smax[n], m);
+                    if (c * 16 + j >= p.NQ) break;
+                    // keys a causal query position cannot see are not stored
+                    if (key < vis) *dst = __uint_as_float(r[j]) * scale;
+                    dst += p.ld;
+                    if (++gi == p.G) {
+                        gi = 0;
+                        ++qpos;
+                        ++vis;
+                        dst += (size_t)(p.Hq - p.G) * p.ld;
                     }
                 }
             }
             tc_fence_before();
             mbar_arrive(&tempty[buf]);
-            if (HIST && w.seg_last(i)) {
-                // all four epilogue warps have counted this kv-head's keys
-                mbar_arrive(hready);
-                ok = mbar_wait(hready, seg & 1, abort);
-                if (!ok) break;
-                for (int e = et; e < p.NQ * kHistBins; e += 128) {
-                    const uint32_t h = hist[e];
-                    if (h) {
-                        const int n = e / kHistBins, bin = e - n * kHistBins;
-                        const int qpos = n / p.G, gi = n - qpos * p.G;
-                        const size_t row = ((size_t)b * p.Q + qpos) * p.Hq + (size_t)kvh * p.G + gi;
-                        atomicAdd(&p.rowhist[row * kHistBins + bin], h);
-                        hist[e] = 0u;
-                    }
-                }
-                if (et < p.NQ) {
-                    const int qpos = et / p.G, gi = et - qpos * p.G;
-                    const size_t row = ((size_t)b * p.Q + qpos) * p.Hq + (size_t)kvh * p.G + gi;
-                    atomicMax(&p.rowmax[row], smax[et]);
-                    smax[et] = 0u;
-                }
-                // every bin is flushed and cleared before the next kv-head's counts
-                mbar_arrive(hclear);
-                ok = mbar_wait(hclear, seg & 1, abort);
-                seg++;
-            }
             w.next(p);
         }
     }
@@ -324,27 +285,25 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-template <int N, bool HIST>
-size_t smem_bytes(int NQ) {
+template <int N>
+size_t smem_bytes() {
     constexpr int S = stages_for(N);
-    return 1024 + (size_t)S * kTileBytes + 2 * (size_t)N * 256 + (HIST ? (size_t)NQ * kHistBins * 4 : 0) +
-           (2 * S + 11) * 8 + 64;
+    return 1024 + (size_t)S * kTileBytes + 2 * (size_t)N * 256 + (2 * S + 9) * 8 + 64;
 }
 
-template <int N, bool HIST>
+template <int N>
 cudaError_t launch_n(const CUtensorMap &km, const CUtensorMap &qm, const ScoreTcParams &p, int num_sms,
                      cudaStream_t stream) {
-    const size_t smem = smem_bytes<N, HIST>(p.NQ);
-    cudaError_t e = cudaFuncSetAttribute(score_tc<N, HIST>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const size_t smem = smem_bytes<N>();
+    cudaError_t e = cudaFuncSetAttribute(score_tc<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    score_tc<N, HIST><<<num_sms, kThreads, smem, stream>>>(km, qm, p);
+    score_tc<N><<<num_sms, kThreads, smem, stream>>>(km, qm, p);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 bool score_tc_supported(int dtype, int NQ) { return dtype == TKA_BF16 && NQ <= 128 && encode_fn() != nullptr; }
-bool score_tc_builds_hist(int NQ) { return NQ <= 8; }
 
 cudaError_t launch_score_tc(const ScoreTcParams &p, const void *q, const void *k_cache, int num_sms,
                             cudaStream_t stream) {
@@ -374,11 +333,10 @@ cudaError_t launch_score_tc(const ScoreTcParams &p, const void *q, const void *k
             return cudaErrorInvalidValue;
     }
     const int NQ = p.NQ;
-    if (NQ <= 8) return launch_n<16, true>(km, qm, p, num_sms, stream);
-    if (NQ <= 16) return launch_n<16, false>(km, qm, p, num_sms, stream);
-    if (NQ <= 32) return launch_n<32, false>(km, qm, p, num_sms, stream);
-    if (NQ <= 64) return launch_n<64, false>(km, qm, p, num_sms, stream);
-    return launch_n<128, false>(km, qm, p, num_sms, stream);
+    if (NQ <= 16) return launch_n<16>(km, qm, p, num_sms, stream);
+    if (NQ <= 32) return launch_n<32>(km, qm, p, num_sms, stream);
+    if (NQ <= 64) return launch_n<64>(km, qm, p, num_sms, stream);
+    return launch_n<128>(km, qm, p, num_sms, stream);
 }
 
 }  // namespace tka

@@ -8,21 +8,19 @@
 // Top-k Sparse Attention via Total Variation Distance" (abstract).
 //
 // One CTA per row.  Scores are compared as order-preserving uint32 keys, so
-// the k-th largest is found exactly by radix selection on the key bits.  Two
-// ways in:
-//   * histogram given (the tensor-core scorer built, per row, the histogram
-//     of the top 11 key bits and the row maximum): the bin holding the k-th
-//     key is read off the histogram, then ONE pass over the row compacts, in
-//     position order, the keys of higher bins (certainly kept) and collects
-//     the keys of that bin as candidates in shared memory.  The candidates are
-//     resolved exactly in shared memory (radix on the low 21 bits, ties to the
-//     lower position) and the two ascending lists are merged.  If the bin holds
-//     more candidates than fit, the row falls back to the path below.
-//   * no histogram: three histogram passes (11 + 11 + 10 bits) find the k-th
-//     key, and a fourth pass compacts the kept positions in order.
-// Either way the pass that writes the output also forms Z_k = sum_kept
-// e^{s-m} and Z_tail = sum_dropped e^{s-m}; the tail mass is
-// Z_tail / (Z_k + Z_tail), formed from the dropped terms directly.
+// the k-th largest is found exactly by radix selection on the key bits.  Pass
+// 1 builds the histogram of the top 11 key bits and the row maximum; the bin
+// holding the k-th key is read off the histogram.  Pass 2 compacts, in
+// position order, the keys of higher bins (certainly kept) and collects the
+// keys of that bin as candidates in shared memory; the candidates are
+// resolved exactly there (radix on the low 21 bits, ties to the lower
+// position) and the two ascending lists are merged.  The row is read from L2
+// (the scorer keeps the K stream out of L2), with 8 float4 loads per thread
+// in flight.  A boundary bin with more candidates than fit falls back to
+// three histogram passes (11 + 11 + 10 bits) and an ordered compaction pass.
+// The pass that writes the output also forms Z_k = sum_kept e^{s-m} and
+// Z_tail = sum_dropped e^{s-m}; the tail mass is Z_tail / (Z_k + Z_tail),
+// formed from the dropped terms directly.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -86,19 +84,21 @@ __device__ void find_bin(const uint32_t *hist, int nbins, uint32_t need, uint32_
     __syncthreads();
 }
 
-// Calls f(i, s[i]) for every i < n, 16 elements per thread per round.
+constexpr int kBatch = 8;  // float4 loads in flight per thread
+
+// Calls f(i, s[i]) for every i < n, 4 * kBatch elements per thread per round.
 template <typename F>
 __device__ __forceinline__ void visit_row(const float *s, int n, F &&f) {
     const int n4 = n >> 2;
     const float4 *s4 = reinterpret_cast<const float4 *>(s);
     const int stride = blockDim.x;
     int i = threadIdx.x;
-    for (; i + 3 * stride < n4; i += 4 * stride) {
-        float4 v[4];
+    for (; i + (kBatch - 1) * stride < n4; i += kBatch * stride) {
+        float4 v[kBatch];
 #pragma unroll
-        for (int u = 0; u < 4; u++) v[u] = __ldcg(s4 + i + u * stride);
+        for (int u = 0; u < kBatch; u++) v[u] = __ldcg(s4 + i + u * stride);
 #pragma unroll
-        for (int u = 0; u < 4; u++) {
+        for (int u = 0; u < kBatch; u++) {
             const int e = 4 * (i + u * stride);
             f(e, v[u].x);
             f(e + 1, v[u].y);
@@ -167,8 +167,8 @@ __device__ void select_all(const SelectParams &p, int row, int vis, float m, con
     finish_row(p, row, m, zk, 0.f, vis, vis, sm);
 }
 
-// Three histogram passes and an ordered compaction pass (no histogram given,
-// or too many candidates in the boundary bin).
+// Three histogram passes and an ordered compaction pass (too many candidates
+// in the boundary bin).
 __device__ void select_multipass(const SelectParams &p, int row, int vis, const SelectSmem &sm) {
     const float *s = p.scores + (size_t)row * p.ld;
     const int k = p.k;
@@ -293,24 +293,20 @@ __global__ void __launch_bounds__(kSelectThreads) select_topk(SelectParams p) {
     const int k = p.k;
     const float *s = p.scores + (size_t)row * p.ld;
 
-    if (!p.rowhist) {
-        if (k >= vis) {
-            float m = -INFINITY;
-            visit_row(s, vis, [&](int, float x) { m = fmaxf(m, x); });
-            m = block_max(m, sm.red);
-            select_all(p, row, vis, m, sm);
-        } else {
-            select_multipass(p, row, vis, sm);
-        }
-        return;
-    }
-
-    const float m = key_to_float(p.rowmax[row]);
-    if (k >= vis) {
+    // pass 1: histogram of the top 11 key bits and the row maximum
+    for (int i = threadIdx.x; i < 2048; i += blockDim.x) sm.hist[i] = 0u;
+    __syncthreads();
+    const bool count = k < vis;
+    float m = -INFINITY;
+    visit_row(s, vis, [&](int, float x) {
+        m = fmaxf(m, x);
+        if (count) atomicAdd(&sm.hist[order_key(x) >> 21], 1u);
+    });
+    m = block_max(m, sm.red);
+    if (!count) {
         select_all(p, row, vis, m, sm);
         return;
     }
-    for (int i = threadIdx.x; i < 2048; i += blockDim.x) sm.hist[i] = p.rowhist[(size_t)row * 2048 + i];
     __syncthreads();
     find_bin(sm.hist, 2048, (uint32_t)k, sm.tmp, &sm.scal[0], &sm.scal[1]);
     const uint32_t b1 = sm.scal[0], above = sm.scal[1], ncand = sm.hist[b1];
@@ -320,49 +316,57 @@ __global__ void __launch_bounds__(kSelectThreads) select_topk(SelectParams p) {
         return;
     }
 
-    // one pass: keys of higher bins go to list A, keys of bin b1 to the candidates
+    // pass 2: keys of higher bins go to list A (in position order), keys of
+    // bin b1 to the candidates; kBatch tiles of loads are issued before
+    // their prefix sums
     uint32_t base_a = 0u, base_c = 0u;
     float zk = 0.f, zt = 0.f;
-    for (int tile = 0; tile < vis; tile += 4 * blockDim.x) {
-        const int i0 = tile + 4 * threadIdx.x;
-        float x[4];
-        load4(s, i0, vis, x);
-        uint32_t key[4], cnt = 0u;
+    const int tile_len = 4 * blockDim.x;
+    for (int base = 0; base < vis; base += kBatch * tile_len) {
+        float x[kBatch][4];
 #pragma unroll
-        for (int j = 0; j < 4; j++) {
-            key[j] = order_key(x[j]);
-            if (i0 + j < vis) cnt += (key[j] >> 21) > b1 ? 1u : ((key[j] >> 21) == b1 ? 0x10000u : 0u);
-        }
-        uint32_t tot;
-        const uint32_t ex = block_excl_scan(cnt, sm.tmp, &tot);
-        uint32_t pa = base_a + (ex & 0xffffu), pc = base_c + (ex >> 16);
+        for (int u = 0; u < kBatch; u++) load4(s, base + u * tile_len + 4 * threadIdx.x, vis, x[u]);
 #pragma unroll
-        for (int j = 0; j < 4; j++) {
-            if (i0 + j >= vis) continue;
-            const uint32_t bin = key[j] >> 21;
-            if (bin > b1) {
-                const float e = __expf(x[j] - m);
-                if (pa < above) {  // always true unless the histogram is wrong
-                    a_idx[pa] = i0 + j;
-                    a_w[pa] = e;
-                }
-                pa++;
-                zk += e;
-            } else if (bin == b1) {
-                if (pc < ncand) {
-                    c_key[pc] = key[j];
-                    c_idx[pc] = i0 + j;
-                }
-                pc++;
-            } else {
-                zt += __expf(x[j] - m);
+        for (int u = 0; u < kBatch; u++) {
+            const int i0 = base + u * tile_len + 4 * threadIdx.x;
+            if (base + u * tile_len >= vis) break;  // uniform across the block
+            uint32_t key[4], cnt = 0u;
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                key[j] = order_key(x[u][j]);
+                if (i0 + j < vis) cnt += (key[j] >> 21) > b1 ? 1u : ((key[j] >> 21) == b1 ? 0x10000u : 0u);
             }
+            uint32_t tot;
+            const uint32_t ex = block_excl_scan(cnt, sm.tmp, &tot);
+            uint32_t pa = base_a + (ex & 0xffffu), pc = base_c + (ex >> 16);
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                if (i0 + j >= vis) continue;
+                const uint32_t bin = key[j] >> 21;
+                if (bin > b1) {
+                    const float e = __expf(x[u][j] - m);
+                    if (pa < above) {  // always true unless the histogram is wrong
+                        a_idx[pa] = i0 + j;
+                        a_w[pa] = e;
+                    }
+                    pa++;
+                    zk += e;
+                } else if (bin == b1) {
+                    if (pc < ncand) {
+                        c_key[pc] = key[j];
+                        c_idx[pc] = i0 + j;
+                    }
+                    pc++;
+                } else {
+                    zt += __expf(x[u][j] - m);
+                }
+            }
+            base_a += tot & 0xffffu;
+            base_c += tot >> 16;
         }
-        base_a += tot & 0xffffu;
-        base_c += tot >> 16;
     }
     if (base_a != above || base_c != ncand) {
-        // the histogram does not describe these scores (a library bug); recompute safely
+        // the two passes disagree (a library bug); recompute safely
         if (threadIdx.x == 0) raise_status(p.status, TKA_DEV_INTERNAL);
         __syncthreads();
         select_multipass(p, row, vis, sm);

@@ -55,8 +55,7 @@ def test_workspace_size_layout(lib):
     n = bd.topk_attn_workspace_size(s, 2048)
     rows = 8 * 32
     # scores + weights + stats + partial (32 splits of 64 keys) + counters
-    # + the scorer's per-row radix histogram (2048 bins) and row maximum
-    want = rows * 32768 * 4 + rows * 2048 * 4 + rows * 16 + rows * 32 * 128 * 4 + 1024 + rows * 2048 * 4 + rows * 4
+    want = rows * 32768 * 4 + rows * 2048 * 4 + rows * 16 + rows * 32 * 128 * 4 + 1024
     assert n == want
     assert bd.topk_attn_workspace_size(shape(L=1001), 7) % 256 == 0
 
