@@ -51,6 +51,8 @@ def parse_args():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch size (smaller cases for profiling)")
     return ap.parse_args()
 
 
@@ -205,9 +207,10 @@ def dist_setup(args):
     return world, rank, local
 
 
-def make_inputs(cfg, rank):
+def make_inputs(cfg, rank, batch=None):
     # each rank decodes its own batch (weak scaling); rank 0 draws the tested workload
-    return workloads.config_workload(cfg, seed=1000 + cfg + 7919 * rank)
+    over = {} if batch is None else {"B": batch}
+    return workloads.config_workload(cfg, seed=1000 + cfg + 7919 * rank, **over)
 
 
 def run_ours(args, world, rank, local):
@@ -216,7 +219,7 @@ def run_ours(args, world, rank, local):
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    w = make_inputs(args.config, rank)
+    w = make_inputs(args.config, rank, args.batch)
     q, kc, vc, lens = (w.q.to(dev), w.k_cache.to(dev), w.v_cache.to(dev), w.seq_lens.to(dev))
     rows = w.B * w.Q * w.Hq
     block = w.variant == "block"
@@ -353,7 +356,7 @@ def run_ours(args, world, rank, local):
         res["stage_us"] = {n: stage_tot[j] / K * 1e3 for j, n in enumerate(["score", "select", "gather"])}
         score_s = stage_tot[0] / K / 1e3
         achieved = dominant_bytes / score_s / 1e9
-        traffic = score_traffic(os.path.join(ROOT, "exact_top_sparse_score_b200", "csrc", "score.cu"))
+        traffic = score_traffic(os.path.join(ROOT, "exact_top_sparse_score_b200", "csrc", "score_tc.cu"))
         res["roofline"] = {"kernel": "score", "bound": "hbm", "achieved": achieved, "peak": peak,
                            "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
                            else "fallback 6.65 TB/s", "unit": "GB/s", "frac": achieved / peak,
@@ -373,7 +376,7 @@ def run_reference(args, rank):
     if rank != 0:
         return None
     import oracle
-    w = make_inputs(args.config, 0)
+    w = make_inputs(args.config, 0, args.batch)
     rows = w.B * w.Q * w.Hq
     k = w.k
 

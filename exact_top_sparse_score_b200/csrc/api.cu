@@ -52,6 +52,16 @@ cudaError_t record(const tka_event_t *events, int i, cudaStream_t s) {
     return cudaEventRecord(reinterpret_cast<cudaEvent_t>(events[i]), s);
 }
 
+struct RecordCtx {
+    const tka_event_t *events;
+    int i;
+    cudaStream_t s;
+};
+cudaError_t record_hook(void *ctx) {
+    const RecordCtx *c = static_cast<const RecordCtx *>(ctx);
+    return record(c->events, c->i, c->s);
+}
+
 float resolve_scale(const tka_shape *s) { return s->scale > 0.f ? s->scale : 1.f / sqrtf((float)s->d); }
 
 // Shape checks shared by both variants.
@@ -173,7 +183,6 @@ tka_status topk_attn_decode_staged(const tka_shape *shape, const void *q, const 
     // the tensor map addresses cache rows with int32 coordinates
     const bool tc = score_tc_supported(shape->dtype, NQ) &&
                     (long long)shape->B * shape->Hkv * shape->L_max < (1LL << 31);
-    if (record(events, 0, s) != cudaSuccess) return TKA_ERR_CUDA;
     if (tc) {
         ScoreTcParams tp;
         tp.status = dev->status;
@@ -182,8 +191,13 @@ tka_status topk_attn_decode_staged(const tka_shape *shape, const void *q, const 
         tp.B = shape->B; tp.Q = shape->Q; tp.Hq = shape->Hq; tp.Hkv = shape->Hkv; tp.G = G;
         tp.L_max = shape->L_max; tp.ld = L.ld; tp.NQ = NQ;
         tp.scale = resolve_scale(shape);
-        if (launch_score_tc(tp, q, k_cache, dev->num_sms, s) != cudaSuccess) return TKA_ERR_CUDA;
+        RecordCtx rc{events, 0, s};
+        ScoreTcHook hook;
+        hook.fn = record_hook;
+        hook.ctx = &rc;
+        if (launch_score_tc(tp, q, k_cache, dev->num_sms, s, hook) != cudaSuccess) return TKA_ERR_CUDA;
     } else {
+        if (record(events, 0, s) != cudaSuccess) return TKA_ERR_CUDA;
         ScoreParams sp;
         sp.status = dev->status;
         sp.q = q;

@@ -84,8 +84,14 @@ struct BlockAttnParams {
 
 cudaError_t launch_score(const ScoreParams &p, int num_sms, cudaStream_t stream);
 bool score_tc_supported(int dtype, int NQ);
+// Called right before a kernel launch, after all host-side preparation
+// (tensor-map encoding, function attributes); a null fn is skipped.
+struct ScoreTcHook {
+    cudaError_t (*fn)(void *ctx) = nullptr;
+    void *ctx = nullptr;
+};
 cudaError_t launch_score_tc(const ScoreTcParams &p, const void *q, const void *k_cache, int num_sms,
-                            cudaStream_t stream);
+                            cudaStream_t stream, const ScoreTcHook &hook);
 cudaError_t launch_select(const SelectParams &p, cudaStream_t stream);
 size_t select_smem_bytes(int k);
 cudaError_t launch_gather(const GatherParams &p, cudaStream_t stream);

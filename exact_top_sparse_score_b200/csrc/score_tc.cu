@@ -293,10 +293,21 @@ size_t smem_bytes() {
 
 template <int N>
 cudaError_t launch_n(const CUtensorMap &km, const CUtensorMap &qm, const ScoreTcParams &p, int num_sms,
-                     cudaStream_t stream) {
+                     cudaStream_t stream, const ScoreTcHook &hook) {
     const size_t smem = smem_bytes<N>();
-    cudaError_t e = cudaFuncSetAttribute(score_tc<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static bool attr_set[64] = {};  // per device: the shared-memory opt-in is a function attribute
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+        e = cudaFuncSetAttribute(score_tc<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+    if (hook.fn) {
+        e = hook.fn(hook.ctx);  // e.g. a timing event, right before the launch
+        if (e != cudaSuccess) return e;
+    }
     score_tc<N><<<num_sms, kThreads, smem, stream>>>(km, qm, p);
     return cudaGetLastError();
 }
@@ -306,7 +317,7 @@ cudaError_t launch_n(const CUtensorMap &km, const CUtensorMap &qm, const ScoreTc
 bool score_tc_supported(int dtype, int NQ) { return dtype == TKA_BF16 && NQ <= 128 && encode_fn() != nullptr; }
 
 cudaError_t launch_score_tc(const ScoreTcParams &p, const void *q, const void *k_cache, int num_sms,
-                            cudaStream_t stream) {
+                            cudaStream_t stream, const ScoreTcHook &hook) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return cudaErrorNotSupported;
     CUtensorMap km, qm;
@@ -333,10 +344,10 @@ cudaError_t launch_score_tc(const ScoreTcParams &p, const void *q, const void *k
             return cudaErrorInvalidValue;
     }
     const int NQ = p.NQ;
-    if (NQ <= 16) return launch_n<16>(km, qm, p, num_sms, stream);
-    if (NQ <= 32) return launch_n<32>(km, qm, p, num_sms, stream);
-    if (NQ <= 64) return launch_n<64>(km, qm, p, num_sms, stream);
-    return launch_n<128>(km, qm, p, num_sms, stream);
+    if (NQ <= 16) return launch_n<16>(km, qm, p, num_sms, stream, hook);
+    if (NQ <= 32) return launch_n<32>(km, qm, p, num_sms, stream, hook);
+    if (NQ <= 64) return launch_n<64>(km, qm, p, num_sms, stream, hook);
+    return launch_n<128>(km, qm, p, num_sms, stream, hook);
 }
 
 }  // namespace tka

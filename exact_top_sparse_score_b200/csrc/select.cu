@@ -7,20 +7,29 @@
 // the discarded mass is the Top-k tail mass of "A Mathematical Theory of
 // Top-k Sparse Attention via Total Variation Distance" (abstract).
 //
-// One CTA per row.  Scores are compared as order-preserving uint32 keys, so
-// the k-th largest is found exactly by radix selection on the key bits.  Pass
-// 1 builds the histogram of the top 11 key bits and the row maximum; the bin
-// holding the k-th key is read off the histogram.  Pass 2 compacts, in
-// position order, the keys of higher bins (certainly kept) and collects the
-// keys of that bin as candidates in shared memory; the candidates are
-// resolved exactly there (radix on the low 21 bits, ties to the lower
-// position) and the two ascending lists are merged.  The row is read from L2
-// (the scorer keeps the K stream out of L2), with 8 float4 loads per thread
-// in flight.  A boundary bin with more candidates than fit falls back to
-// three histogram passes (11 + 11 + 10 bits) and an ordered compaction pass.
-// The pass that writes the output also forms Z_k = sum_kept e^{s-m} and
-// Z_tail = sum_dropped e^{s-m}; the tail mass is Z_tail / (Z_k + Z_tail),
-// formed from the dropped terms directly.
+// One CTA (32 warps) per row; every warp owns a contiguous
+// segment of the row, lane l holding positions l, l + 32, ... of it, so a warp
+// compacts 32 consecutive positions at a time with one ballot.  A segment is
+// streamed in batches of 32 x 32 positions with all loads of a batch in
+// flight together (a segment that fits one batch is read once and kept in
+// registers for all passes); the rows come from L2.  Scores are compared as
+// order-preserving uint32 keys:
+//   pass 1  the row maximum and the histogram of the top 11 key bits of a
+//           position-uniform 1/8 sample give a bin range that holds the k-th
+//           key with high probability;
+//   pass 2  keys above the range are counted, keys inside it are collected
+//           (in position order) into per-warp candidate lists;
+//   exact radix selection over the candidates' full keys (11 + 11 + 10 bits)
+//           yields the k-th key T and how many of the keys equal to T are
+//           kept (the lowest positions);
+//   pass 3  every key is tested against that exact rule and the kept
+//           positions are written straight to their ascending slots (warp
+//           prefix sums plus per-warp offsets), while Z_k = sum_kept e^{s-m}
+//           and Z_tail = sum_dropped e^{s-m} are accumulated; the tail mass
+//           Z_tail / (Z_k + Z_tail) is formed from the dropped terms directly.
+// If the sampled range misses the k-th key, or a warp collects more
+// candidates than fit, the row falls back to three exact histogram passes and
+// an ordered compaction pass over the row.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -28,12 +37,12 @@ namespace tka {
 
 namespace {
 
-constexpr int kSelectThreads = 512;
-constexpr int kCandCap = 4096;
+constexpr int kSelectThreads = 1024;
+constexpr int kWarps = kSelectThreads / 32;
+constexpr int kWarpCand = 256;                  // candidates per warp held in shared memory
+constexpr int kHeld = 32;                       // scores per lane held in registers per batch
+constexpr int kSampleMinLen = 16384;            // rows this long histogram a 1/8 sample in pass 1
 
-__device__ __forceinline__ float key_to_float(uint32_t k) {
-    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
-}
 
 // Exclusive prefix sum of one value per thread over the block; *total gets
 // the block sum.  `tmp` holds >= 32 words of shared memory.
@@ -257,30 +266,22 @@ __device__ void select_multipass(const SelectParams &p, int row, int vis, const 
     finish_row(p, row, m, zk, zt, base_sel, (uint32_t)k, sm);
 }
 
-// Number of elements of the ascending array a[0..n) that are < x.
-__device__ __forceinline__ int lower_bound(const int32_t *a, int n, int32_t x) {
-    int lo = 0, hi = n;
-    while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (a[mid] < x)
-            lo = mid + 1;
-        else
-            hi = mid;
-    }
-    return lo;
+__device__ __forceinline__ uint32_t lanemask_lt() {
+    uint32_t m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
 }
 
-__global__ void __launch_bounds__(kSelectThreads) select_topk(SelectParams p) {
-    extern __shared__ uint32_t dyn[];
+__global__ void __launch_bounds__(kSelectThreads, 1) select_topk(SelectParams p) {
+    extern __shared__ __align__(16) uint32_t dyn[];
     SelectSmem sm;
-    sm.hist = dyn;
-    sm.tmp = dyn + 2048;
-    sm.red = reinterpret_cast<float *>(dyn + 2048 + 32);
-    sm.scal = dyn + 2048 + 64;
-    int32_t *a_idx = reinterpret_cast<int32_t *>(dyn + 2048 + 64 + 8);  // [k]
-    float *a_w = reinterpret_cast<float *>(a_idx + p.k);                 // [k]
-    uint32_t *c_key = reinterpret_cast<uint32_t *>(a_w + p.k);           // [kCandCap]
-    int32_t *c_idx = reinterpret_cast<int32_t *>(c_key + kCandCap);      // [kCandCap]
+    sm.hist = dyn;                                                   // [2048]
+    sm.tmp = dyn + 2048;                                             // [32]
+    sm.red = reinterpret_cast<float *>(dyn + 2048 + 32);             // [32]
+    sm.scal = dyn + 2048 + 64;                                       // [8]
+    uint32_t *wstat = dyn + 2048 + 72;                               // [kWarps][8]
+    uint32_t *wc_key = wstat + kWarps * 8;                           // [kWarps][kWarpCand]
+    int32_t *wc_pos = reinterpret_cast<int32_t *>(wc_key + kWarps * kWarpCand);  // [kWarps][kWarpCand]
 
     const int row = blockIdx.x;
     const int b = row / (p.Q * p.Hq), qpos = (row / p.Hq) % p.Q;
@@ -292,166 +293,232 @@ __global__ void __launch_bounds__(kSelectThreads) select_topk(SelectParams p) {
     const int vis = visible_keys(seq_len, p.Q, qpos);
     const int k = p.k;
     const float *s = p.scores + (size_t)row * p.ld;
-
-    // pass 1: histogram of the top 11 key bits and the row maximum
-    for (int i = threadIdx.x; i < 2048; i += blockDim.x) sm.hist[i] = 0u;
-    __syncthreads();
-    const bool count = k < vis;
-    float m = -INFINITY;
-    visit_row(s, vis, [&](int, float x) {
-        m = fmaxf(m, x);
-        if (count) atomicAdd(&sm.hist[order_key(x) >> 21], 1u);
-    });
-    m = block_max(m, sm.red);
-    if (!count) {
+    if (k >= vis) {  // every visible key is kept
+        float m = -INFINITY;
+        visit_row(s, vis, [&](int, float x) { m = fmaxf(m, x); });
+        m = block_max(m, sm.red);
         select_all(p, row, vis, m, sm);
         return;
     }
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t lt = lanemask_lt();
+    // this warp's contiguous segment; lane l holds positions lo + 32 r + l of
+    // each batch of 32 * kHeld positions
+    const int seg = (((vis + kWarps - 1) / kWarps) + 31) & ~31;
+    const int lo = min(vis, warp * seg), hi = min(vis, lo + seg);
+    const int nbatch = (hi - lo + 32 * kHeld - 1) / (32 * kHeld);
+    const bool resident = nbatch <= 1;  // the whole segment fits in registers
+    float x[kHeld];
+    auto load_batch = [&](int bi) {
+        const int p0 = lo + bi * 32 * kHeld + lane;
+#pragma unroll
+        for (int r = 0; r < kHeld; r++) x[r] = p0 + 32 * r < hi ? __ldcg(s + p0 + 32 * r) : 0.f;
+    };
+    if (resident) load_batch(0);
+
+    // pass 1: the row maximum, and the histogram of the top 11 key bits of a
+    // position-uniform sample (positions that are multiples of 8; every
+    // position on short rows) -- the threshold is looked for there
+    for (int i = threadIdx.x; i < 2048; i += kSelectThreads) sm.hist[i] = 0u;
     __syncthreads();
-    find_bin(sm.hist, 2048, (uint32_t)k, sm.tmp, &sm.scal[0], &sm.scal[1]);
-    const uint32_t b1 = sm.scal[0], above = sm.scal[1], ncand = sm.hist[b1];
-    if (ncand > (uint32_t)kCandCap) {
-        __syncthreads();
-        select_multipass(p, row, vis, sm);
-        return;
+    const bool sampled = vis >= kSampleMinLen;
+    const bool sampler = !sampled || (lane & 7) == 0;  // lo is a multiple of 32
+    float m = -INFINITY;
+    for (int bi = 0; bi < nbatch; bi++) {
+        if (!resident) load_batch(bi);
+        const int p0 = lo + bi * 32 * kHeld + lane;
+#pragma unroll
+        for (int r = 0; r < kHeld; r++) {
+            if (p0 + 32 * r < hi) {
+                m = fmaxf(m, x[r]);
+                if (sampler) atomicAdd(&sm.hist[order_key(x[r]) >> 21], 1u);
+            }
+        }
+    }
+    m = block_max(m, sm.red);
+    __syncthreads();
+    // bins above b_hi are kept; bins [b_lo, b_hi] hold the candidates.  On the
+    // sample the k-th key has rank about k/8; the range is widened by 4
+    // binomial standard deviations each way and checked exactly below.
+    uint32_t b_hi, b_lo;
+    {
+        const int slog = sampled ? 3 : 0;
+        const uint32_t nsample = (uint32_t)((vis + (1 << slog) - 1) >> slog);
+        const float ks = (float)k / (float)(1 << slog);
+        const float margin = sampled ? 4.f * sqrtf(ks) + 4.f : 0.f;
+        const uint32_t need_hi = (uint32_t)fmaxf(1.f, floorf(ks - margin));
+        const uint32_t need_lo = (uint32_t)fminf((float)nsample, ceilf(ks + margin));
+        find_bin(sm.hist, 2048, need_hi, sm.tmp, &sm.scal[0], &sm.scal[1]);
+        b_hi = sm.scal[0];
+        find_bin(sm.hist, 2048, max(need_lo, need_hi), sm.tmp, &sm.scal[0], &sm.scal[1]);
+        b_lo = sm.scal[0];
     }
 
-    // pass 2: keys of higher bins go to list A (in position order), keys of
-    // bin b1 to the candidates; kBatch tiles of loads are issued before
-    // their prefix sums
-    uint32_t base_a = 0u, base_c = 0u;
-    float zk = 0.f, zt = 0.f;
-    const int tile_len = 4 * blockDim.x;
-    for (int base = 0; base < vis; base += kBatch * tile_len) {
-        float x[kBatch][4];
+    // pass 2: count the keys of bins above b_hi; collect the keys of bins
+    // [b_lo, b_hi], in position order, into this warp's candidate list
+    uint32_t nwin = 0u, ncw = 0u;
+    uint32_t *my_key = wc_key + warp * kWarpCand;
+    int32_t *my_pos = wc_pos + warp * kWarpCand;
+    for (int bi = 0; bi < nbatch; bi++) {
+        if (!resident) load_batch(bi);
+        const int p0 = lo + bi * 32 * kHeld + lane;
 #pragma unroll
-        for (int u = 0; u < kBatch; u++) load4(s, base + u * tile_len + 4 * threadIdx.x, vis, x[u]);
-#pragma unroll
-        for (int u = 0; u < kBatch; u++) {
-            const int i0 = base + u * tile_len + 4 * threadIdx.x;
-            if (base + u * tile_len >= vis) break;  // uniform across the block
-            uint32_t key[4], cnt = 0u;
-#pragma unroll
-            for (int j = 0; j < 4; j++) {
-                key[j] = order_key(x[u][j]);
-                if (i0 + j < vis) cnt += (key[j] >> 21) > b1 ? 1u : ((key[j] >> 21) == b1 ? 0x10000u : 0u);
-            }
-            uint32_t tot;
-            const uint32_t ex = block_excl_scan(cnt, sm.tmp, &tot);
-            uint32_t pa = base_a + (ex & 0xffffu), pc = base_c + (ex >> 16);
-#pragma unroll
-            for (int j = 0; j < 4; j++) {
-                if (i0 + j >= vis) continue;
-                const uint32_t bin = key[j] >> 21;
-                if (bin > b1) {
-                    const float e = __expf(x[u][j] - m);
-                    if (pa < above) {  // always true unless the histogram is wrong
-                        a_idx[pa] = i0 + j;
-                        a_w[pa] = e;
-                    }
-                    pa++;
-                    zk += e;
-                } else if (bin == b1) {
-                    if (pc < ncand) {
-                        c_key[pc] = key[j];
-                        c_idx[pc] = i0 + j;
-                    }
-                    pc++;
-                } else {
-                    zt += __expf(x[u][j] - m);
+        for (int r = 0; r < kHeld; r++) {
+            const bool valid = p0 + 32 * r < hi;
+            const uint32_t key = order_key(x[r]);
+            const uint32_t bin = key >> 21;
+            nwin += __popc(__ballot_sync(0xffffffffu, valid && bin > b_hi));
+            const bool cand = valid && bin >= b_lo && bin <= b_hi;
+            const uint32_t cb = __ballot_sync(0xffffffffu, cand);
+            if (cand) {
+                const uint32_t slot = ncw + __popc(cb & lt);
+                if (slot < (uint32_t)kWarpCand) {
+                    my_key[slot] = key;
+                    my_pos[slot] = p0 + 32 * r;
                 }
             }
-            base_a += tot & 0xffffu;
-            base_c += tot >> 16;
+            ncw += __popc(cb);
         }
     }
-    if (base_a != above || base_c != ncand) {
-        // the two passes disagree (a library bug); recompute safely
-        if (threadIdx.x == 0) raise_status(p.status, TKA_DEV_INTERNAL);
+    if (lane == 0) {
+        wstat[warp * 8 + 0] = nwin;
+        wstat[warp * 8 + 1] = ncw;
+    }
+    __syncthreads();
+    uint32_t above = 0u, ncand = 0u;
+    bool overflow = false;
+    for (int w = 0; w < kWarps; w++) {
+        above += wstat[w * 8 + 0];
+        ncand += wstat[w * 8 + 1];
+        overflow |= wstat[w * 8 + 1] > (uint32_t)kWarpCand;
+    }
+    if (overflow || above >= (uint32_t)k || above + ncand < (uint32_t)k) {
+        // the sampled range missed the k-th key or a warp's list overflowed:
+        // take the exact multi-pass route
         __syncthreads();
         select_multipass(p, row, vis, sm);
         return;
     }
-    __syncthreads();
 
-    // resolve the boundary bin: r of its ncand keys are kept
-    const uint32_t r = (uint32_t)k - above;
-    uint32_t *hist = sm.hist;
-    for (int i = threadIdx.x; i < 2048; i += blockDim.x) hist[i] = 0u;
-    __syncthreads();
-    for (uint32_t c = threadIdx.x; c < ncand; c += blockDim.x) atomicAdd(&hist[(c_key[c] >> 10) & 0x7ffu], 1u);
-    __syncthreads();
-    find_bin(hist, 2048, r, sm.tmp, &sm.scal[0], &sm.scal[1]);
-    const uint32_t b2 = sm.scal[0];
-    uint32_t gt = sm.scal[1];
-    const uint32_t pre = (b1 << 11) | b2;
-    for (int i = threadIdx.x; i < 2048; i += blockDim.x) hist[i] = 0u;
-    __syncthreads();
-    for (uint32_t c = threadIdx.x; c < ncand; c += blockDim.x)
-        if ((c_key[c] >> 10) == pre) atomicAdd(&hist[c_key[c] & 0x3ffu], 1u);
-    __syncthreads();
-    find_bin(hist, 1024, r - gt, sm.tmp, &sm.scal[0], &sm.scal[1]);
-    const uint32_t b3 = sm.scal[0];
-    gt += sm.scal[1];
-    const uint32_t T = (pre << 10) | b3, n_eq = hist[b3], r_eq = r - gt;
-    const bool rank_ties = n_eq != r_eq;
-
-    // compact the chosen candidates in place (candidates are in position order)
-    uint32_t base_b = 0u, base_eq = 0u;
-    for (uint32_t c0 = 0; c0 < ncand; c0 += blockDim.x) {
-        const uint32_t c = c0 + threadIdx.x;
-        const bool have = c < ncand;
-        const uint32_t key = have ? c_key[c] : 0u;
-        const int32_t pos = have ? c_idx[c] : 0;
-        uint32_t eq_total = 0u, eq_rank = base_eq;
-        if (rank_ties) eq_rank += block_excl_scan(have && key == T ? 1u : 0u, sm.tmp, &eq_total);
-        const bool chosen = have && (key == T ? (!rank_ties || eq_rank < r_eq) : key > T);
-        uint32_t tot;
-        const uint32_t dst = base_b + block_excl_scan(chosen ? 1u : 0u, sm.tmp, &tot);  // ends with a barrier
-        if (have) {
-            const float e = __expf(key_to_float(key) - m);
-            if (chosen) {
-                c_idx[dst] = pos;
-                reinterpret_cast<float *>(c_key)[dst] = e;
-                zk += e;
-            } else {
-                zt += e;
-            }
+    // exact radix selection over the candidates' full 32-bit keys (11 + 11 +
+    // 10 bits): r of them are kept
+    const uint32_t need = (uint32_t)k - above;
+    uint32_t pre = 0u, gt = 0u, T = 0u;
+    for (int level = 0; level < 3; level++) {
+        const int shift = level == 0 ? 21 : (level == 1 ? 10 : 0);
+        const int nb = level == 2 ? 1024 : 2048;
+        for (int i = threadIdx.x; i < 2048; i += kSelectThreads) sm.hist[i] = 0u;
+        __syncthreads();
+        for (int e = threadIdx.x; e < kWarps * kWarpCand; e += kSelectThreads) {
+            const int w = e / kWarpCand, i = e - w * kWarpCand;
+            if ((uint32_t)i >= wstat[w * 8 + 1]) continue;
+            const uint32_t key = wc_key[e];
+            if (level == 0 || (key >> (shift + (level == 1 ? 11 : 10))) == pre)
+                atomicAdd(&sm.hist[(key >> shift) & (uint32_t)(nb - 1)], 1u);
         }
         __syncthreads();
-        base_b += tot;
-        base_eq += eq_total;
+        find_bin(sm.hist, nb, need - gt, sm.tmp, &sm.scal[0], &sm.scal[1]);
+        const uint32_t bin = sm.scal[0];
+        gt += sm.scal[1];
+        if (level < 2)
+            pre = (pre << (level == 0 ? 0 : 11)) | bin;
+        else
+            T = (pre << 10) | bin;
     }
-    // merge the two ascending lists into the output
+    // keys equal to T: the first r_eq of them (by position) are kept
+    const uint32_t r_eq = need - gt;
+
+    // per warp: candidates above T and ties at T, then output offsets
+    {
+        uint32_t g = 0u, t = 0u;
+        for (uint32_t i = lane; i < ncw; i += 32) {
+            g += my_key[i] > T;
+            t += my_key[i] == T;
+        }
+        g = warp_sum(g);
+        t = warp_sum(t);
+        if (lane == 0) {
+            wstat[warp * 8 + 2] = g;
+            wstat[warp * 8 + 3] = t;
+        }
+    }
+    __syncthreads();
+    uint32_t out_run = 0u, tie_run = 0u, n_eq = 0u;
+    for (int w = 0; w < kWarps; w++) {
+        const uint32_t tie_w = wstat[w * 8 + 3];
+        if (w < warp) {
+            const uint32_t kept_ties = r_eq > tie_run ? min(tie_w, r_eq - tie_run) : 0u;
+            out_run += wstat[w * 8 + 0] + wstat[w * 8 + 2] + kept_ties;
+            tie_run += tie_w;
+        }
+        n_eq += tie_w;
+    }
+    const bool rank_ties = n_eq != r_eq;
+    const uint32_t out_begin = out_run;
+
+    // pass 3: the exact rule -- key > T, or key == T among the first r_eq
+    // ties -- written straight to the final ascending positions, with the
+    // softmax sums of kept and dropped keys
     int32_t *idx = p.idx + (size_t)row * k;
     float *wv = p.w + (size_t)row * k;
-    const float *b_w = reinterpret_cast<const float *>(c_key);
-    const int na = (int)above, nb = (int)base_b;
-    for (int i = threadIdx.x; i < na; i += blockDim.x) {
-        const int pos = i + lower_bound(c_idx, nb, a_idx[i]);
-        idx[pos] = a_idx[i];
-        wv[pos] = a_w[i];
+    float zk = 0.f, zt = 0.f;
+    for (int bi = 0; bi < nbatch; bi++) {
+        if (!resident) load_batch(bi);
+        const int p0 = lo + bi * 32 * kHeld + lane;
+#pragma unroll
+        for (int r = 0; r < kHeld; r++) {
+            const bool valid = p0 + 32 * r < hi;
+            const uint32_t key = order_key(x[r]);
+            bool sel = valid && key > T;
+            if (rank_ties) {
+                const bool tie = valid && key == T;
+                const uint32_t tb = __ballot_sync(0xffffffffu, tie);
+                if (tie) sel = tie_run + __popc(tb & lt) < r_eq;
+                tie_run += __popc(tb);
+            } else {
+                sel = sel || (valid && key == T);
+            }
+            const uint32_t sb = __ballot_sync(0xffffffffu, sel);
+            if (valid) {
+                const float e = __expf(x[r] - m);
+                if (sel) {
+                    const uint32_t o = out_run + __popc(sb & lt);
+                    if (o < (uint32_t)k) {  // always true unless the counts above are wrong
+                        idx[o] = p0 + 32 * r;
+                        wv[o] = e;
+                    }
+                    zk += e;
+                } else {
+                    zt += e;
+                }
+            }
+            out_run += __popc(sb);
+        }
     }
-    for (int i = threadIdx.x; i < nb; i += blockDim.x) {
-        const int pos = i + lower_bound(a_idx, na, c_idx[i]);
-        idx[pos] = c_idx[i];
-        wv[pos] = b_w[i];
-    }
-    finish_row(p, row, m, zk, zt, above + base_b, (uint32_t)k, sm);
+    if (lane == 0) wstat[warp * 8 + 4] = out_run - out_begin;
+    __syncthreads();
+    uint32_t written = 0u;
+    for (int w = 0; w < kWarps; w++) written += wstat[w * 8 + 4];
+    finish_row(p, row, m, zk, zt, written, (uint32_t)k, sm);
 }
 
 }  // namespace
 
-size_t select_smem_bytes(int k) {
-    return (size_t)(2048 + 64 + 8) * 4 + (size_t)k * 8 + (size_t)kCandCap * 8;
+size_t select_smem_bytes(int) {
+    return (size_t)(2048 + 72 + kWarps * 8) * 4 + (size_t)kWarps * kWarpCand * 8;
 }
 
 cudaError_t launch_select(const SelectParams &p, cudaStream_t stream) {
     const int rows = p.B * p.Q * p.Hq;
     const size_t smem = select_smem_bytes(p.k);
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(select_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static bool attr_set[64] = {};  // per device: the shared-memory opt-in is a function attribute
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (smem > 48 * 1024 && (dev < 0 || dev >= 64 || !attr_set[dev])) {
+        e = cudaFuncSetAttribute(select_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
     select_topk<<<rows, kSelectThreads, smem, stream>>>(p);
     return cudaGetLastError();
