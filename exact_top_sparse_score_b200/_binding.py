@@ -53,6 +53,10 @@ def load_library() -> ctypes.CDLL:
         lib.topk_attn_decode_staged.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp,
                                                 ctypes.POINTER(_vp)]
         lib.topk_attn_decode_staged.restype = ctypes.c_int
+        lib.topk_attn_static_workspace_capacity.argtypes = []
+        lib.topk_attn_static_workspace_capacity.restype = _sz
+        lib.topk_attn_decode_static.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp]
+        lib.topk_attn_decode_static.restype = ctypes.c_int
         lib.topk_block_pool_keys.argtypes = [_shape_p, _vp, _vp, _i32, _vp, _vp]
         lib.topk_block_pool_keys.restype = ctypes.c_int
         lib.topk_block_attn_workspace_size.argtypes = [_shape_p, _i32, _i32]
@@ -195,6 +199,33 @@ def topk_attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tens
     if rc:
         raise TopkAttnError("topk_attn_decode", rc)
     return out, idx, tail_mass
+
+
+def topk_attn_decode_static(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, seq_lens: torch.Tensor,
+                            k: int, *, out: torch.Tensor, idx: torch.Tensor, tail_mass: Optional[torch.Tensor] = None,
+                            scale: float = 0.0, stream=None) -> None:
+    """topk_attn_decode on the library's built-in scratch array: the caller
+    passes every output buffer and nothing is allocated (no torch allocation
+    either).  Raises TopkAttnError (TKA_ERR_WORKSPACE) when the shape needs
+    more scratch than topk_attn_static_workspace_capacity()."""
+    lib = load_library()
+    shape = make_shape(q, k_cache, scale)
+    B, Q, Hq, d = q.shape
+    if seq_lens.dtype != torch.int32 or tuple(seq_lens.shape) != (B,):
+        raise TypeError("seq_lens must be int32 [B]")
+    _check_out("out", out, torch.float32, (B, Q, Hq, d))
+    _check_out("idx", idx, torch.int32, (B, Q, Hq, k))
+    _check_out("tail_mass", tail_mass, torch.float32, (B, Q, Hq))
+    _check_cuda(q=q, k_cache=k_cache, v_cache=v_cache, seq_lens=seq_lens, out=out, idx=idx, tail_mass=tail_mass)
+    rc = lib.topk_attn_decode_static(ctypes.byref(shape), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                     seq_lens.data_ptr(), k, out.data_ptr(), idx.data_ptr(), _ptr(tail_mass),
+                                     _stream(stream))
+    if rc:
+        raise TopkAttnError("topk_attn_decode_static", rc)
+
+
+def topk_attn_static_workspace_capacity() -> int:
+    return int(load_library().topk_attn_static_workspace_capacity())
 
 
 def topk_block_pool_keys(k_cache: torch.Tensor, seq_lens: torch.Tensor, block_size: int, *,

@@ -108,6 +108,24 @@ tka_status topk_attn_decode_staged(const tka_shape *shape, const void *q, const 
                                    int32_t *idx, float *tail_mass, void *workspace, size_t workspace_bytes,
                                    tka_stream_t stream, const tka_event_t events[4]);
 
+/* topk_attn_decode without a workspace argument, for callers that cannot
+ * allocate device memory (an engine that reserves all device memory for its
+ * own pool and forbids other allocations while serving, or a host runtime with
+ * no device allocator).  The pages describe no such call; it is a library
+ * convenience.  The scratch space is an array compiled into the library,
+ * topk_attn_static_workspace_capacity() bytes (48 MiB) on every GPU that loads
+ * it, held until the process exits.  The first call on a device (with that
+ * device current) looks up the array's device address; make that first call
+ * before any stream capture.  Every call on a device shares the array: calls
+ * whose work overlaps on the GPU race, so order them (one stream, or events).
+ * Shapes whose topk_attn_workspace_size() exceeds the capacity return
+ * TKA_ERR_WORKSPACE; other arguments are checked as in topk_attn_decode.
+ * Allocates nothing. */
+size_t topk_attn_static_workspace_capacity(void);
+tka_status topk_attn_decode_static(const tka_shape *shape, const void *q, const void *k_cache,
+                                   const void *v_cache, const int32_t *seq_lens, int32_t k, float *out,
+                                   int32_t *idx, float *tail_mass, tka_stream_t stream);
+
 /* MoBA block keys: block_keys[b, h, j, :] = mean of K[b, h, i, :] over the keys
  * of block j below seq_lens[b] (a partial last block is averaged over the keys
  * it holds; blocks past the end are written as zero).  block_keys is fp32
