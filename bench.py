@@ -10,7 +10,9 @@ L=32768, k=2048, bf16 cache.
 
 Prints ONE JSON line (rank 0).  Timing: W untimed warm-up steps, then exactly
 K timed steps, each bracketed by CUDA events on the launching stream, with an
-L2 flush (a 256 MiB write) between steps outside the events; the sum of the
+L2 flush between steps outside the events (a 256 MiB write, then a 256 MiB
+read, so that no dirty line of the flush buffer is left in L2 to be written
+back inside the timed region); the sum of the
 K step times, max over ranks.  Multi-GPU (torchrun) runs one independent
 replica per GPU (the path shards by sequence with no exchange): weak scaling.
 
@@ -230,7 +232,7 @@ def run_ours(args, world, rank, local):
                          dtype=torch.uint8, device=dev)
         out = torch.empty((w.B, w.Q, w.Hq, w.d), dtype=torch.float32, device=dev)
         bidx = torch.empty((w.B, w.Q, w.Hq, w.top_blocks + 1), dtype=torch.int32, device=dev)
-        launches_per_step = 2
+        launches_per_step = 3  # block_scores, block_topk, block_attn
 
         def step(events=None, qq=q):
             if events:
@@ -254,7 +256,13 @@ def run_ours(args, world, rank, local):
         alg = alg_bytes_token(w, k)
         dominant_bytes = k_bytes(w) + q.numel() * q.element_size()
 
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def l2_flush():
+        flush_w.zero_()  # evicts everything the step left in L2 ...
+        flush_r.amax()   # ... and leaves only clean lines behind
+
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -271,7 +279,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
         for i in range(K):
-            flush.zero_()
+            l2_flush()
             step(evs[i])
         torch.cuda.synchronize()
     if world > 1:
@@ -295,7 +303,7 @@ def run_ours(args, world, rank, local):
         d2h = sum(t.numel() * t.element_size() for t in outs)
         e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
         for i in range(K):
-            flush.zero_()
+            l2_flush()
             e2e_ev[i][0].record()
             q_step.copy_(q_host, non_blocking=True)
             lens_step.copy_(lens_host, non_blocking=True)
@@ -341,7 +349,7 @@ def run_ours(args, world, rank, local):
             "k": k, "block_size": w.block_size, "top_blocks": w.top_blocks,
             "seq_lens": "full" if int(w.seq_lens.min()) == w.L_max else [int(x) for x in w.seq_lens],
             "accumulate": "fp32", "parallelism": f"replica x{world} (independent sequences per GPU)",
-            "l2": "flushed between timed steps (256 MiB write outside the timed events)",
+            "l2": "flushed between timed steps (256 MiB write + 256 MiB read, outside the timed events)",
         },
         "us_per_step": ms * 1e3,
         "tokens_per_s": world * w.B * w.Q / (ms / 1e3),

@@ -111,18 +111,22 @@ TokenLayout token_layout(const tka_shape *s, int k) {
 }
 
 // Workspace of topk_block_attn_decode:
+//   bscore    fp32 [rows, nblk_max]  block scores
 //   block_idx int32 [rows, top+1]  (used when the caller passes none)
 //   part_ml   float4 [rows, top+1]
 //   part_acc  fp32 [rows, top+1, 128]
 //   counters  uint32 [rows]
 struct BlockLayout {
-    size_t block_idx, part_ml, part_acc, counters, total;
+    size_t bscore, block_idx, part_ml, part_acc, counters, total;
 };
 
-BlockLayout block_layout(const tka_shape *s, int top_blocks) {
+BlockLayout block_layout(const tka_shape *s, int block_size, int top_blocks) {
     BlockLayout L;
     const size_t rows = (size_t)s->B * s->Hq, slots = (size_t)top_blocks + 1;
+    const size_t nblk_max = ((size_t)s->L_max + block_size - 1) / block_size;
     size_t off = 0;
+    L.bscore = off;
+    off = align_up(off + rows * nblk_max * sizeof(float), 256);
     L.block_idx = off;
     off = align_up(off + rows * slots * sizeof(int32_t), 256);
     L.part_ml = off;
@@ -142,6 +146,8 @@ tka_status check_block_args(const tka_shape *s, int block_size, int top_blocks) 
     if (block_size != 16 && block_size != 32 && block_size != 64 && block_size != 128) return TKA_ERR_UNSUPPORTED;
     if (s->Q != 1 || top_blocks > 255) return TKA_ERR_UNSUPPORTED;
     if ((s->L_max + block_size - 1) / block_size > 8192) return TKA_ERR_UNSUPPORTED;
+    // bf16 K blocks are fetched through a tensor map whose row coordinate is a 32-bit int
+    if (s->dtype == TKA_BF16 && (long long)s->B * s->Hkv * s->L_max >= (1ll << 31)) return TKA_ERR_UNSUPPORTED;
     return TKA_OK;
 }
 
@@ -280,7 +286,7 @@ tka_status topk_block_pool_keys(const tka_shape *shape, const void *k_cache, con
 
 size_t topk_block_attn_workspace_size(const tka_shape *shape, int32_t block_size, int32_t top_blocks) {
     if (check_block_args(shape, block_size, top_blocks) != TKA_OK) return 0;
-    return block_layout(shape, top_blocks).total;
+    return block_layout(shape, block_size, top_blocks).total;
 }
 
 tka_status topk_block_attn_decode(const tka_shape *shape, const void *q, const void *k_cache, const void *v_cache,
@@ -293,7 +299,7 @@ tka_status topk_block_attn_decode(const tka_shape *shape, const void *q, const v
     if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(block_keys, 16) ||
         !aligned(out, 16) || !aligned(seq_lens, 4) || (block_idx && !aligned(block_idx, 4)))
         return TKA_ERR_INVALID_ARG;
-    const BlockLayout L = block_layout(shape, top_blocks);
+    const BlockLayout L = block_layout(shape, block_size, top_blocks);
     if (!workspace || !aligned(workspace, 256) || workspace_bytes < L.total) return TKA_ERR_WORKSPACE;
     DeviceInfo *dev = nullptr;
     if (device_info(&dev) != cudaSuccess) return TKA_ERR_CUDA;
@@ -312,6 +318,7 @@ tka_status topk_block_attn_decode(const tka_shape *shape, const void *q, const v
     sp.B = shape->B; sp.Hq = shape->Hq; sp.Hkv = shape->Hkv; sp.G = G; sp.L_max = shape->L_max;
     sp.block_size = block_size; sp.nblk_max = nblk_max; sp.top_blocks = top_blocks; sp.dtype = shape->dtype;
     sp.scale = resolve_scale(shape);
+    sp.bscore = reinterpret_cast<float *>(ws + L.bscore);
     sp.block_idx = bidx;
     sp.counters = counters;
     if (launch_block_select(sp, s) != cudaSuccess) return TKA_ERR_CUDA;
@@ -328,7 +335,7 @@ tka_status topk_block_attn_decode(const tka_shape *shape, const void *q, const v
     ap.part_acc = reinterpret_cast<float *>(ws + L.part_acc);
     ap.counters = counters;
     ap.out = out;
-    if (launch_block_attn(ap, s) != cudaSuccess) return TKA_ERR_CUDA;
+    if (launch_block_attn(ap, k_cache, dev->num_sms, s) != cudaSuccess) return TKA_ERR_CUDA;
     return TKA_OK;
 }
 

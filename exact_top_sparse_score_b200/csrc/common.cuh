@@ -72,4 +72,53 @@ __device__ __forceinline__ float block_max(float v, float *red) {
     return warp_max(t);
 }
 
+// Exclusive prefix sum of one value per thread over the block; *total gets
+// the block sum.  `tmp` holds >= 32 words of shared memory.
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *tmp, uint32_t *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    uint32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    __syncthreads();
+    if (lane == 31) tmp[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t s = lane < nw ? tmp[lane] : 0u;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, s, o);
+            if (lane >= o) s += y;
+        }
+        tmp[lane] = s;
+    }
+    __syncthreads();
+    *total = tmp[nw - 1];
+    return (warp ? tmp[warp - 1] : 0u) + x - v;
+}
+
+// Finds the bin holding the need-th largest element of a histogram whose
+// bins are ordered by key: writes the bin and the count of elements in higher
+// bins to *out_bin / *out_above.  Requires 1 <= need <= total count.
+__device__ inline void find_bin(const uint32_t *hist, int nbins, uint32_t need, uint32_t *tmp, uint32_t *out_bin,
+                         uint32_t *out_above) {
+    const int per = (nbins + blockDim.x - 1) / blockDim.x;
+    const int p0 = threadIdx.x * per;  // descending positions [p0, p0 + per)
+    uint32_t local = 0;
+    for (int p = p0; p < p0 + per && p < nbins; p++) local += hist[nbins - 1 - p];
+    uint32_t total;
+    uint32_t cum = block_excl_scan(local, tmp, &total);
+    for (int p = p0; p < p0 + per && p < nbins; p++) {
+        const uint32_t h = hist[nbins - 1 - p];
+        if (cum < need && cum + h >= need) {
+            *out_bin = (uint32_t)(nbins - 1 - p);
+            *out_above = cum;
+        }
+        cum += h;
+    }
+    __syncthreads();
+}
+
 }  // namespace tka

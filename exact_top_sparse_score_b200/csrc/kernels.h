@@ -1,6 +1,7 @@
 // Launch interfaces of the Top-k decode-attention kernels (internal).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -65,6 +66,7 @@ struct BlockSelectParams {
     const int32_t *seq_lens;
     int B, Hq, Hkv, G, L_max, block_size, nblk_max, top_blocks, dtype;
     float scale;
+    float *bscore;            // [B*Hq, nblk_max] block scores of the competing blocks
     int32_t *block_idx;       // [B*Hq, top_blocks + 1] (workspace or caller's)
     unsigned *counters;       // [B*Hq], zeroed here for the attention step
 };
@@ -76,11 +78,19 @@ struct BlockAttnParams {
     const int32_t *block_idx; // [rows, top_blocks + 1]
     int B, Hq, Hkv, G, L_max, block_size, top_blocks, dtype;
     float scale;
-    float4 *part_ml;          // [rows, top_blocks + 1] {m, l}
+    float4 *part_ml;          // [rows, top_blocks + 1] {m, l} per piece of a row
     float *part_acc;          // [rows, top_blocks + 1, 128]
     unsigned *counters;       // [rows]
     float *out;               // [rows, 128]
+    int stages;               // set by the launcher
+    uint32_t stage_bytes;
 };
+
+// cuTensorMapEncodeTiled, fetched from the driver once (null if unavailable).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn();
 
 cudaError_t launch_score(const ScoreParams &p, int num_sms, cudaStream_t stream);
 bool score_tc_supported(int dtype, int NQ);
@@ -97,6 +107,6 @@ size_t select_smem_bytes(int k);
 cudaError_t launch_gather(const GatherParams &p, cudaStream_t stream);
 cudaError_t launch_block_pool(const BlockPoolParams &p, cudaStream_t stream);
 cudaError_t launch_block_select(const BlockSelectParams &p, cudaStream_t stream);
-cudaError_t launch_block_attn(const BlockAttnParams &p, cudaStream_t stream);
+cudaError_t launch_block_attn(const BlockAttnParams &p, const void *k_cache, int num_sms, cudaStream_t stream);
 
 }  // namespace tka

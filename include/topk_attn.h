@@ -144,7 +144,7 @@ size_t topk_block_attn_workspace_size(const tka_shape *shape, int32_t block_size
  * and out is dense softmax attention over their keys below seq_lens[b].
  * block_idx (nullable) is int32 [B, 1, Hq, top_blocks + 1], ascending, -1
  * padded.  Supported: block_size in {16, 32, 64, 128}, 0 <= top_blocks <= 255,
- * ceil(L_max / block_size) <= 8192. */
+ * ceil(L_max / block_size) <= 8192, and for bf16 B * Hkv * L_max < 2^31. */
 tka_status topk_block_attn_decode(const tka_shape *shape, const void *q, const void *k_cache,
                                   const void *v_cache, const float *block_keys,
                                   const int32_t *seq_lens, int32_t block_size, int32_t top_blocks,

@@ -133,6 +133,8 @@ BLOCK_CASES = [
     ("bf16", 1, 4, 1, 640, None, 128, 2),
     ("bf16", 2, 8, 2, 700, [700, 64], 64, 30),          # top_blocks >= competing blocks: dense
     ("bf16", 1, 8, 2, 256, [1], 64, 4),                 # one-key sequence
+    ("bf16", 2, 8, 2, 3000, [3000, 2500], 32, 0),       # only the current block
+    ("bf16", 1, 8, 2, 65536, [65521], 16, 255),         # 4095 blocks, the largest top_blocks
 ]
 
 
@@ -148,3 +150,52 @@ def test_block_parity_small(case, cuda_device):
     torch.cuda.synchronize()
     assert tka.topk_attn_device_status() == 0
     check_block(w, bs, top, out, bidx, oracle.block_attn(w, bs, top))
+
+
+def test_block_parity_exact_ties(cuda_device):
+    """Blocks repeat with period 4, so every block score is shared by about a
+    quarter of the blocks and the top_blocks boundary falls inside a run of
+    exactly equal scores: the kept blocks must be the lowest-numbered ones."""
+    bs, top, L = 32, 10, 4096
+    w = workloads.make_workload(1, 1, 8, 2, L, dtype="bf16", seed=77)
+    nblk = L // bs
+    for j in range(4, nblk - 1):
+        w.k_cache[:, :, j * bs:(j + 1) * bs] = w.k_cache[:, :, (j % 4) * bs:(j % 4 + 1) * bs]
+    q, kc, vc, lens_d = to_device(w)
+    bk = tka.topk_block_pool_keys(kc, lens_d, bs)
+    out, bidx = tka.topk_block_attn_decode(q, kc, vc, bk, lens_d, bs, top)
+    torch.cuda.synchronize()
+    assert tka.topk_attn_device_status() == 0
+    ref = oracle.block_attn(w, bs, top)
+    # equal block keys give bit-equal scores on both sides, so the lists agree exactly
+    assert np.array_equal(bidx.cpu().numpy(), ref["block_idx"])
+    assert check_block(w, bs, top, out, bidx, ref) == 0
+
+
+def test_block_repeat_calls_are_bitwise_identical(cuda_device):
+    """Rows split between CTAs are merged in piece order, not arrival order."""
+    w = workloads.make_workload(4, 1, 32, 8, 8192, dtype="bf16", seed=79)
+    q, kc, vc, lens = to_device(w)
+    bk = tka.topk_block_pool_keys(kc, lens, 64)
+    a = [t.clone() for t in tka.topk_block_attn_decode(q, kc, vc, bk, lens, 64, 20)]
+    b = tka.topk_block_attn_decode(q, kc, vc, bk, lens, 64, 20)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_block_bad_seq_len_raises_status_and_skips_sequence(cuda_device):
+    w = workloads.make_workload(2, 1, 8, 2, 2048, dtype="bf16", seed=80)
+    q, kc, vc, lens = to_device(w)
+    bk = tka.topk_block_pool_keys(kc, lens, 32)
+    bad = lens.clone()
+    bad[1] = 0
+    out = torch.full((2, 1, 8, 128), 7.0, dtype=torch.float32, device="cuda")
+    tka.topk_attn_device_status()
+    tka.topk_block_attn_decode(q, kc, vc, bk, bad, 32, 6, out=out)
+    assert tka.topk_attn_device_status() & tka.DEV_BAD_SEQ_LEN
+    assert tka.topk_attn_device_status() == 0
+    assert (out[1] == 7.0).all()
+    w0 = workloads.make_workload(1, 1, 8, 2, 2048, dtype="bf16", seed=80)
+    ref = oracle.block_attn(w0, 32, 6)
+    _, bidx0 = tka.topk_block_attn_decode(q[:1], kc[:1], vc[:1], bk[:1], lens[:1], 32, 6)
+    check_block(w0, 32, 6, out[:1], bidx0, ref)
