@@ -34,6 +34,25 @@ __device__ __forceinline__ uint32_t order_key(float f) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// order_key with -0.0 mapped to +0.0, so that key order is exactly the order
+// of float comparisons (for non-NaN values): a > b iff key(a) > key(b), and
+// a == b iff key(a) == key(b).
+__device__ __forceinline__ uint32_t canon_key(float f) { return order_key(__fadd_rn(f, 0.f)); }
+
+// 2^t by the hardware approximation (PTX ex2.approx.ftz.f32).
+__device__ __forceinline__ float exp2_approx(float t) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(t));
+    return r;
+}
+
+constexpr float kLog2e = 1.4426950408889634f;  // log2(e): e^x = 2^(x log2 e)
+
+// Inverse of order_key.
+__device__ __forceinline__ float key_float(uint32_t key) {
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
+
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 

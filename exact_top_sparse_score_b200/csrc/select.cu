@@ -7,22 +7,23 @@
 // the discarded mass is the Top-k tail mass of "A Mathematical Theory of
 // Top-k Sparse Attention via Total Variation Distance" (abstract).
 //
-// One CTA (32 warps) per row; every warp owns a contiguous
-// segment of the row, lane l holding positions l, l + 32, ... of it, so a warp
-// compacts 32 consecutive positions at a time with one ballot.  A segment is
-// streamed in batches of 32 x 32 positions with all loads of a batch in
-// flight together (a segment that fits one batch is read once and kept in
-// registers for all passes); the rows come from L2.  Scores are compared as
-// order-preserving uint32 keys:
+// One CTA (32 warps) per row; every warp owns a contiguous segment of the
+// row, lane l holding positions l, l + 32, ... of it, so a warp compacts 32
+// consecutive positions at a time with one ballot.  A segment is streamed in
+// batches of 32 x 32 positions with all loads of a batch in flight together
+// (a segment that fits one batch is read once and kept in registers for all
+// passes); the rows come from L2.  Ranks are taken on order-preserving uint32
+// keys with -0 folded into +0 (canon_key), so key order is float order and
+// the per-position tests below are plain float comparisons:
 //   pass 1  the row maximum and the histogram of the top 11 key bits of a
-//           position-uniform 1/8 sample give a bin range that holds the k-th
-//           key with high probability;
-//   pass 2  keys above the range are counted, keys inside it are collected
-//           (in position order) into per-warp candidate lists;
+//           sample (every eighth group of 32 positions) give a bin range that
+//           holds the k-th key with high probability;
+//   pass 2  scores above the range are counted, keys inside it are collected
+//           (unordered) into per-warp candidate lists;
 //   exact radix selection over the candidates' full keys (11 + 11 + 10 bits)
 //           yields the k-th key T and how many of the keys equal to T are
 //           kept (the lowest positions);
-//   pass 3  every key is tested against that exact rule and the kept
+//   pass 3  every score is tested against that exact rule and the kept
 //           positions are written straight to their ascending slots (warp
 //           prefix sums plus per-warp offsets), while Z_k = sum_kept e^{s-m}
 //           and Z_tail = sum_dropped e^{s-m} are accumulated; the tail mass
@@ -137,7 +138,7 @@ __device__ void select_multipass(const SelectParams &p, int row, int vis, const 
     float m = -INFINITY;
     visit_row(s, vis, [&](int, float x) {
         m = fmaxf(m, x);
-        atomicAdd(&hist[order_key(x) >> 21], 1u);
+        atomicAdd(&hist[canon_key(x) >> 21], 1u);
     });
     m = block_max(m, sm.red);
     __syncthreads();
@@ -147,7 +148,7 @@ __device__ void select_multipass(const SelectParams &p, int row, int vis, const 
     for (int i = threadIdx.x; i < 2048; i += blockDim.x) hist[i] = 0u;
     __syncthreads();
     visit_row(s, vis, [&](int, float x) {
-        const uint32_t key = order_key(x);
+        const uint32_t key = canon_key(x);
         if ((key >> 21) == b1) atomicAdd(&hist[(key >> 10) & 0x7ffu], 1u);
     });
     __syncthreads();
@@ -158,7 +159,7 @@ __device__ void select_multipass(const SelectParams &p, int row, int vis, const 
     for (int i = threadIdx.x; i < 2048; i += blockDim.x) hist[i] = 0u;
     __syncthreads();
     visit_row(s, vis, [&](int, float x) {
-        const uint32_t key = order_key(x);
+        const uint32_t key = canon_key(x);
         if ((key >> 10) == pre) atomicAdd(&hist[key & 0x3ffu], 1u);
     });
     __syncthreads();
@@ -179,7 +180,7 @@ __device__ void select_multipass(const SelectParams &p, int row, int vis, const 
         uint32_t key[4], n_eq_t = 0u;
 #pragma unroll
         for (int j = 0; j < 4; j++) {
-            key[j] = order_key(x[j]);
+            key[j] = canon_key(x[j]);
             if (i0 + j < vis && key[j] == T) n_eq_t++;
         }
         uint32_t eq_total = 0u, eq_rank = base_eq;
@@ -231,7 +232,6 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_topk(SelectParams p)
     sm.scal = dyn + 2048 + 64;                                       // [8]
     uint32_t *wstat = dyn + 2048 + 72;                               // [kWarps][8]
     uint32_t *wc_key = wstat + kWarps * 8;                           // [kWarps][kWarpCand]
-    int32_t *wc_pos = reinterpret_cast<int32_t *>(wc_key + kWarps * kWarpCand);  // [kWarps][kWarpCand]
 
     const int row = blockIdx.x;
     const int b = row / (p.Q * p.Hq), qpos = (row / p.Hq) % p.Q;
@@ -253,7 +253,8 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_topk(SelectParams p)
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint32_t lt = lanemask_lt();
     // this warp's contiguous segment; lane l holds positions lo + 32 r + l of
-    // each batch of 32 * kHeld positions
+    // each batch of 32 * kHeld positions, -inf past the segment's end (so the
+    // passes below need no bounds tests: -inf is never kept and weighs 0)
     const int seg = (((vis + kWarps - 1) / kWarps) + 31) & ~31;
     const int lo = min(vis, warp * seg), hi = min(vis, lo + seg);
     const int nbatch = (hi - lo + 32 * kHeld - 1) / (32 * kHeld);
@@ -262,78 +263,74 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_topk(SelectParams p)
     auto load_batch = [&](int bi) {
         const int p0 = lo + bi * 32 * kHeld + lane;
 #pragma unroll
-        for (int r = 0; r < kHeld; r++) x[r] = p0 + 32 * r < hi ? __ldcg(s + p0 + 32 * r) : 0.f;
+        for (int r = 0; r < kHeld; r++) x[r] = p0 + 32 * r < hi ? __ldcg(s + p0 + 32 * r) : -INFINITY;
     };
     if (resident) load_batch(0);
 
     // pass 1: the row maximum, and the histogram of the top 11 key bits of a
-    // position-uniform sample (positions that are multiples of 8; every
-    // position on short rows) -- the threshold is looked for there
+    // sample: every eighth group of 32 consecutive positions (every position
+    // on short rows) -- the threshold is looked for there
     for (int i = threadIdx.x; i < 2048; i += kSelectThreads) sm.hist[i] = 0u;
     __syncthreads();
     const bool sampled = vis >= kSampleMinLen;
-    const bool sampler = !sampled || (lane & 7) == 0;  // lo is a multiple of 32
     float m = -INFINITY;
+    uint32_t nsample = 0u;
     for (int bi = 0; bi < nbatch; bi++) {
         if (!resident) load_batch(bi);
         const int p0 = lo + bi * 32 * kHeld + lane;
 #pragma unroll
         for (int r = 0; r < kHeld; r++) {
-            if (p0 + 32 * r < hi) {
-                m = fmaxf(m, x[r]);
-                if (sampler) atomicAdd(&sm.hist[order_key(x[r]) >> 21], 1u);
+            m = fmaxf(m, x[r]);
+            if ((!sampled || (r & 7) == 0) && p0 + 32 * r < hi) {
+                atomicAdd(&sm.hist[canon_key(x[r]) >> 21], 1u);
+                nsample++;
             }
         }
     }
-    m = block_max(m, sm.red);
-    __syncthreads();
+    if (lane == 0) wstat[warp * 8 + 1] = 0u;  // this warp's candidate count, for pass 2
+    nsample = warp_sum(nsample);
+    if (lane == 0) wstat[warp * 8 + 6] = nsample;
+    m = block_max(m, sm.red);  // contains __syncthreads
+    uint32_t total_sample = 0u;
+    for (int w = 0; w < kWarps; w++) total_sample += wstat[w * 8 + 6];
     // bins above b_hi are kept; bins [b_lo, b_hi] hold the candidates.  On the
-    // sample the k-th key has rank about k/8; the range is widened by 4
-    // binomial standard deviations each way and checked exactly below.
-    uint32_t b_hi, b_lo;
+    // sample the k-th key has rank about k * nsample / vis; the range is
+    // widened by 4 binomial standard deviations each way and checked exactly
+    // below.  As floats: x >= hi_t is above, lo_t <= x < hi_t a candidate.
+    float hi_t, lo_t;
     {
-        const int slog = sampled ? 3 : 0;
-        const uint32_t nsample = (uint32_t)((vis + (1 << slog) - 1) >> slog);
-        const float ks = (float)k / (float)(1 << slog);
+        const float ks = (float)k * (float)total_sample / (float)vis;
         const float margin = sampled ? 4.f * sqrtf(ks) + 4.f : 0.f;
         const uint32_t need_hi = (uint32_t)fmaxf(1.f, floorf(ks - margin));
-        const uint32_t need_lo = (uint32_t)fminf((float)nsample, ceilf(ks + margin));
+        const uint32_t need_lo = (uint32_t)fminf((float)total_sample, ceilf(ks + margin));
         find_bin(sm.hist, 2048, need_hi, sm.tmp, &sm.scal[0], &sm.scal[1]);
-        b_hi = sm.scal[0];
+        const uint32_t b_hi = sm.scal[0];
         find_bin(sm.hist, 2048, max(need_lo, need_hi), sm.tmp, &sm.scal[0], &sm.scal[1]);
-        b_lo = sm.scal[0];
+        const uint32_t b_lo = sm.scal[0];
+        // a NaN threshold compares false: nothing above bin 2044 (+inf) or below bin 4 (-FLT_MAX)
+        hi_t = b_hi >= 2044u ? __uint_as_float(0x7fc00000u) : key_float((b_hi + 1u) << 21);
+        lo_t = key_float(b_lo << 21);
     }
 
-    // pass 2: count the keys of bins above b_hi; collect the keys of bins
-    // [b_lo, b_hi], in position order, into this warp's candidate list
-    uint32_t nwin = 0u, ncw = 0u;
+    // pass 2: count the positions above the range; collect the keys inside it
+    // (in any order: only their values matter) into this warp's candidate list
+    uint32_t nwin = 0u;
     uint32_t *my_key = wc_key + warp * kWarpCand;
-    int32_t *my_pos = wc_pos + warp * kWarpCand;
     for (int bi = 0; bi < nbatch; bi++) {
         if (!resident) load_batch(bi);
-        const int p0 = lo + bi * 32 * kHeld + lane;
 #pragma unroll
         for (int r = 0; r < kHeld; r++) {
-            const bool valid = p0 + 32 * r < hi;
-            const uint32_t key = order_key(x[r]);
-            const uint32_t bin = key >> 21;
-            nwin += __popc(__ballot_sync(0xffffffffu, valid && bin > b_hi));
-            const bool cand = valid && bin >= b_lo && bin <= b_hi;
-            const uint32_t cb = __ballot_sync(0xffffffffu, cand);
-            if (cand) {
-                const uint32_t slot = ncw + __popc(cb & lt);
-                if (slot < (uint32_t)kWarpCand) {
-                    my_key[slot] = key;
-                    my_pos[slot] = p0 + 32 * r;
-                }
+            const float xv = x[r];
+            const bool above = xv >= hi_t;
+            nwin += above;
+            if (xv >= lo_t && !above) {
+                const uint32_t slot = atomicAdd(&wstat[warp * 8 + 1], 1u);
+                if (slot < (uint32_t)kWarpCand) my_key[slot] = canon_key(xv);
             }
-            ncw += __popc(cb);
         }
     }
-    if (lane == 0) {
-        wstat[warp * 8 + 0] = nwin;
-        wstat[warp * 8 + 1] = ncw;
-    }
+    nwin = warp_sum(nwin);
+    if (lane == 0) wstat[warp * 8 + 0] = nwin;
     __syncthreads();
     uint32_t above = 0u, ncand = 0u;
     bool overflow = false;
@@ -381,6 +378,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_topk(SelectParams p)
     // per warp: candidates above T and ties at T, then output offsets
     {
         uint32_t g = 0u, t = 0u;
+        const uint32_t ncw = wstat[warp * 8 + 1];
         for (uint32_t i = lane; i < ncw; i += 32) {
             g += my_key[i] > T;
             t += my_key[i] == T;
@@ -406,43 +404,48 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_topk(SelectParams p)
     const bool rank_ties = n_eq != r_eq;
     const uint32_t out_begin = out_run;
 
-    // pass 3: the exact rule -- key > T, or key == T among the first r_eq
-    // ties -- written straight to the final ascending positions, with the
-    // softmax sums of kept and dropped keys
+    // pass 3: the exact rule -- s > T, or s == T among the first r_eq ties
+    // (s >= T when every tie is kept) -- written straight to the final
+    // ascending positions, with the softmax sums of kept and dropped scores.
+    // As float comparisons: canon_key order is float order.
+    const float T_f = key_float(T);
+    const float m_l2e = m * kLog2e;
     int32_t *idx = p.idx + (size_t)row * k;
     float *wv = p.w + (size_t)row * k;
     float zk = 0.f, zt = 0.f;
+    auto emit = [&](bool sel, float e, int pos) {
+        const uint32_t sb = __ballot_sync(0xffffffffu, sel);
+        if (sel) {
+            const uint32_t o = out_run + __popc(sb & lt);
+            if (o < (uint32_t)k) {  // always true unless the counts above are wrong
+                idx[o] = pos;
+                wv[o] = e;
+            }
+            zk += e;
+        } else {
+            zt += e;
+        }
+        out_run += __popc(sb);
+    };
     for (int bi = 0; bi < nbatch; bi++) {
         if (!resident) load_batch(bi);
         const int p0 = lo + bi * 32 * kHeld + lane;
+        if (rank_ties) {
 #pragma unroll
-        for (int r = 0; r < kHeld; r++) {
-            const bool valid = p0 + 32 * r < hi;
-            const uint32_t key = order_key(x[r]);
-            bool sel = valid && key > T;
-            if (rank_ties) {
-                const bool tie = valid && key == T;
+            for (int r = 0; r < kHeld; r++) {
+                const float xv = x[r];
+                const bool tie = xv == T_f;
                 const uint32_t tb = __ballot_sync(0xffffffffu, tie);
-                if (tie) sel = tie_run + __popc(tb & lt) < r_eq;
+                const bool sel = xv > T_f || (tie && tie_run + __popc(tb & lt) < r_eq);
                 tie_run += __popc(tb);
-            } else {
-                sel = sel || (valid && key == T);
+                emit(sel, exp2_approx(fmaf(xv, kLog2e, -m_l2e)), p0 + 32 * r);
             }
-            const uint32_t sb = __ballot_sync(0xffffffffu, sel);
-            if (valid) {
-                const float e = __expf(x[r] - m);
-                if (sel) {
-                    const uint32_t o = out_run + __popc(sb & lt);
-                    if (o < (uint32_t)k) {  // always true unless the counts above are wrong
-                        idx[o] = p0 + 32 * r;
-                        wv[o] = e;
-                    }
-                    zk += e;
-                } else {
-                    zt += e;
-                }
+        } else {
+#pragma unroll
+            for (int r = 0; r < kHeld; r++) {
+                const float xv = x[r];
+                emit(xv >= T_f, exp2_approx(fmaf(xv, kLog2e, -m_l2e)), p0 + 32 * r);
             }
-            out_run += __popc(sb);
         }
     }
     if (lane == 0) wstat[warp * 8 + 4] = out_run - out_begin;
@@ -455,7 +458,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_topk(SelectParams p)
 }  // namespace
 
 size_t select_smem_bytes(int) {
-    return (size_t)(2048 + 72 + kWarps * 8) * 4 + (size_t)kWarps * kWarpCand * 8;
+    return (size_t)(2048 + 72 + kWarps * 8) * 4 + (size_t)kWarps * kWarpCand * 4;
 }
 
 cudaError_t launch_select(const SelectParams &p, cudaStream_t stream) {
