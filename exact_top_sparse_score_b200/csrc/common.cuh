@@ -118,24 +118,62 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *tmp, u
     return (warp ? tmp[warp - 1] : 0u) + x - v;
 }
 
+// Inclusive prefix sum of v over the warp.
+__device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += y;
+    }
+    return v;
+}
+
 // Finds the bin holding the need-th largest element of a histogram whose
 // bins are ordered by key: writes the bin and the count of elements in higher
-// bins to *out_bin / *out_above.  Requires 1 <= need <= total count.
-__device__ inline void find_bin(const uint32_t *hist, int nbins, uint32_t need, uint32_t *tmp, uint32_t *out_bin,
-                         uint32_t *out_above) {
-    const int per = (nbins + blockDim.x - 1) / blockDim.x;
-    const int p0 = threadIdx.x * per;  // descending positions [p0, p0 + per)
-    uint32_t local = 0;
-    for (int p = p0; p < p0 + per && p < nbins; p++) local += hist[nbins - 1 - p];
-    uint32_t total;
-    uint32_t cum = block_excl_scan(local, tmp, &total);
-    for (int p = p0; p < p0 + per && p < nbins; p++) {
-        const uint32_t h = hist[nbins - 1 - p];
-        if (cum < need && cum + h >= need) {
-            *out_bin = (uint32_t)(nbins - 1 - p);
-            *out_above = cum;
+// bins to *out_bin / *out_above.  Requires 1 <= need <= total count, nbins a
+// multiple of 32 (at most 2048).  Called by the whole block, which first
+// meets at a barrier (so the histogram is complete and the results of a
+// previous call have been read); warp 0 does the search (lane l sums the nbins/32 bins below the top l nbins/32,
+// starting at a lane-dependent bin so that the loads spread over the banks;
+// a prefix sum over the lanes finds the lane holding the bin, and the warp
+// then scans that lane's bins 32 at a time); the block waits at a barrier.
+__device__ inline void find_bin(const uint32_t *hist, int nbins, uint32_t need, uint32_t *, uint32_t *out_bin,
+                                uint32_t *out_above) {
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        const int per = nbins >> 5;
+        const int top = nbins - 1 - lane * per;
+        uint32_t local = 0u;
+        for (int i = 0; i < per; i++) local += hist[top - (i + lane) % per];
+        const uint32_t cum = warp_incl_scan(local);
+        const uint32_t before = cum - local;
+        const uint32_t hit = __ballot_sync(0xffffffffu, before < need && cum >= need);
+        if (hit == 0u) {
+            if (lane == 0) {  // need outside [1, total]: never true for a valid call
+                *out_bin = 0u;
+                *out_above = 0u;
+            }
+        } else {
+            const int L = __ffs(hit) - 1;
+            const int topL = nbins - 1 - L * per;
+            uint32_t c = __shfl_sync(0xffffffffu, before, L);
+            for (int i0 = 0; i0 < per; i0 += 32) {
+                const uint32_t h = i0 + lane < per ? hist[topL - i0 - lane] : 0u;
+                const uint32_t inc = warp_incl_scan(h);
+                const uint32_t excl = c + inc - h;
+                const uint32_t fb = __ballot_sync(0xffffffffu, excl < need && excl + h >= need);
+                if (fb != 0u) {
+                    if (lane == __ffs(fb) - 1) {
+                        *out_bin = (uint32_t)(topL - i0 - lane);
+                        *out_above = excl;
+                    }
+                    break;
+                }
+                c += __shfl_sync(0xffffffffu, inc, 31);
+            }
         }
-        cum += h;
     }
     __syncthreads();
 }

@@ -39,7 +39,7 @@ namespace tka {
 namespace {
 
 constexpr int kSelectThreads = 1024;
-constexpr int kWarps = kSelectThreads / 32;
+constexpr int kWarps = kSelectThreads / 32;  // 32: per-warp words are reduced by one warp, lane w reading warp w's
 constexpr int kWarpCand = 256;                  // candidates per warp held in shared memory
 constexpr int kHeld = 32;                       // scores per lane held in registers per batch
 constexpr int kSampleMinLen = 16384;            // rows this long histogram a 1/8 sample in pass 1
@@ -291,8 +291,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_topk(SelectParams p)
     nsample = warp_sum(nsample);
     if (lane == 0) wstat[warp * 8 + 6] = nsample;
     m = block_max(m, sm.red);  // contains __syncthreads
-    uint32_t total_sample = 0u;
-    for (int w = 0; w < kWarps; w++) total_sample += wstat[w * 8 + 6];
+    const uint32_t total_sample = warp_sum(wstat[lane * 8 + 6]);  // kWarps == 32
     // bins above b_hi are kept; bins [b_lo, b_hi] hold the candidates.  On the
     // sample the k-th key has rank about k * nsample / vis; the range is
     // widened by 4 binomial standard deviations each way and checked exactly
@@ -332,13 +331,10 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_topk(SelectParams p)
     nwin = warp_sum(nwin);
     if (lane == 0) wstat[warp * 8 + 0] = nwin;
     __syncthreads();
-    uint32_t above = 0u, ncand = 0u;
-    bool overflow = false;
-    for (int w = 0; w < kWarps; w++) {
-        above += wstat[w * 8 + 0];
-        ncand += wstat[w * 8 + 1];
-        overflow |= wstat[w * 8 + 1] > (uint32_t)kWarpCand;
-    }
+    // block totals, every warp reducing the per-warp words (lane w reads warp w's)
+    const uint32_t above = warp_sum(wstat[lane * 8 + 0]);
+    const uint32_t ncand = warp_sum(wstat[lane * 8 + 1]);
+    const bool overflow = __any_sync(0xffffffffu, wstat[lane * 8 + 1] > (uint32_t)kWarpCand);
     if (overflow || above >= (uint32_t)k || above + ncand < (uint32_t)k) {
         // the sampled range missed the k-th key or a warp's list overflowed:
         // take the exact multi-pass route
@@ -356,10 +352,8 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_topk(SelectParams p)
         const int nb = level == 2 ? 1024 : 2048;
         for (int i = threadIdx.x; i < 2048; i += kSelectThreads) sm.hist[i] = 0u;
         __syncthreads();
-        for (int e = threadIdx.x; e < kWarps * kWarpCand; e += kSelectThreads) {
-            const int w = e / kWarpCand, i = e - w * kWarpCand;
-            if ((uint32_t)i >= wstat[w * 8 + 1]) continue;
-            const uint32_t key = wc_key[e];
+        for (uint32_t i = lane; i < wstat[warp * 8 + 1]; i += 32) {  // this warp's own list
+            const uint32_t key = my_key[i];
             if (level == 0 || (key >> (shift + (level == 1 ? 11 : 10))) == pre)
                 atomicAdd(&sm.hist[(key >> shift) & (uint32_t)(nb - 1)], 1u);
         }
@@ -378,8 +372,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_topk(SelectParams p)
     // per warp: candidates above T and ties at T, then output offsets
     {
         uint32_t g = 0u, t = 0u;
-        const uint32_t ncw = wstat[warp * 8 + 1];
-        for (uint32_t i = lane; i < ncw; i += 32) {
+        for (uint32_t i = lane; i < wstat[warp * 8 + 1]; i += 32) {
             g += my_key[i] > T;
             t += my_key[i] == T;
         }
@@ -391,15 +384,18 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_topk(SelectParams p)
         }
     }
     __syncthreads();
-    uint32_t out_run = 0u, tie_run = 0u, n_eq = 0u;
-    for (int w = 0; w < kWarps; w++) {
-        const uint32_t tie_w = wstat[w * 8 + 3];
-        if (w < warp) {
-            const uint32_t kept_ties = r_eq > tie_run ? min(tie_w, r_eq - tie_run) : 0u;
-            out_run += wstat[w * 8 + 0] + wstat[w * 8 + 2] + kept_ties;
-            tie_run += tie_w;
-        }
-        n_eq += tie_w;
+    // output offsets: warp w keeps its scores above the range, its candidates
+    // above T and the ties at T that fall among the first r_eq of the row
+    uint32_t out_run, tie_run, n_eq;
+    {
+        const uint32_t tie_l = wstat[lane * 8 + 3];
+        const uint32_t tie_incl = warp_incl_scan(tie_l), tie_excl = tie_incl - tie_l;
+        const uint32_t kept_l = wstat[lane * 8 + 0] + wstat[lane * 8 + 2] +
+                                (r_eq > tie_excl ? min(tie_l, r_eq - tie_excl) : 0u);
+        const uint32_t out_incl = warp_incl_scan(kept_l);
+        out_run = __shfl_sync(0xffffffffu, out_incl - kept_l, warp);
+        tie_run = __shfl_sync(0xffffffffu, tie_excl, warp);
+        n_eq = __shfl_sync(0xffffffffu, tie_incl, 31);
     }
     const bool rank_ties = n_eq != r_eq;
     const uint32_t out_begin = out_run;
@@ -450,8 +446,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_topk(SelectParams p)
     }
     if (lane == 0) wstat[warp * 8 + 4] = out_run - out_begin;
     __syncthreads();
-    uint32_t written = 0u;
-    for (int w = 0; w < kWarps; w++) written += wstat[w * 8 + 4];
+    const uint32_t written = warp_sum(wstat[lane * 8 + 4]);
     finish_row(p, row, m, zk, zt, written, (uint32_t)k, sm);
 }
 
