@@ -242,8 +242,9 @@ tka_status topk_attn_decode_staged(const tka_shape *shape, const void *q, const 
     gp.partial = reinterpret_cast<float *>(ws + L.partial);
     gp.counters = se.counters;
     gp.out = out;
-    // about 8 CTAs per SM in total, never fewer than kMinKeysPerSplit keys per CTA
-    int splits = (dev->num_sms * 8 + rows - 1) / rows;
+    // one wave of eight CTAs per SM (splits = floor(8 x SMs / rows), at least 1),
+    // never fewer than kMinKeysPerSplit keys per CTA
+    int splits = (dev->num_sms * 8) / rows;
     if (splits > L.max_splits) splits = L.max_splits;
     if (splits < 1) splits = 1;
     gp.per_split = (k + splits - 1) / splits;

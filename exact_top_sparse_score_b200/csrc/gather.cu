@@ -10,9 +10,10 @@
 // positions.  The slice's positions and weights are first staged in shared
 // memory (coalesced), so the V loads that follow depend on nothing in
 // flight: a V row is 256 bytes in bf16, read by 16 lanes with one 16-byte
-// load each, and every lane keeps 8 rows in flight.  The slices of a row are
-// summed by whichever CTA of the row finishes last (an atomic ticket, no
-// waiting), in slice order, so the result does not depend on scheduling.
+// load each, and every lane keeps 4 rows in flight (eight CTAs per SM).
+// The slices of a row are summed by whichever CTA of the row finishes last
+// (an atomic ticket, no waiting), in slice order, so the result does not
+// depend on scheduling.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -22,7 +23,7 @@ namespace {
 
 constexpr int kGatherThreads = 256;
 constexpr int kChunk = 512;  // positions staged in shared memory at a time
-constexpr int kUnroll = 8;
+constexpr int kUnroll = 4;
 
 __device__ __forceinline__ uint4 ldg_stream(const void *p) {
     uint4 r;
@@ -48,7 +49,7 @@ __device__ __forceinline__ void fma_row(float (&acc)[16 / sizeof(T)], float wt, 
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kGatherThreads) gather_pv(GatherParams p) {
+__global__ void __launch_bounds__(kGatherThreads, 8) gather_pv(GatherParams p) {
     constexpr int kPer = 16 / sizeof(T);              // elements per lane
     constexpr int kLanesPerRow = kHeadDim / kPer;     // 16 (bf16) or 32 (fp32)
     constexpr int kRowsPerWarp = 32 / kLanesPerRow;   // 2 or 1

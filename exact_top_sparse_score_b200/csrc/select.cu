@@ -279,11 +279,21 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_topk(SelectParams p)
         if (!resident) load_batch(bi);
         const int p0 = lo + bi * 32 * kHeld + lane;
 #pragma unroll
-        for (int r = 0; r < kHeld; r++) {
-            m = fmaxf(m, x[r]);
-            if ((!sampled || (r & 7) == 0) && p0 + 32 * r < hi) {
-                atomicAdd(&sm.hist[canon_key(x[r]) >> 21], 1u);
-                nsample++;
+        for (int r = 0; r < kHeld; r++) m = fmaxf(m, x[r]);
+        if (sampled) {
+#pragma unroll
+            for (int r = 0; r < kHeld; r += 8) {
+                if (p0 + 32 * r < hi) {
+                    atomicAdd(&sm.hist[canon_key(x[r]) >> 21], 1u);
+                    nsample++;
+                }
+            }
+        } else {
+            for (int r = 0; r < kHeld; r++) {  // short rows: every position (not unrolled: rare)
+                if (p0 + 32 * r < hi) {
+                    atomicAdd(&sm.hist[canon_key(x[r]) >> 21], 1u);
+                    nsample++;
+                }
             }
         }
     }
@@ -324,7 +334,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_topk(SelectParams p)
             nwin += above;
             if (xv >= lo_t && !above) {
                 const uint32_t slot = atomicAdd(&wstat[warp * 8 + 1], 1u);
-                if (slot < (uint32_t)kWarpCand) my_key[slot] = canon_key(xv);
+                if (slot < (uint32_t)kWarpCand) my_key[slot] = __float_as_uint(xv);  // converted when ranked
             }
         }
     }
@@ -353,7 +363,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_topk(SelectParams p)
         for (int i = threadIdx.x; i < 2048; i += kSelectThreads) sm.hist[i] = 0u;
         __syncthreads();
         for (uint32_t i = lane; i < wstat[warp * 8 + 1]; i += 32) {  // this warp's own list
-            const uint32_t key = my_key[i];
+            const uint32_t key = canon_key(__uint_as_float(my_key[i]));
             if (level == 0 || (key >> (shift + (level == 1 ? 11 : 10))) == pre)
                 atomicAdd(&sm.hist[(key >> shift) & (uint32_t)(nb - 1)], 1u);
         }
@@ -373,8 +383,9 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_topk(SelectParams p)
     {
         uint32_t g = 0u, t = 0u;
         for (uint32_t i = lane; i < wstat[warp * 8 + 1]; i += 32) {
-            g += my_key[i] > T;
-            t += my_key[i] == T;
+            const uint32_t key = canon_key(__uint_as_float(my_key[i]));
+            g += key > T;
+            t += key == T;
         }
         g = warp_sum(g);
         t = warp_sum(t);
