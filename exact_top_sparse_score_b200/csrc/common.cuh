@@ -129,53 +129,74 @@ __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v) {
     return v;
 }
 
-// Finds the bin holding the need-th largest element of a histogram whose
-// bins are ordered by key: writes the bin and the count of elements in higher
-// bins to *out_bin / *out_above.  Requires 1 <= need <= total count, nbins a
-// multiple of 32 (at most 2048).  Called by the whole block, which first
-// meets at a barrier (so the histogram is complete and the results of a
-// previous call have been read); warp 0 does the search (lane l sums the nbins/32 bins below the top l nbins/32,
-// starting at a lane-dependent bin so that the loads spread over the banks;
-// a prefix sum over the lanes finds the lane holding the bin, and the warp
-// then scans that lane's bins 32 at a time); the block waits at a barrier.
-__device__ inline void find_bin(const uint32_t *hist, int nbins, uint32_t need, uint32_t *, uint32_t *out_bin,
-                                uint32_t *out_above) {
+// Finds, on one warp, the bin holding the need-th largest element of a
+// histogram of NB bins ordered by key: the bin and the count of elements in
+// higher bins, in every lane.  Requires 1 <= need <= total count and NB a
+// power of two in [32, 2048].  Lane l sums the NB/32 bins below the top
+// l NB/32 (all loads in flight together, starting at a lane-dependent bin so
+// that they spread over the banks), a prefix sum over the lanes finds the
+// lane holding the bin, and the warp then scans that lane's bins 32 at a time.
+template <int NB>
+__device__ inline void warp_find_bin(const uint32_t *hist, uint32_t need, uint32_t &bin, uint32_t &above) {
+    static_assert(NB >= 32 && NB <= 2048 && (NB & (NB - 1)) == 0, "bins: a power of two in [32, 2048]");
+    constexpr int kPer = NB / 32;
+    const int lane = threadIdx.x & 31;
+    const int top = NB - 1 - lane * kPer;
+    uint32_t local = 0u;
+#pragma unroll
+    for (int i = 0; i < kPer; i++) local += hist[top - ((i + lane) & (kPer - 1))];
+    const uint32_t cum = warp_incl_scan(local);
+    const uint32_t before = cum - local;
+    const uint32_t hit = __ballot_sync(0xffffffffu, before < need && cum >= need);
+    bin = 0u;  // need outside [1, total]: never the case for a valid call
+    above = 0u;
+    if (hit != 0u) {
+        const int L = __ffs(hit) - 1;
+        const int topL = NB - 1 - L * kPer;
+        uint32_t c = __shfl_sync(0xffffffffu, before, L);
+#pragma unroll
+        for (int i0 = 0; i0 < kPer; i0 += 32) {
+            const uint32_t h = i0 + lane < kPer ? hist[topL - i0 - lane] : 0u;
+            const uint32_t inc = warp_incl_scan(h);
+            const uint32_t excl = c + inc - h;
+            const uint32_t fb = __ballot_sync(0xffffffffu, excl < need && excl + h >= need);
+            if (fb != 0u) {
+                const int f = __ffs(fb) - 1;
+                bin = (uint32_t)(topL - i0 - f);
+                above = __shfl_sync(0xffffffffu, excl, f);
+                break;
+            }
+            c += __shfl_sync(0xffffffffu, inc, 31);
+        }
+    }
+}
+
+// The same search for the whole block: the block first meets at a barrier
+// (so the histogram is complete and the results of a previous call have been
+// read), warp 0 searches and writes the results, and the block meets again.
+template <int NB>
+__device__ inline void find_bin_n(const uint32_t *hist, uint32_t need, uint32_t *out_bin, uint32_t *out_above) {
     __syncthreads();
     if (threadIdx.x < 32) {
-        const int lane = threadIdx.x;
-        const int per = nbins >> 5;
-        const int top = nbins - 1 - lane * per;
-        uint32_t local = 0u;
-        for (int i = 0; i < per; i++) local += hist[top - (i + lane) % per];
-        const uint32_t cum = warp_incl_scan(local);
-        const uint32_t before = cum - local;
-        const uint32_t hit = __ballot_sync(0xffffffffu, before < need && cum >= need);
-        if (hit == 0u) {
-            if (lane == 0) {  // need outside [1, total]: never true for a valid call
-                *out_bin = 0u;
-                *out_above = 0u;
-            }
-        } else {
-            const int L = __ffs(hit) - 1;
-            const int topL = nbins - 1 - L * per;
-            uint32_t c = __shfl_sync(0xffffffffu, before, L);
-            for (int i0 = 0; i0 < per; i0 += 32) {
-                const uint32_t h = i0 + lane < per ? hist[topL - i0 - lane] : 0u;
-                const uint32_t inc = warp_incl_scan(h);
-                const uint32_t excl = c + inc - h;
-                const uint32_t fb = __ballot_sync(0xffffffffu, excl < need && excl + h >= need);
-                if (fb != 0u) {
-                    if (lane == __ffs(fb) - 1) {
-                        *out_bin = (uint32_t)(topL - i0 - lane);
-                        *out_above = excl;
-                    }
-                    break;
-                }
-                c += __shfl_sync(0xffffffffu, inc, 31);
-            }
+        uint32_t bin, above;
+        warp_find_bin<NB>(hist, need, bin, above);
+        if (threadIdx.x == 0) {
+            *out_bin = bin;
+            *out_above = above;
         }
     }
     __syncthreads();
+}
+
+// find_bin_n for nbins = 256, 1024 or 2048 (the sizes the kernels use).
+__device__ inline void find_bin(const uint32_t *hist, int nbins, uint32_t need, uint32_t *, uint32_t *out_bin,
+                                uint32_t *out_above) {
+    if (nbins == 2048)
+        find_bin_n<2048>(hist, need, out_bin, out_above);
+    else if (nbins == 1024)
+        find_bin_n<1024>(hist, need, out_bin, out_above);
+    else
+        find_bin_n<256>(hist, need, out_bin, out_above);
 }
 
 }  // namespace tka

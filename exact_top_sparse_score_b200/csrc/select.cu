@@ -39,7 +39,8 @@ namespace tka {
 namespace {
 
 constexpr int kSelectThreads = 1024;
-constexpr int kWarps = kSelectThreads / 32;  // 32: per-warp words are reduced by one warp, lane w reading warp w's
+constexpr int kWarps = kSelectThreads / 32;  // <= 32: per-warp words are reduced by one warp, lane w reading warp w's
+constexpr int kSelectCtasPerSm = 1024 / kSelectThreads;
 constexpr int kWarpCand = 256;                  // candidates per warp held in shared memory
 constexpr int kHeld = 32;                       // scores per lane held in registers per batch
 constexpr int kSampleMinLen = 16384;            // rows this long histogram a 1/8 sample in pass 1
@@ -93,16 +94,27 @@ __device__ __forceinline__ void load4(const float *s, int i0, int n, float (&x)[
 struct SelectSmem {
     uint32_t *hist;  // [2048]
     uint32_t *tmp;   // [32]
-    float *red;      // [32]
+    float *red;      // [64]
     uint32_t *scal;  // [2]: bin, above
 };
 
 // Writes stats, tail and counter of a finished row.
 __device__ __forceinline__ void finish_row(const SelectParams &p, int row, float m, float zk, float zt,
                                            uint32_t written, uint32_t kept, const SelectSmem &sm) {
-    zk = block_sum(zk, sm.red);
-    __syncthreads();
-    zt = block_sum(zt, sm.red);
+    {
+        // both block sums with one pair of barriers
+        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+        zk = warp_sum(zk);
+        zt = warp_sum(zt);
+        __syncthreads();
+        if (lane == 0) {
+            sm.red[2 * warp] = zk;
+            sm.red[2 * warp + 1] = zt;
+        }
+        __syncthreads();
+        zk = warp_sum(lane < nw ? sm.red[2 * lane] : 0.f);
+        zt = warp_sum(lane < nw ? sm.red[2 * lane + 1] : 0.f);
+    }
     if (threadIdx.x == 0) {
         if (written != kept) raise_status(p.status, TKA_DEV_INTERNAL);
         p.stats[row] = make_float4(m, zk, zt, 0.f);
@@ -223,15 +235,16 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
     return m;
 }
 
-__global__ void __launch_bounds__(kSelectThreads, 1) select_topk(SelectParams p) {
+__global__ void __launch_bounds__(kSelectThreads, kSelectCtasPerSm) select_topk(SelectParams p) {
     extern __shared__ __align__(16) uint32_t dyn[];
     SelectSmem sm;
     sm.hist = dyn;                                                   // [2048]
     sm.tmp = dyn + 2048;                                             // [32]
-    sm.red = reinterpret_cast<float *>(dyn + 2048 + 32);             // [32]
-    sm.scal = dyn + 2048 + 64;                                       // [8]
-    uint32_t *wstat = dyn + 2048 + 72;                               // [kWarps][8]
+    sm.red = reinterpret_cast<float *>(dyn + 2048 + 32);             // [64]
+    sm.scal = dyn + 2048 + 96;                                       // [8]
+    uint32_t *wstat = dyn + 2048 + 104;                              // [kWarps][8]
     uint32_t *wc_key = wstat + kWarps * 8;                           // [kWarps][kWarpCand]
+    uint32_t *hist2 = wc_key + kWarps * kWarpCand;                   // [2048] second radix histogram
 
     const int row = blockIdx.x;
     const int b = row / (p.Q * p.Hq), qpos = (row / p.Hq) % p.Q;
@@ -301,7 +314,9 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_topk(SelectParams p)
     nsample = warp_sum(nsample);
     if (lane == 0) wstat[warp * 8 + 6] = nsample;
     m = block_max(m, sm.red);  // contains __syncthreads
-    const uint32_t total_sample = warp_sum(wstat[lane * 8 + 6]);  // kWarps == 32
+    // word f of the lane-th warp (0 past the last warp), for warp-wide reductions
+    auto wword = [&](int f) { return lane < kWarps ? wstat[lane * 8 + f] : 0u; };
+    const uint32_t total_sample = warp_sum(wword(6));
     // bins above b_hi are kept; bins [b_lo, b_hi] hold the candidates.  On the
     // sample the k-th key has rank about k * nsample / vis; the range is
     // widened by 4 binomial standard deviations each way and checked exactly
@@ -312,10 +327,18 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_topk(SelectParams p)
         const float margin = sampled ? 4.f * sqrtf(ks) + 4.f : 0.f;
         const uint32_t need_hi = (uint32_t)fmaxf(1.f, floorf(ks - margin));
         const uint32_t need_lo = (uint32_t)fminf((float)total_sample, ceilf(ks + margin));
-        find_bin(sm.hist, 2048, need_hi, sm.tmp, &sm.scal[0], &sm.scal[1]);
-        const uint32_t b_hi = sm.scal[0];
-        find_bin(sm.hist, 2048, max(need_lo, need_hi), sm.tmp, &sm.scal[0], &sm.scal[1]);
-        const uint32_t b_lo = sm.scal[0];
+        __syncthreads();
+        if (warp == 0) {
+            uint32_t bh, bl, unused;
+            warp_find_bin<2048>(sm.hist, need_hi, bh, unused);
+            warp_find_bin<2048>(sm.hist, max(need_lo, need_hi), bl, unused);
+            if (lane == 0) {
+                sm.scal[0] = bh;
+                sm.scal[1] = bl;
+            }
+        }
+        __syncthreads();
+        const uint32_t b_hi = sm.scal[0], b_lo = sm.scal[1];
         // a NaN threshold compares false: nothing above bin 2044 (+inf) or below bin 4 (-FLT_MAX)
         hi_t = b_hi >= 2044u ? __uint_as_float(0x7fc00000u) : key_float((b_hi + 1u) << 21);
         lo_t = key_float(b_lo << 21);
@@ -342,9 +365,9 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_topk(SelectParams p)
     if (lane == 0) wstat[warp * 8 + 0] = nwin;
     __syncthreads();
     // block totals, every warp reducing the per-warp words (lane w reads warp w's)
-    const uint32_t above = warp_sum(wstat[lane * 8 + 0]);
-    const uint32_t ncand = warp_sum(wstat[lane * 8 + 1]);
-    const bool overflow = __any_sync(0xffffffffu, wstat[lane * 8 + 1] > (uint32_t)kWarpCand);
+    const uint32_t above = warp_sum(wword(0));
+    const uint32_t ncand = warp_sum(wword(1));
+    const bool overflow = __any_sync(0xffffffffu, wword(1) > (uint32_t)kWarpCand);
     if (overflow || above >= (uint32_t)k || above + ncand < (uint32_t)k) {
         // the sampled range missed the k-th key or a warp's list overflowed:
         // take the exact multi-pass route
@@ -357,18 +380,37 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_topk(SelectParams p)
     // 10 bits): r of them are kept
     const uint32_t need = (uint32_t)k - above;
     uint32_t pre = 0u, gt = 0u, T = 0u;
+    // two histograms: level L counts into sm.hist (L even) or hist2 (L odd)
+    // while the other one is cleared for level L + 1; warp 0 searches between
+    // two barriers
+    for (int i = threadIdx.x; i < 2048; i += kSelectThreads) {
+        sm.hist[i] = 0u;
+        hist2[i] = 0u;
+    }
+    __syncthreads();
     for (int level = 0; level < 3; level++) {
         const int shift = level == 0 ? 21 : (level == 1 ? 10 : 0);
-        const int nb = level == 2 ? 1024 : 2048;
-        for (int i = threadIdx.x; i < 2048; i += kSelectThreads) sm.hist[i] = 0u;
-        __syncthreads();
+        const uint32_t nbm = level == 2 ? 1023u : 2047u;
+        uint32_t *h = (level & 1) ? hist2 : sm.hist;
         for (uint32_t i = lane; i < wstat[warp * 8 + 1]; i += 32) {  // this warp's own list
             const uint32_t key = canon_key(__uint_as_float(my_key[i]));
-            if (level == 0 || (key >> (shift + (level == 1 ? 11 : 10))) == pre)
-                atomicAdd(&sm.hist[(key >> shift) & (uint32_t)(nb - 1)], 1u);
+            if (level == 0 || (key >> (shift + (level == 1 ? 11 : 10))) == pre) atomicAdd(&h[(key >> shift) & nbm], 1u);
+        }
+        if (level == 1)
+            for (int i = threadIdx.x; i < 2048; i += kSelectThreads) sm.hist[i] = 0u;
+        __syncthreads();
+        if (warp == 0) {
+            uint32_t bin, above_bin;
+            if (level == 2)
+                warp_find_bin<1024>(h, need - gt, bin, above_bin);
+            else
+                warp_find_bin<2048>(h, need - gt, bin, above_bin);
+            if (lane == 0) {
+                sm.scal[0] = bin;
+                sm.scal[1] = above_bin;
+            }
         }
         __syncthreads();
-        find_bin(sm.hist, nb, need - gt, sm.tmp, &sm.scal[0], &sm.scal[1]);
         const uint32_t bin = sm.scal[0];
         gt += sm.scal[1];
         if (level < 2)
@@ -399,9 +441,9 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_topk(SelectParams p)
     // above T and the ties at T that fall among the first r_eq of the row
     uint32_t out_run, tie_run, n_eq;
     {
-        const uint32_t tie_l = wstat[lane * 8 + 3];
+        const uint32_t tie_l = wword(3);
         const uint32_t tie_incl = warp_incl_scan(tie_l), tie_excl = tie_incl - tie_l;
-        const uint32_t kept_l = wstat[lane * 8 + 0] + wstat[lane * 8 + 2] +
+        const uint32_t kept_l = wword(0) + wword(2) +
                                 (r_eq > tie_excl ? min(tie_l, r_eq - tie_excl) : 0u);
         const uint32_t out_incl = warp_incl_scan(kept_l);
         out_run = __shfl_sync(0xffffffffu, out_incl - kept_l, warp);
@@ -457,14 +499,14 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_topk(SelectParams p)
     }
     if (lane == 0) wstat[warp * 8 + 4] = out_run - out_begin;
     __syncthreads();
-    const uint32_t written = warp_sum(wstat[lane * 8 + 4]);
+    const uint32_t written = warp_sum(wword(4));
     finish_row(p, row, m, zk, zt, written, (uint32_t)k, sm);
 }
 
 }  // namespace
 
 size_t select_smem_bytes(int) {
-    return (size_t)(2048 + 72 + kWarps * 8) * 4 + (size_t)kWarps * kWarpCand * 4;
+    return (size_t)(2048 + 104 + kWarps * 8) * 4 + (size_t)kWarps * kWarpCand * 4 + 2048 * 4;
 }
 
 cudaError_t launch_select(const SelectParams &p, cudaStream_t stream) {
