@@ -52,6 +52,8 @@ def _load():
         lib.oracle_row_scores.restype = _i
         lib.oracle_topk_attn.argtypes = [_i] * 7 + [_d, _vp, _vp, _vp, _ip, _i, _dp, _ip, _dp, _dp, _i]
         lib.oracle_topk_attn.restype = _i
+        lib.oracle_certified_attn.argtypes = [_i] * 7 + [_d, _vp, _vp, _vp, _ip, _d, _i, _dp, _ip, _dp, _ip, _i]
+        lib.oracle_certified_attn.restype = _i
         lib.oracle_block_pool.argtypes = [_i] * 5 + [_vp, _ip, _i, _dp]
         lib.oracle_block_pool.restype = _i
         lib.oracle_block_attn.argtypes = [_i] * 6 + [_d, _vp, _vp, _vp, _ip, _i, _i, _dp, _ip, _dp, _dp, _i]
@@ -95,6 +97,27 @@ def topk_attn(w, k: int, scale: float = 0.0, nthreads: int = 0) -> dict:
     if rc:
         raise ValueError(f"oracle_topk_attn failed with code {rc}")
     return dict(out=out, idx=idx, tail=tail, kth=kth)
+
+
+def certified_attn(w, eps: float, k_max: int, scale: float = 0.0, nthreads: int = 0) -> dict:
+    """Certified adaptive Top-k decode attention over every row of ``w``.
+
+    Per row the smallest k (at most min(k_max, vis)) whose discarded softmax
+    tail mass is <= eps.  Returns out [B,Q,Hq,d] f64, idx [B,Q,Hq,k_max]
+    int32 (ascending, -1 padded), tail [B,Q,Hq] f64 and k_used [B,Q,Hq] int32.
+    """
+    lib = _load()
+    q, kc, vc, lens = _arr(w, w.q), _arr(w, w.k_cache), _arr(w, w.v_cache), _lens(w)
+    out = np.zeros((w.B, w.Q, w.Hq, w.d), np.float64)
+    idx = np.zeros((w.B, w.Q, w.Hq, k_max), np.int32)
+    tail = np.zeros((w.B, w.Q, w.Hq), np.float64)
+    k_used = np.zeros((w.B, w.Q, w.Hq), np.int32)
+    rc = lib.oracle_certified_attn(w.B, w.Q, w.Hq, w.Hkv, w.d, w.L_max, _code(w.dtype), scale,
+                                   q.ctypes.data, kc.ctypes.data, vc.ctypes.data, lens, eps, k_max,
+                                   out, idx, tail, k_used, nthreads)
+    if rc:
+        raise ValueError(f"oracle_certified_attn failed with code {rc}")
+    return dict(out=out, idx=idx, tail=tail, k_used=k_used)
 
 
 def row_scores(w, b: int, qpos: int, h: int, scale: float = 0.0) -> np.ndarray:

@@ -116,6 +116,30 @@ int oracle_row_scores(int B, int Q, int Hq, int Hkv, int d, int L_max, int dtype
 }
 
 /*
+ * Steps 3-6 for one row whose visible positions are already in (score
+ * descending, position ascending) order in sp[0..vis): keep the first kk,
+ * softmax over them, P.V, the discarded mass and the ascending idx (padded
+ * with -1 up to idx_len).  sel is scratch of vis entries.
+ */
+static void attend_prefix(const scored_pos *sp, int vis, int kk, const void *v_cache, int dtype, size_t voff,
+                          int d, double *o, double *tail_r, int32_t *ir, int idx_len, int32_t *sel) {
+    double m = sp[0].s;
+    double z_k = 0.0, z_tail = 0.0;
+    for (int j = 0; j < kk; j++) z_k += exp(sp[j].s - m);
+    for (int j = kk; j < vis; j++) z_tail += exp(sp[j].s - m);
+    for (int c = 0; c < d; c++) o[c] = 0.0;
+    for (int j = 0; j < kk; j++) {
+        double p = exp(sp[j].s - m) / z_k;
+        const size_t row = voff + (size_t)sp[j].i * d;
+        for (int c = 0; c < d; c++) o[c] += p * load_elem(v_cache, dtype, row + c);
+    }
+    if (tail_r) *tail_r = z_tail / (z_k + z_tail);
+    for (int j = 0; j < kk; j++) sel[j] = sp[j].i;
+    qsort(sel, (size_t)kk, sizeof(int32_t), cmp_int_asc);
+    for (int j = 0; j < idx_len; j++) ir[j] = j < kk ? sel[j] : -1;
+}
+
+/*
  * Token Top-k decode attention over all rows.
  *   out [B,Q,Hq,d], idx [B,Q,Hq,k], tail [B,Q,Hq], kth_score [B,Q,Hq] (the
  *   smallest kept score; -inf-free: equals the row minimum when k >= vis).
@@ -153,28 +177,81 @@ int oracle_topk_attn(int B, int Q, int Hq, int Hkv, int d, int L_max, int dtype,
             for (int i = 0; i < vis; i++) { sp[i].s = s[i]; sp[i].i = i; }
             qsort(sp, (size_t)vis, sizeof(scored_pos), cmp_score_desc);
             int kk = k < vis ? k : vis;
-            /* 3. normalisers */
-            double m = sp[0].s;
-            double z_k = 0.0, z_tail = 0.0;
-            for (int j = 0; j < kk; j++) z_k += exp(sp[j].s - m);
-            for (int j = kk; j < vis; j++) z_tail += exp(sp[j].s - m);
-            /* 4. P.V over the kept rows */
-            double *o = out + (size_t)r * d;
-            for (int c = 0; c < d; c++) o[c] = 0.0;
+            /* 3.-6. normalisers, P.V over the kept rows, discarded mass, idx */
             size_t voff = ((size_t)b * Hkv + kvh) * (size_t)L_max * d;
-            for (int j = 0; j < kk; j++) {
-                double p = exp(sp[j].s - m) / z_k;
-                const size_t row = voff + (size_t)sp[j].i * d;
-                for (int c = 0; c < d; c++) o[c] += p * load_elem(v_cache, dtype, row + c);
-            }
-            /* 5. discarded mass */
-            if (tail) tail[r] = z_tail / (z_k + z_tail);
+            attend_prefix(sp, vis, kk, v_cache, dtype, voff, d, out + (size_t)r * d, tail ? tail + r : NULL,
+                          idx + (size_t)r * k, k, sel);
             if (kth_score) kth_score[r] = sp[kk - 1].s;
-            /* 6. ascending positions, -1 padding */
-            for (int j = 0; j < kk; j++) sel[j] = sp[j].i;
-            qsort(sel, (size_t)kk, sizeof(int32_t), cmp_int_asc);
-            int32_t *ir = idx + (size_t)r * k;
-            for (int j = 0; j < k; j++) ir[j] = j < kk ? sel[j] : -1;
+        }
+        free(sp);
+        free(s);
+        free(sel);
+    }
+    return status;
+}
+
+/*
+ * Certified adaptive Top-k ("A Mathematical Theory of Top-k Sparse Attention
+ * via Total Variation Distance", abstract): the truncation error of Top-k
+ * attention in total variation is the discarded softmax tail mass
+ * tau_k = 1 - Z_k / Z, so the certified k of a row is the smallest k with
+ * tau_k <= eps.  Per row, over the same (score descending, position
+ * ascending) order as oracle_topk_attn:
+ *   k_used = min{ k >= 1 : 1 - (sum_{j < k} e^{s_(j) - m}) / Z <= eps }, capped
+ *   at min(k_max, vis) (when even that many keys leave more than eps outside,
+ *   the cap is used and the returned tail exceeds eps);
+ * then out, tail and idx exactly as oracle_topk_attn with k = k_used, idx
+ * padded with -1 up to k_max.  k_used [B,Q,Hq] int32; tail may be NULL.
+ */
+int oracle_certified_attn(int B, int Q, int Hq, int Hkv, int d, int L_max, int dtype, double scale,
+                          const void *q, const void *k_cache, const void *v_cache, const int32_t *seq_lens,
+                          double eps, int k_max, double *out, int32_t *idx, double *tail, int32_t *k_used,
+                          int nthreads) {
+    if (!check_shape(B, Q, Hq, Hkv, d, L_max, dtype) || k_max < 1 || !(eps >= 0.0) || eps >= 1.0) return OR_BAD_ARG;
+    for (int b = 0; b < B; b++)
+        if (seq_lens[b] > L_max || visible(seq_lens[b], Q, 0) < 1) return OR_BAD_ARG;
+    const int G = Hq / Hkv;
+    const long rows = (long)B * Q * Hq;
+    int status = OR_OK;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+#pragma omp parallel
+    {
+        scored_pos *sp = (scored_pos *)malloc(sizeof(scored_pos) * (size_t)L_max);
+        double *s = (double *)malloc(sizeof(double) * (size_t)L_max);
+        int32_t *sel = (int32_t *)malloc(sizeof(int32_t) * (size_t)L_max);
+        if (!sp || !s || !sel) {
+#pragma omp atomic write
+            status = OR_NO_MEMORY;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (long r = 0; r < rows; r++) {
+            if (!sp || !s || !sel) continue;
+            int h = (int)(r % Hq), qpos = (int)((r / Hq) % Q), b = (int)(r / ((long)Hq * Q));
+            int kvh = h / G;
+            int vis = oracle_row_scores(B, Q, Hq, Hkv, d, L_max, dtype, scale, q, k_cache, seq_lens,
+                                        b, qpos, h, s);
+            for (int i = 0; i < vis; i++) { sp[i].s = s[i]; sp[i].i = i; }
+            qsort(sp, (size_t)vis, sizeof(scored_pos), cmp_score_desc);
+            double m = sp[0].s;
+            double z = 0.0;
+            for (int j = 0; j < vis; j++) z += exp(sp[j].s - m);
+            /* the smallest prefix of the order whose discarded mass is <= eps */
+            int cap = k_max < vis ? k_max : vis;
+            int kk = cap;
+            double z_k = 0.0;
+            for (int j = 0; j < cap; j++) {
+                z_k += exp(sp[j].s - m);
+                if (1.0 - z_k / z <= eps) {
+                    kk = j + 1;
+                    break;
+                }
+            }
+            size_t voff = ((size_t)b * Hkv + kvh) * (size_t)L_max * d;
+            attend_prefix(sp, vis, kk, v_cache, dtype, voff, d, out + (size_t)r * d, tail ? tail + r : NULL,
+                          idx + (size_t)r * k_max, k_max, sel);
+            k_used[r] = kk;
         }
         free(sp);
         free(s);

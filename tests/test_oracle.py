@@ -336,3 +336,86 @@ def test_block_attention_over_kept_tokens():
     P = torch.softmax(torch.from_numpy(torch_scores(w)), dim=-1).numpy()
     kept_mass = (P * mask.transpose(1, 2).numpy()).sum(-1)
     np.testing.assert_allclose(r["tail"], 1 - kept_mass, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- certified adaptive Top-k
+
+def test_certified_large_eps_keeps_only_the_argmax():
+    w = workloads.make_workload(2, 2, 8, 4, 300, dtype="bf16", seq_lens=[300, 211], seed=61)
+    r = oracle.certified_attn(w, eps=1.0 - 1e-12, k_max=64)
+    s = torch_scores(w)
+    assert np.all(r["k_used"] == 1)
+    for b in range(2):
+        for qp in range(2):
+            for h in range(8):
+                j = int(np.argmax(s[b, qp, h]))
+                assert r["idx"][b, qp, h, 0] == j and np.all(r["idx"][b, qp, h, 1:] == -1)
+                np.testing.assert_array_equal(r["out"][b, qp, h], _f64(w.v_cache[b, h // 2, j]).numpy())
+
+
+def test_certified_zero_eps_is_dense_attention():
+    w = workloads.make_workload(2, 3, 4, 2, 90, dtype="f32", seq_lens=[90, 41], seed=62)
+    r = oracle.certified_attn(w, eps=0.0, k_max=90)
+    np.testing.assert_allclose(r["out"], dense_sdpa(w), rtol=1e-12, atol=1e-12)
+    for b in range(2):
+        for qp in range(3):
+            assert np.all(r["k_used"][b, qp] == int(w.seq_lens[b]) - 3 + qp + 1)
+    assert np.all(r["tail"] == 0.0)
+
+
+@pytest.mark.parametrize("eps,k_max", [(0.3, 600), (0.05, 600), (0.5, 40), (0.2, 150)])
+def test_certified_k_is_the_smallest_certified_prefix(eps, k_max):
+    """Brute force on softmax probabilities from torch: the kept set is the
+    lexsort top-k_used, its discarded mass is <= eps, and one key fewer would
+    leave more than eps outside (unless k_used is at the cap)."""
+    w = workloads.make_workload(2, 2, 4, 2, 600, dtype="bf16", seq_lens=[600, 350], k_mean_std=0.5, seed=63)
+    r = oracle.certified_attn(w, eps=eps, k_max=k_max)
+    s = torch_scores(w)
+    P = torch.softmax(torch.from_numpy(s), dim=-1).numpy()
+    for b in range(2):
+        for qp in range(2):
+            for h in range(4):
+                vis = int(w.seq_lens[b]) - 2 + qp + 1
+                ku = int(r["k_used"][b, qp, h])
+                sel = lexsort_topk(s[b, qp, h], ku)
+                got = r["idx"][b, qp, h]
+                assert np.array_equal(got[:ku], sel) and np.all(got[ku:] == -1)
+                order = np.lexsort((np.arange(vis), -s[b, qp, h, :vis]))
+                cum = np.cumsum(P[b, qp, h][order])
+                tau = 1.0 - cum[ku - 1]
+                assert abs(r["tail"][b, qp, h] - tau) < 1e-12
+                cap = min(k_max, vis)
+                if ku < cap or tau <= eps:
+                    assert tau <= eps + 1e-12
+                else:
+                    assert ku == cap and tau > eps  # not certifiable within the cap
+                if ku > 1:
+                    assert 1.0 - cum[ku - 2] > eps - 1e-12
+
+
+def test_certified_minimal_k_follows_the_gaussian_rule():
+    # i.i.d. Gaussian scores N(0, sigma^2), sigma = |q|/sqrt(d): the smallest
+    # k with tail mass <= eps satisfies k/n ~ 1 - Phi(sigma + Phi^{-1}(eps)).
+    from scipy.stats import norm
+    errs = []
+    for seed in range(32):
+        w = workloads.make_workload(1, 1, 1, 1, 4096, dtype="f32", seed=7000 + seed)
+        r = oracle.certified_attn(w, eps=0.2, k_max=4096)
+        sigma = float(torch.linalg.vector_norm(_f64(w.q[0, 0, 0]))) / math.sqrt(128)
+        pred = norm.sf(sigma + norm.ppf(0.2))
+        errs.append(r["k_used"][0, 0, 0] / 4096 - pred)
+    errs = np.array(errs)
+    assert abs(errs.mean()) < 0.01, errs.mean()
+    assert np.abs(errs).max() < 0.05, np.abs(errs).max()
+
+
+def test_certified_equals_fixed_k_at_the_chosen_k():
+    w = workloads.make_workload(1, 2, 4, 1, 500, dtype="bf16", seed=64)
+    r = oracle.certified_attn(w, eps=0.25, k_max=500)
+    for qp in range(2):
+        for h in range(4):
+            ku = int(r["k_used"][0, qp, h])
+            f = oracle.topk_attn(w, k=ku)
+            np.testing.assert_array_equal(r["out"][0, qp, h], f["out"][0, qp, h])
+            np.testing.assert_array_equal(r["idx"][0, qp, h, :ku], f["idx"][0, qp, h])
+            assert r["tail"][0, qp, h] == f["tail"][0, qp, h]

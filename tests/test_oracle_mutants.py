@@ -19,14 +19,20 @@ MUTANTS = {
     "scale_dropped": ("s_out[i] = sc * acc;", "s_out[i] = acc;"),
     "gqa_head_map_modulo": ("int G = Hq / Hkv, kvh = h / G;", "int G = Hq / Hkv, kvh = h % Hkv; (void)G;"),
     "ties_to_higher_position": ("return (x->i > y->i) - (x->i < y->i);", "return (x->i < y->i) - (x->i > y->i);"),
-    "tail_over_kept_mass": ("tail[r] = z_tail / (z_k + z_tail);", "tail[r] = z_tail / z_k;"),
+    "tail_over_kept_mass": ("*tail_r = z_tail / (z_k + z_tail);", "*tail_r = z_tail / z_k;"),
     "softmax_over_all_keys": ("double p = exp(sp[j].s - m) / z_k;", "double p = exp(sp[j].s - m) / (z_k + z_tail);"),
     "causal_off_by_one": ("return seq_len - Q + qpos + 1;", "return seq_len - Q + qpos + (qpos > 0);"),
-    "values_from_keys": ("o[c] += p * load_elem(v_cache, dtype, row + c);", "o[c] += p * load_elem(k_cache, dtype, row + c);"),
+    "values_from_keys": ("attend_prefix(sp, vis, kk, v_cache, dtype, voff, d, out + (size_t)r * d, tail ? tail + r : NULL,\n"
+                         "                          idx + (size_t)r * k, k, sel);",
+                         "attend_prefix(sp, vis, kk, k_cache, dtype, voff, d, out + (size_t)r * d, tail ? tail + r : NULL,\n"
+                         "                          idx + (size_t)r * k, k, sel);"),
     "q_index_transposed": ("size_t qoff = (((size_t)b * Q + qpos) * Hq + h) * d;",
                            "size_t qoff = (((size_t)b * Hq + h) * Q + qpos) * d;"),
     "block_mean_over_full_size": ("bk[(size_t)j * d + c] = hi > lo ? acc / (double)(hi - lo) : 0.0;",
                                   "bk[(size_t)j * d + c] = hi > lo ? acc / (double)block_size : 0.0;"),
+    "certified_k_one_too_many": ("                    kk = j + 1;\n", "                    kk = j + 1 < cap ? j + 2 : cap;\n"),
+    "certified_mass_of_capped_prefix": ("for (int j = 0; j < vis; j++) z += exp(sp[j].s - m);",
+                                        "for (int j = 0; j < (k_max < vis ? k_max : vis); j++) z += exp(sp[j].s - m);"),
     "current_block_not_forced": ("kept[nk] = nblk - 1; /* the current block */",
                                  "kept[nk] = nk < nblk - 1 ? sp[nk].i : nblk - 1;"),
 }
