@@ -18,6 +18,7 @@ from ._binding import (  # noqa: F401
     library_path,
     load_library,
     topk_attn_decode,
+    topk_attn_decode_certified,
     topk_attn_decode_static,
     topk_attn_static_workspace_capacity,
     topk_attn_device_status,

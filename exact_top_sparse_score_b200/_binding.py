@@ -53,6 +53,9 @@ def load_library() -> ctypes.CDLL:
         lib.topk_attn_decode_staged.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp,
                                                 ctypes.POINTER(_vp)]
         lib.topk_attn_decode_staged.restype = ctypes.c_int
+        lib.topk_attn_decode_certified.argtypes = [_shape_p, _vp, _vp, _vp, _vp, ctypes.c_float, _i32, _vp, _vp,
+                                                   _vp, _vp, _vp, _sz, _vp]
+        lib.topk_attn_decode_certified.restype = ctypes.c_int
         lib.topk_attn_static_workspace_capacity.argtypes = []
         lib.topk_attn_static_workspace_capacity.restype = _sz
         lib.topk_attn_decode_static.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp]
@@ -199,6 +202,52 @@ def topk_attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tens
     if rc:
         raise TopkAttnError("topk_attn_decode", rc)
     return out, idx, tail_mass
+
+
+def topk_attn_decode_certified(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                               seq_lens: torch.Tensor, eps: float, k_max: int, *, scale: float = 0.0,
+                               out: Optional[torch.Tensor] = None, idx: Optional[torch.Tensor] = None,
+                               tail_mass: Optional[torch.Tensor] = None, k_used: Optional[torch.Tensor] = None,
+                               workspace: Optional[torch.Tensor] = None, stream=None):
+    """Certified adaptive Top-k decode attention: per row the smallest k (at
+    most k_max) whose discarded softmax tail mass is <= eps.  Returns
+    (out fp32 [B,Q,Hq,d], idx int32 [B,Q,Hq,k_max], tail fp32 [B,Q,Hq],
+    k_used int32 [B,Q,Hq])."""
+    lib = load_library()
+    shape = make_shape(q, k_cache, scale)
+    B, Q, Hq, d = q.shape
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, Q, Hq, d), dtype=torch.float32, device=dev)
+    if idx is None:
+        idx = torch.empty((B, Q, Hq, k_max), dtype=torch.int32, device=dev)
+    if tail_mass is None:
+        tail_mass = torch.empty((B, Q, Hq), dtype=torch.float32, device=dev)
+    if k_used is None:
+        k_used = torch.empty((B, Q, Hq), dtype=torch.int32, device=dev)
+    if seq_lens.dtype != torch.int32 or tuple(seq_lens.shape) != (B,):
+        raise TypeError("seq_lens must be int32 [B]")
+    if v_cache.dtype != k_cache.dtype or v_cache.shape != k_cache.shape:
+        raise TypeError("v_cache must match k_cache in dtype and shape")
+    _check_out("out", out, torch.float32, (B, Q, Hq, d))
+    _check_out("idx", idx, torch.int32, (B, Q, Hq, k_max))
+    _check_out("tail_mass", tail_mass, torch.float32, (B, Q, Hq))
+    _check_out("k_used", k_used, torch.int32, (B, Q, Hq))
+    if workspace is not None and workspace.dtype != torch.uint8:
+        raise TypeError("workspace must be a uint8 tensor")
+    _check_cuda(q=q, k_cache=k_cache, v_cache=v_cache, seq_lens=seq_lens, out=out, idx=idx, tail_mass=tail_mass,
+                k_used=k_used, workspace=workspace)
+    nbytes = topk_attn_workspace_size(shape, k_max)
+    if nbytes == 0:
+        raise TopkAttnError("topk_attn_workspace_size", 2)
+    sh = _stream(stream)
+    ws = _workspace(nbytes, dev, workspace, sh)
+    rc = lib.topk_attn_decode_certified(ctypes.byref(shape), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                        seq_lens.data_ptr(), float(eps), k_max, out.data_ptr(), idx.data_ptr(),
+                                        tail_mass.data_ptr(), k_used.data_ptr(), ws.data_ptr(), nbytes, sh)
+    if rc:
+        raise TopkAttnError("topk_attn_decode_certified", rc)
+    return out, idx, tail_mass, k_used
 
 
 def topk_attn_decode_static(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, seq_lens: torch.Tensor,

@@ -13,7 +13,6 @@ namespace {
 __device__ unsigned int g_status = 0u;
 
 constexpr int kMaxDevices = 64;
-constexpr int kMaxK = 8192;
 constexpr int kMaxQ = 64;
 constexpr int kMaxRowsPerKvHead = 256;  // Q * G
 constexpr int kMaxLen = 1 << 24;
@@ -163,10 +162,21 @@ size_t topk_attn_workspace_size(const tka_shape *shape, int32_t k) {
     return token_layout(shape, k).total;
 }
 
-tka_status topk_attn_decode_staged(const tka_shape *shape, const void *q, const void *k_cache,
-                                   const void *v_cache, const int32_t *seq_lens, int32_t k, float *out,
-                                   int32_t *idx, float *tail_mass, void *workspace, size_t workspace_bytes,
-                                   tka_stream_t stream, const tka_event_t events[4]) {
+}  // extern "C"
+
+namespace {
+
+// The certified variant's extra arguments (null for a fixed k).
+struct CertArgs {
+    float eps;
+    int32_t *k_used;
+};
+
+// Score -> select (k) -> [certify] -> gather on `stream`.
+tka_status decode_impl(const tka_shape *shape, const void *q, const void *k_cache, const void *v_cache,
+                       const int32_t *seq_lens, int32_t k, float *out, int32_t *idx, float *tail_mass,
+                       void *workspace, size_t workspace_bytes, tka_stream_t stream, const tka_event_t events[4],
+                       const CertArgs *cert) {
     tka_status st = check_shape(shape);
     if (st != TKA_OK) return st;
     if (k < 1) return TKA_ERR_INVALID_ARG;
@@ -228,6 +238,21 @@ tka_status topk_attn_decode_staged(const tka_shape *shape, const void *q, const 
     se.tail = tail_mass;
     se.counters = reinterpret_cast<unsigned *>(ws + L.counters);
     if (launch_select(se, s) != cudaSuccess) return TKA_ERR_CUDA;
+    if (cert) {
+        CertifyParams cp;
+        cp.status = dev->status;
+        cp.scores = scores;
+        cp.seq_lens = seq_lens;
+        cp.B = shape->B; cp.Q = shape->Q; cp.Hq = shape->Hq; cp.L_max = shape->L_max; cp.ld = L.ld;
+        cp.k_max = k;
+        cp.eps = cert->eps;
+        cp.idx = idx;
+        cp.w = se.w;
+        cp.stats = se.stats;
+        cp.tail = tail_mass;
+        cp.k_used = cert->k_used;
+        if (launch_certify(cp, s) != cudaSuccess) return TKA_ERR_CUDA;
+    }
     if (record(events, 2, s) != cudaSuccess) return TKA_ERR_CUDA;
 
     GatherParams gp;
@@ -242,6 +267,7 @@ tka_status topk_attn_decode_staged(const tka_shape *shape, const void *q, const 
     gp.partial = reinterpret_cast<float *>(ws + L.partial);
     gp.counters = se.counters;
     gp.out = out;
+    gp.kcount = cert ? cert->k_used : nullptr;
     // one wave of eight CTAs per SM (splits = floor(8 x SMs / rows), at least 1),
     // never fewer than kMinKeysPerSplit keys per CTA
     int splits = (dev->num_sms * 8) / rows;
@@ -252,6 +278,28 @@ tka_status topk_attn_decode_staged(const tka_shape *shape, const void *q, const 
     if (launch_gather(gp, s) != cudaSuccess) return TKA_ERR_CUDA;
     if (record(events, 3, s) != cudaSuccess) return TKA_ERR_CUDA;
     return TKA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+tka_status topk_attn_decode_staged(const tka_shape *shape, const void *q, const void *k_cache,
+                                   const void *v_cache, const int32_t *seq_lens, int32_t k, float *out,
+                                   int32_t *idx, float *tail_mass, void *workspace, size_t workspace_bytes,
+                                   tka_stream_t stream, const tka_event_t events[4]) {
+    return decode_impl(shape, q, k_cache, v_cache, seq_lens, k, out, idx, tail_mass, workspace, workspace_bytes,
+                       stream, events, nullptr);
+}
+
+tka_status topk_attn_decode_certified(const tka_shape *shape, const void *q, const void *k_cache,
+                                      const void *v_cache, const int32_t *seq_lens, float eps, int32_t k_max,
+                                      float *out, int32_t *idx, float *tail_mass, int32_t *k_used,
+                                      void *workspace, size_t workspace_bytes, tka_stream_t stream) {
+    if (!(eps >= 0.f) || !(eps < 1.f) || !k_used || !aligned(k_used, 4)) return TKA_ERR_INVALID_ARG;
+    const CertArgs cert{eps, k_used};
+    return decode_impl(shape, q, k_cache, v_cache, seq_lens, k_max, out, idx, tail_mass, workspace,
+                       workspace_bytes, stream, nullptr, &cert);
 }
 
 tka_status topk_attn_decode(const tka_shape *shape, const void *q, const void *k_cache, const void *v_cache,

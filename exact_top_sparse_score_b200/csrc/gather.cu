@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(kGatherThreads, 8) gather_pv(GatherParams p) {
     const int seq_len = p.seq_lens[b];
     if (!seq_len_ok(seq_len, p.Q, p.L_max)) return;  // the select step raised the status
     const int vis = visible_keys(seq_len, p.Q, qpos);
-    const int kept = p.k < vis ? p.k : vis;
+    const int kept = p.kcount ? min(p.kcount[row], min(p.k, vis)) : min(p.k, vis);
     const int lo = split * p.per_split;
     const int hi = min(kept, lo + p.per_split);
 

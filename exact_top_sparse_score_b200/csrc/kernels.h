@@ -7,6 +7,8 @@
 
 namespace tka {
 
+constexpr int kMaxK = 8192;  // largest k (and k_max) the select and certify steps take
+
 struct ScoreParams {
     unsigned *status;         // device status word (TKA_DEV_* bits)
     const void *q;            // [B, Q, Hq, 128]
@@ -49,6 +51,20 @@ struct GatherParams {
     unsigned *counters;       // [rows]
     float *out;               // [rows, 128]
     int splits, per_split;
+    const int32_t *kcount;    // [rows] kept positions per row, or null: min(k, visible keys)
+};
+
+struct CertifyParams {
+    unsigned *status;         // device status word (TKA_DEV_* bits)
+    const float *scores;      // [rows, ld]
+    const int32_t *seq_lens;
+    int B, Q, Hq, L_max, ld, k_max;
+    float eps;
+    int32_t *idx;             // [rows, k_max] in: the top k_max ascending; out: the certified prefix
+    float *w;                 // [rows, k_max] e^{s - m}, compacted like idx
+    float4 *stats;            // [rows] {m, Z_k, Z_tail, 0}, rewritten
+    float *tail;              // [rows] or null
+    int32_t *k_used;          // [rows]
 };
 
 struct BlockPoolParams {
@@ -105,6 +121,7 @@ cudaError_t launch_score_tc(const ScoreTcParams &p, const void *q, const void *k
 cudaError_t launch_select(const SelectParams &p, cudaStream_t stream);
 size_t select_smem_bytes(int k);
 cudaError_t launch_gather(const GatherParams &p, cudaStream_t stream);
+cudaError_t launch_certify(const CertifyParams &p, cudaStream_t stream);
 cudaError_t launch_block_pool(const BlockPoolParams &p, cudaStream_t stream);
 cudaError_t launch_block_select(const BlockSelectParams &p, cudaStream_t stream);
 cudaError_t launch_block_attn(const BlockAttnParams &p, const void *k_cache, int num_sms, cudaStream_t stream);

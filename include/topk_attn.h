@@ -108,6 +108,26 @@ tka_status topk_attn_decode_staged(const tka_shape *shape, const void *q, const 
                                    int32_t *idx, float *tail_mass, void *workspace, size_t workspace_bytes,
                                    tka_stream_t stream, const tka_event_t events[4]);
 
+/* Certified adaptive Top-k ("A Mathematical Theory of Top-k Sparse Attention
+ * via Total Variation Distance", abstract: the Top-k truncation error in total
+ * variation is the discarded softmax tail mass).  Per query row, k is the
+ * smallest number of keys, taken in (score descending, position ascending)
+ * order, whose discarded tail mass 1 - Z_k / Z is at most eps, capped at
+ * min(k_max, visible keys); when even k_max keys leave more than eps outside,
+ * the row keeps k_max and its tail_mass exceeds eps.  out, idx and tail_mass
+ * are then exactly those of topk_attn_decode with that row's k.
+ *   eps       in [0, 1); 0 keeps every visible key (when k_max allows).
+ *   k_max     1..8192; idx is int32 [B,Q,Hq,k_max], ascending, -1 padded
+ *             past the row's k.
+ *   k_used    int32 [B,Q,Hq] device buffer: each row's k.
+ *   workspace topk_attn_workspace_size(shape, k_max) bytes.
+ * Other arguments, layouts and errors as topk_attn_decode; eps outside
+ * [0, 1) or a missing k_used is TKA_ERR_INVALID_ARG. */
+tka_status topk_attn_decode_certified(const tka_shape *shape, const void *q, const void *k_cache,
+                                      const void *v_cache, const int32_t *seq_lens, float eps, int32_t k_max,
+                                      float *out, int32_t *idx, float *tail_mass, int32_t *k_used,
+                                      void *workspace, size_t workspace_bytes, tka_stream_t stream);
+
 /* topk_attn_decode without a workspace argument, for callers that cannot
  * allocate device memory (an engine that reserves all device memory for its
  * own pool and forbids other allocations while serving, or a host runtime with

@@ -126,3 +126,60 @@ def check_block(w, block_size, top_blocks, out, bidx, ref, scale=0.0):
             want = (e[:, None] * V).sum(0) / e.sum()
             assert _close(out[b, 0, h], want, atol, rtol).all(), f"{where}: out invalid for its own blocks"
     return n_band
+
+
+CERT_TOL = 1e-4  # slack on the eps comparison for fp32 scores and masses
+
+
+def check_certified(w, eps, k_max, out, idx, tail, k_used, ref, scale=0.0, rows_checked=None):
+    """Asserts parity of topk_attn_decode_certified with oracle.certified_attn output `ref`.
+
+    Every row: k_used is certified and minimal against the oracle's fp64 tail
+    masses (within CERT_TOL of eps, or at the cap); idx holds the top-k_used
+    positions (up to the tie band around the k_used-th score), ascending and
+    -1 padded; out and tail match an fp64 evaluation over the kept set.  Rows
+    whose k_used equals the oracle's compare idx, out and tail with it
+    directly.  Returns the number of rows whose k differs from the oracle's."""
+    out = out.detach().cpu().double().numpy()
+    idx = idx.detach().cpu().numpy()
+    tail = tail.detach().cpu().double().numpy()
+    k_used = k_used.detach().cpu().numpy()
+    atol, rtol = out_tol(w.dtype)
+    rows = rows_checked or [(b, qp, h) for b in range(w.B) for qp in range(w.Q) for h in range(w.Hq)]
+    n_diff = 0
+    for r_i, (b, qp, h) in enumerate(rows):
+        if rows_checked:
+            ro, ri, rt, rk = ref["out"][r_i], ref["idx"][r_i], ref["tail"][r_i], ref["k_used"][r_i]
+        else:
+            ro, ri, rt, rk = (ref["out"][b, qp, h], ref["idx"][b, qp, h], ref["tail"][b, qp, h],
+                              ref["k_used"][b, qp, h])
+        where = f"row (b={b}, q={qp}, h={h})"
+        vis = _vis(w, b, qp)
+        cap = min(k_max, vis)
+        kg = int(k_used[b, qp, h])
+        assert 1 <= kg <= cap, f"{where}: k_used {kg} outside [1, {cap}]"
+        s = oracle.row_scores(w, b, qp, h, scale)
+        order = np.lexsort((np.arange(vis), -s))
+        e = np.exp(s[order] - s[order[0]])
+        tau = 1.0 - np.cumsum(e) / e.sum()  # tau[j] = tail mass of the top j + 1
+        if kg < cap:
+            assert tau[kg - 1] <= eps + CERT_TOL, f"{where}: k={kg} leaves {tau[kg - 1]:.6f} > eps"
+        if kg > 1:
+            assert tau[kg - 2] > eps - CERT_TOL, f"{where}: k={kg} not minimal ({tau[kg - 2]:.6f} <= eps)"
+        g = idx[b, qp, h]
+        assert np.all(g[kg:] == -1), f"{where}: padding"
+        gs = g[:kg]
+        assert np.all(gs >= 0) and np.all(gs < vis) and np.all(np.diff(gs) > 0), f"{where}: kept list"
+        top = np.sort(order[:kg])
+        diff = np.setxor1d(gs, top)
+        kth = s[order[kg - 1]]
+        assert np.all(np.abs(s[diff] - kth) <= BAND), f"{where}: set differs outside the tie band"
+        if kg == rk and np.array_equal(gs, ri[:kg]):
+            assert _close(out[b, qp, h], ro, atol, rtol).all(), f"{where}: out"
+            assert abs(tail[b, qp, h] - rt) <= TAIL_TOL, f"{where}: tail {tail[b, qp, h]} vs {rt}"
+            continue
+        n_diff += kg != rk
+        vo, vt = _set_eval(w, s, gs, b, h)
+        assert _close(out[b, qp, h], vo, atol, rtol).all(), f"{where}: out invalid for its own set"
+        assert abs(tail[b, qp, h] - vt) <= TAIL_TOL, f"{where}: tail invalid for its own set"
+    return n_diff
