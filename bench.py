@@ -55,6 +55,9 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch size (smaller cases for profiling)")
+    ap.add_argument("--certified-eps", type=float, default=None,
+                    help="certified adaptive Top-k: per row the smallest k (at most the workload's k) "
+                         "whose discarded tail mass is <= EPS")
     return ap.parse_args()
 
 
@@ -73,11 +76,12 @@ def k_bytes(w):
     return sum(int(w.seq_lens[b]) for b in range(w.B)) * w.Hkv * w.d * elem_bytes(w)
 
 
-def alg_bytes_token(w, k):
+def alg_bytes_token(w, k, kept=None):
     """Algorithmic bytes of one step: full K read + the k kept K and V rows of
-    every query row + q, out, idx and tail."""
+    every query row (or `kept` rows in total) + q, out, idx and tail."""
     row = w.d * elem_bytes(w)
-    kept = sum(min(k, visible(w, b, qp)) for b in range(w.B) for qp in range(w.Q)) * w.Hq
+    if kept is None:
+        kept = sum(min(k, visible(w, b, qp)) for b in range(w.B) for qp in range(w.Q)) * w.Hq
     rows = w.B * w.Q * w.Hq
     return k_bytes(w) + kept * 2 * row + rows * w.d * (elem_bytes(w) + 4) + rows * (k * 4 + 4)
 
@@ -176,7 +180,7 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- CPU oracle
 
-def time_oracle(w, k, budget_s=10.0, max_reps=50):
+def time_oracle(w, k, budget_s=10.0, max_reps=50, eps=None):
     """The oracle as it stands on this host's cores, whole workload repeated
     until `budget_s` has elapsed.  Returns (queries/s, cores, sample text)."""
     import oracle
@@ -185,6 +189,8 @@ def time_oracle(w, k, budget_s=10.0, max_reps=50):
     while True:
         if w.variant == "block":
             oracle.block_attn(w, w.block_size, w.top_blocks)
+        elif eps is not None:
+            oracle.certified_attn(w, eps, k)
         else:
             oracle.topk_attn(w, k)
         reps += 1
@@ -225,6 +231,7 @@ def run_ours(args, world, rank, local):
     q, kc, vc, lens = (w.q.to(dev), w.k_cache.to(dev), w.v_cache.to(dev), w.seq_lens.to(dev))
     rows = w.B * w.Q * w.Hq
     block = w.variant == "block"
+    certified = args.certified_eps is not None and not block
     k = w.k
     if block:
         bk = tka.topk_block_pool_keys(kc, lens, w.block_size)
@@ -249,10 +256,21 @@ def run_ours(args, world, rank, local):
         idx = torch.empty((w.B, w.Q, w.Hq, k), dtype=torch.int32, device=dev)
         tail = torch.empty((w.B, w.Q, w.Hq), dtype=torch.float32, device=dev)
         launches_per_step = 3
+        if certified:
+            k_used = torch.empty((w.B, w.Q, w.Hq), dtype=torch.int32, device=dev)
+            launches_per_step = 4  # + certify
 
-        def step(events=None, qq=q):
-            tka.topk_attn_decode(qq, kc, vc, lens, k, out=out, idx=idx, tail_mass=tail, workspace=ws,
-                                 stage_events=events)
+            def step(events=None, qq=q):
+                if events:
+                    events[0].record()
+                tka.topk_attn_decode_certified(qq, kc, vc, lens, args.certified_eps, k, out=out, idx=idx,
+                                               tail_mass=tail, k_used=k_used, workspace=ws)
+                if events:
+                    events[3].record()
+        else:
+            def step(events=None, qq=q):
+                tka.topk_attn_decode(qq, kc, vc, lens, k, out=out, idx=idx, tail_mass=tail, workspace=ws,
+                                     stage_events=events)
         alg = alg_bytes_token(w, k)
         dominant_bytes = k_bytes(w) + q.numel() * q.element_size()
 
@@ -285,7 +303,7 @@ def run_ours(args, world, rank, local):
     if world > 1:
         torch.distributed.barrier()
     step_ms = [e[0].elapsed_time(e[3]) for e in evs]
-    stage_ms = None if block else [[e[j].elapsed_time(e[j + 1]) for e in evs] for j in range(3)]
+    stage_ms = None if block or certified else [[e[j].elapsed_time(e[j + 1]) for e in evs] for j in range(3)]
     total_ms = sum(step_ms)
 
     e2e_ms = None
@@ -297,7 +315,7 @@ def run_ours(args, world, rank, local):
         lens_host = w.seq_lens.pin_memory()
         q_step = torch.empty_like(q)
         lens_step = torch.empty_like(lens)
-        outs = [out, bidx] if block else [out, idx, tail]
+        outs = [out, bidx] if block else ([out, idx, tail, k_used] if certified else [out, idx, tail])
         hosts = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
         h2d = q_host.numel() * q_host.element_size() + lens_host.numel() * 4
         d2h = sum(t.numel() * t.element_size() for t in outs)
@@ -310,6 +328,9 @@ def run_ours(args, world, rank, local):
             if block:
                 tka.topk_block_attn_decode(q_step, kc, vc, bk, lens_step, w.block_size, w.top_blocks, out=out,
                                            block_idx=bidx, workspace=ws)
+            elif certified:
+                tka.topk_attn_decode_certified(q_step, kc, vc, lens_step, args.certified_eps, k, out=out,
+                                               idx=idx, tail_mass=tail, k_used=k_used, workspace=ws)
             else:
                 tka.topk_attn_decode(q_step, kc, vc, lens_step, k, out=out, idx=idx, tail_mass=tail, workspace=ws)
             for h, t in zip(hosts, outs):
@@ -350,6 +371,7 @@ def run_ours(args, world, rank, local):
             "seq_lens": "full" if int(w.seq_lens.min()) == w.L_max else [int(x) for x in w.seq_lens],
             "accumulate": "fp32", "parallelism": f"replica x{world} (independent sequences per GPU)",
             "l2": "flushed between timed steps (256 MiB write + 256 MiB read, outside the timed events)",
+            **({"certified_eps": args.certified_eps, "k_max": k} if certified else {}),
         },
         "us_per_step": ms * 1e3,
         "tokens_per_s": world * w.B * w.Q / (ms / 1e3),
@@ -360,6 +382,23 @@ def run_ours(args, world, rank, local):
         "gpu_launches": launches_per_step * K,
         "clocks": clocks.summary(),
     }
+    if certified:
+        ku = k_used.cpu().long()
+        alg = alg_bytes_token(w, k, kept=int(ku.sum()))
+        res["alg_bytes_per_step"] = alg
+        res["alg_gbs"] = alg / (ms / 1e3) / 1e9
+        res["alg_frac_of_spec_8tbs"] = res["alg_gbs"] / SPEC_HBM_GBS
+        res["alg_frac_of_measured_hbm"] = res["alg_gbs"] / peak
+        res["certified"] = {"eps": args.certified_eps, "k_max": k, "k_used_mean": float(ku.float().mean()),
+                            "k_used_min": int(ku.min()), "k_used_max": int(ku.max()),
+                            "rows_at_k_max": int((ku == k).sum()),
+                            "tail_max": float(tail.max())}
+        # no per-kernel events on this path: the whole step against the copy peak
+        res["roofline"] = {"kernel": "whole step (score + select + certify + gather)", "bound": "hbm",
+                           "achieved": res["alg_gbs"], "peak": peak,
+                           "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
+                           else "fallback 6.65 TB/s", "unit": "GB/s", "frac": res["alg_gbs"] / peak,
+                           "traffic": None, "alg_bytes_per_launch": alg}
     if stage_ms:
         res["stage_us"] = {n: stage_tot[j] / K * 1e3 for j, n in enumerate(["score", "select", "gather"])}
         score_s = stage_tot[0] / K / 1e3
@@ -374,7 +413,7 @@ def run_ours(args, world, rank, local):
         res["e2e"] = {"value": world * rows / (e2e_step / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                       "d2h_bytes_per_step": d2h, "ms_per_step": e2e_step}
     if world == 1 and not args.no_cpu_baseline:
-        v, cores, sample = time_oracle(w, k)
+        v, cores, sample = time_oracle(w, k, eps=args.certified_eps if certified else None)
         res["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
     return res
 
@@ -391,6 +430,8 @@ def run_reference(args, rank):
     def step():
         if w.variant == "block":
             oracle.block_attn(w, w.block_size, w.top_blocks)
+        elif args.certified_eps is not None:
+            oracle.certified_attn(w, args.certified_eps, k)
         else:
             oracle.topk_attn(w, k)
     for _ in range(args.warmup):

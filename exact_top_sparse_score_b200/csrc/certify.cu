@@ -16,8 +16,8 @@
 //     kept keys do not reach it, the row keeps them all (the certificate then
 //     fails and the returned tail mass exceeds eps);
 //   - otherwise a mass-weighted radix selection over the scores' order keys
-//     (11 + 11 + 10 bits) finds the key T at which the cumulative mass from the
-//     top reaches the target, the mass and count above T, and from the mass of
+//     (levels of at most 2048 bins over the range the kept keys span) finds
+//     the key T at which the cumulative mass from the top reaches the target, the mass and count above T, and from the mass of
 //     one key equal to T how many such keys (lowest positions first) are needed;
 //   - the kept positions are compacted in place, in ascending order, and the
 //     row's stats, tail mass and k are rewritten.
@@ -28,8 +28,8 @@ namespace tka {
 
 namespace {
 
-constexpr int kCertThreads = 1024;
-constexpr int kCertPer = kMaxK / kCertThreads;  // consecutive kept entries per thread
+constexpr int kCertThreads = 1024;                  // most threads per row (k_max = 8192)
+constexpr int kCertPer = kMaxK / kCertThreads;      // consecutive kept entries per thread
 constexpr int kFixedShift = 40;                 // w in (0, 1] -> integer w * 2^40; 8192 of them fit in 2^53
 
 __device__ __forceinline__ unsigned long long warp_incl_scan64(unsigned long long v) {
@@ -93,7 +93,10 @@ __device__ void warp_find_mass(const unsigned long long *hm, const uint32_t *hc,
     cnt_above = warp_sum(cnt);
 }
 
-__global__ void __launch_bounds__(kCertThreads, 1) certify_topk(CertifyParams p) {
+// blockDim.x = k_max / kCertPer rounded up to whole warps (at least two), so
+// that short rows leave room for several CTAs per SM.
+template <int kMaxThreads>
+__global__ void __launch_bounds__(kMaxThreads) certify_topk(CertifyParams p) {
     __shared__ unsigned long long hmass[2048];
     __shared__ uint32_t hcnt[2048];
     __shared__ uint32_t tmp[32];
@@ -101,6 +104,7 @@ __global__ void __launch_bounds__(kCertThreads, 1) certify_topk(CertifyParams p)
     __shared__ float redf[64];
     __shared__ unsigned long long s_mass;
     __shared__ uint32_t s_bin, s_cnt;
+    __shared__ uint32_t s_kmin[32], s_kmax[32];
 
     const int row = blockIdx.x;
     const int b = row / (p.Q * p.Hq), qpos = (row / p.Hq) % p.Q;
@@ -136,7 +140,8 @@ __global__ void __launch_bounds__(kCertThreads, 1) certify_topk(CertifyParams p)
     mine = warp_sum64(mine);
     if (lane == 0) red64[warp] = mine;
     __syncthreads();
-    const unsigned long long kept_mass = warp_sum64(red64[lane]);  // 32 warps
+    const int nw = blockDim.x >> 5;
+    const unsigned long long kept_mass = warp_sum64(lane < nw ? red64[lane] : 0ull);
     const float4 st = p.stats[row];
     const double Z = (double)st.y + (double)st.z;
     const double target_d = ceil((1.0 - (double)p.eps) * Z * (double)(1ull << kFixedShift));
@@ -146,22 +151,44 @@ __global__ void __launch_bounds__(kCertThreads, 1) certify_topk(CertifyParams p)
     uint32_t T = 0u, need_eq = 0u;
     bool cut = kept_mass >= target;  // otherwise all kk stay (not certifiable within k_max)
     if (cut) {
+        // The kept keys lie in [kmin, kmax].  Each level splits the current
+        // key range [lo, lo + 2^span) into at most 2048 bins of 2^shift keys,
+        // so the bins follow where the keys actually are (few keys share a
+        // bin: few conflicting atomics), and at most three levels reach a
+        // single key.
+        uint32_t kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
+        for (int u = 0; u < kCertPer; u++) {
+            if (kCertPer * (int)threadIdx.x + u < kk) {
+                kmin = min(kmin, key[u]);
+                kmax = max(kmax, key[u]);
+            }
+        }
+        kmin = __reduce_min_sync(0xffffffffu, kmin);
+        kmax = __reduce_max_sync(0xffffffffu, kmax);
+        if (lane == 0) {
+            s_kmin[warp] = kmin;
+            s_kmax[warp] = kmax;
+        }
+        __syncthreads();
+        kmin = __reduce_min_sync(0xffffffffu, lane < nw ? s_kmin[lane] : 0xffffffffu);
+        kmax = __reduce_max_sync(0xffffffffu, lane < nw ? s_kmax[lane] : 0u);
+        uint32_t lo = kmin;
+        int span = 32 - __clz((int)(kmax - kmin));  // bits of the range
         unsigned long long mass_above = 0ull;
-        uint32_t cnt_above = 0u, pre = 0u;
-        for (int level = 0; level < 3; level++) {
-            const int shift = level == 0 ? 21 : (level == 1 ? 10 : 0);
-            const int width = level == 2 ? 10 : 11;
-            const uint32_t nbm = (1u << width) - 1u;
-            for (int i = threadIdx.x; i < 2048; i += kCertThreads) {
+        uint32_t cnt_above = 0u;
+        for (;;) {
+            const int shift = span > 11 ? span - 11 : 0;
+            for (int i = threadIdx.x; i < 2048; i += blockDim.x) {
                 hmass[i] = 0ull;
                 hcnt[i] = 0u;
             }
             __syncthreads();
 #pragma unroll
             for (int u = 0; u < kCertPer; u++) {
-                const int j = kCertPer * threadIdx.x + u;
-                if (j < kk && (level == 0 || (key[u] >> (shift + width)) == pre)) {
-                    const uint32_t bn = (key[u] >> shift) & nbm;
+                const uint32_t rel = key[u] - lo;  // wraps for keys below lo
+                if (kCertPer * (int)threadIdx.x + u < kk && (span >= 32 || (rel >> span) == 0u)) {
+                    const uint32_t bn = rel >> shift;
                     atomicAdd(&hmass[bn], fx[u]);
                     atomicAdd(&hcnt[bn], 1u);
                 }
@@ -170,10 +197,7 @@ __global__ void __launch_bounds__(kCertThreads, 1) certify_topk(CertifyParams p)
             if (warp == 0) {
                 uint32_t bn, ca;
                 unsigned long long ma;
-                if (level == 2)
-                    warp_find_mass<1024>(hmass, hcnt, target - mass_above, bn, ma, ca);
-                else
-                    warp_find_mass<2048>(hmass, hcnt, target - mass_above, bn, ma, ca);
+                warp_find_mass<2048>(hmass, hcnt, target - mass_above, bn, ma, ca);
                 if (lane == 0) {
                     s_bin = bn;
                     s_mass = ma;
@@ -181,20 +205,22 @@ __global__ void __launch_bounds__(kCertThreads, 1) certify_topk(CertifyParams p)
                 }
             }
             __syncthreads();
-            pre = level == 0 ? s_bin : ((pre << width) | s_bin);
             mass_above += s_mass;
             cnt_above += s_cnt;
-            if (level == 2) {
-                // keys equal to T all carry the same weight
+            lo += s_bin << shift;
+            span = shift;
+            if (shift == 0) {
+                // keys equal to T = lo all carry the same weight
                 const unsigned long long m_eq = hmass[s_bin];
                 const uint32_t n_eq = hcnt[s_bin];
                 const unsigned long long w_eq = n_eq ? m_eq / n_eq : 1ull;
                 const unsigned long long rest = target - mass_above;
                 need_eq = (uint32_t)min((unsigned long long)n_eq, (rest + w_eq - 1ull) / w_eq);
+                break;
             }
             __syncthreads();  // the histograms are cleared again next level
         }
-        T = pre;
+        T = lo;
         k = (int)(cnt_above + need_eq);
     }
 
@@ -241,7 +267,7 @@ __global__ void __launch_bounds__(kCertThreads, 1) certify_topk(CertifyParams p)
         }
     }
     __syncthreads();  // all kept entries placed before the padding is written
-    for (int j = k + (int)threadIdx.x; j < kk; j += kCertThreads) idx[j] = -1;
+    for (int j = k + (int)threadIdx.x; j < kk; j += blockDim.x) idx[j] = -1;
     // both sums with one barrier pair
     zk = warp_sum(zk);
     zdrop = warp_sum(zdrop);
@@ -250,8 +276,8 @@ __global__ void __launch_bounds__(kCertThreads, 1) certify_topk(CertifyParams p)
         redf[2 * warp + 1] = zdrop;
     }
     __syncthreads();
-    zk = warp_sum(redf[2 * lane]);
-    zdrop = warp_sum(redf[2 * lane + 1]);
+    zk = warp_sum(lane < nw ? redf[2 * lane] : 0.f);
+    zdrop = warp_sum(lane < nw ? redf[2 * lane + 1] : 0.f);
     if (threadIdx.x == 0) {
         const float zt = st.z + zdrop;
         p.stats[row] = make_float4(st.x, zk, zt, 0.f);
@@ -264,7 +290,11 @@ __global__ void __launch_bounds__(kCertThreads, 1) certify_topk(CertifyParams p)
 
 cudaError_t launch_certify(const CertifyParams &p, cudaStream_t stream) {
     if (p.k_max > kMaxK) return cudaErrorInvalidValue;
-    certify_topk<<<p.B * p.Q * p.Hq, kCertThreads, 0, stream>>>(p);
+    const int threads = max(64, min(kCertThreads, (p.k_max + kCertPer * 32 - 1) / (kCertPer * 32) * 32));
+    if (threads <= 256)
+        certify_topk<256><<<p.B * p.Q * p.Hq, threads, 0, stream>>>(p);
+    else
+        certify_topk<kCertThreads><<<p.B * p.Q * p.Hq, threads, 0, stream>>>(p);
     return cudaGetLastError();
 }
 
