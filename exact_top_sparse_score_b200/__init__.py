@@ -10,6 +10,7 @@ device.
 from ._binding import (  # noqa: F401
     TKA_BF16,
     TKA_F32,
+    DEV_BAD_PAGE,
     DEV_BAD_SEQ_LEN,
     DEV_INTERNAL,
     DEV_TIMEOUT,
@@ -19,6 +20,7 @@ from ._binding import (  # noqa: F401
     load_library,
     topk_attn_decode,
     topk_attn_decode_certified,
+    topk_attn_decode_paged,
     topk_attn_decode_static,
     topk_attn_static_workspace_capacity,
     topk_attn_device_status,

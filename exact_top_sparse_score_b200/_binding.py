@@ -11,7 +11,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_NAME = "libtopk_attn.so"
 
 TKA_F32, TKA_BF16 = 0, 1
-DEV_BAD_SEQ_LEN, DEV_INTERNAL, DEV_TIMEOUT = 0x1, 0x2, 0x4
+DEV_BAD_SEQ_LEN, DEV_INTERNAL, DEV_TIMEOUT, DEV_BAD_PAGE = 0x1, 0x2, 0x4, 0x8
 _STATUS = {0: "TKA_OK", 1: "TKA_ERR_INVALID_ARG", 2: "TKA_ERR_UNSUPPORTED", 3: "TKA_ERR_WORKSPACE",
            4: "TKA_ERR_CUDA"}
 
@@ -56,6 +56,9 @@ def load_library() -> ctypes.CDLL:
         lib.topk_attn_decode_certified.argtypes = [_shape_p, _vp, _vp, _vp, _vp, ctypes.c_float, _i32, _vp, _vp,
                                                    _vp, _vp, _vp, _sz, _vp]
         lib.topk_attn_decode_certified.restype = ctypes.c_int
+        lib.topk_attn_decode_paged.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _i32, _vp,
+                                               _vp, _vp, _vp, _sz, _vp]
+        lib.topk_attn_decode_paged.restype = ctypes.c_int
         lib.topk_attn_static_workspace_capacity.argtypes = []
         lib.topk_attn_static_workspace_capacity.restype = _sz
         lib.topk_attn_decode_static.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp]
@@ -201,6 +204,55 @@ def topk_attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tens
         rc = lib.topk_attn_decode_staged(*args, evs)
     if rc:
         raise TopkAttnError("topk_attn_decode", rc)
+    return out, idx, tail_mass
+
+
+def topk_attn_decode_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,
+                           block_table: torch.Tensor, seq_lens: torch.Tensor, k: int, *, scale: float = 0.0,
+                           out: Optional[torch.Tensor] = None, idx: Optional[torch.Tensor] = None,
+                           tail_mass: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                           stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Exact Top-k decode attention over a paged cache: k_pages / v_pages
+    [num_pages, Hkv, page_size, d], block_table int32 [B, max_pages] (logical
+    page j of sequence b -> physical page).  Returns (out, idx, tail) as
+    topk_attn_decode does on the equivalent contiguous cache."""
+    lib = load_library()
+    if q.dim() != 4 or k_pages.dim() != 4 or block_table.dim() != 2:
+        raise ValueError("q [B,Q,Hq,d], pages [num_pages,Hkv,page_size,d], block_table [B,max_pages]")
+    B, Q, Hq, d = q.shape
+    num_pages, Hkv, page_size, dk = k_pages.shape
+    max_pages = block_table.shape[1]
+    if dk != d or block_table.shape[0] != B:
+        raise ValueError("q, pages and block_table shapes disagree")
+    if q.dtype != k_pages.dtype or v_pages.dtype != k_pages.dtype or v_pages.shape != k_pages.shape:
+        raise TypeError("q, k_pages and v_pages must share dtype and shape")
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32 or tuple(seq_lens.shape) != (B,):
+        raise TypeError("block_table and seq_lens must be int32")
+    shape = tka_shape(B, Q, Hq, Hkv, d, max_pages * page_size, _dtype_code(k_pages), float(scale))
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, Q, Hq, d), dtype=torch.float32, device=dev)
+    if idx is None:
+        idx = torch.empty((B, Q, Hq, k), dtype=torch.int32, device=dev)
+    if tail_mass is None:
+        tail_mass = torch.empty((B, Q, Hq), dtype=torch.float32, device=dev)
+    _check_out("out", out, torch.float32, (B, Q, Hq, d))
+    _check_out("idx", idx, torch.int32, (B, Q, Hq, k))
+    _check_out("tail_mass", tail_mass, torch.float32, (B, Q, Hq))
+    if workspace is not None and workspace.dtype != torch.uint8:
+        raise TypeError("workspace must be a uint8 tensor")
+    _check_cuda(q=q, k_pages=k_pages, v_pages=v_pages, block_table=block_table, seq_lens=seq_lens, out=out,
+                idx=idx, tail_mass=tail_mass, workspace=workspace)
+    nbytes = topk_attn_workspace_size(shape, k)
+    if nbytes == 0:
+        raise TopkAttnError("topk_attn_workspace_size", 2)
+    sh = _stream(stream)
+    ws = _workspace(nbytes, dev, workspace, sh)
+    rc = lib.topk_attn_decode_paged(ctypes.byref(shape), q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
+                                    block_table.data_ptr(), max_pages, num_pages, page_size, seq_lens.data_ptr(), k,
+                                    out.data_ptr(), idx.data_ptr(), tail_mass.data_ptr(), ws.data_ptr(), nbytes, sh)
+    if rc:
+        raise TopkAttnError("topk_attn_decode_paged", rc)
     return out, idx, tail_mass
 
 

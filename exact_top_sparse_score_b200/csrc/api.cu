@@ -176,7 +176,7 @@ struct CertArgs {
 tka_status decode_impl(const tka_shape *shape, const void *q, const void *k_cache, const void *v_cache,
                        const int32_t *seq_lens, int32_t k, float *out, int32_t *idx, float *tail_mass,
                        void *workspace, size_t workspace_bytes, tka_stream_t stream, const tka_event_t events[4],
-                       const CertArgs *cert) {
+                       const CertArgs *cert, const PageTable *pages = nullptr) {
     tka_status st = check_shape(shape);
     if (st != TKA_OK) return st;
     if (k < 1) return TKA_ERR_INVALID_ARG;
@@ -198,7 +198,7 @@ tka_status decode_impl(const tka_shape *shape, const void *q, const void *k_cach
     const int NQ = shape->Q * G;
     // the tensor map addresses cache rows with int32 coordinates
     const bool tc = score_tc_supported(shape->dtype, NQ) &&
-                    (long long)shape->B * shape->Hkv * shape->L_max < (1LL << 31);
+                    (pages || (long long)shape->B * shape->Hkv * shape->L_max < (1LL << 31));
     if (tc) {
         ScoreTcParams tp;
         tp.status = dev->status;
@@ -207,6 +207,7 @@ tka_status decode_impl(const tka_shape *shape, const void *q, const void *k_cach
         tp.B = shape->B; tp.Q = shape->Q; tp.Hq = shape->Hq; tp.Hkv = shape->Hkv; tp.G = G;
         tp.L_max = shape->L_max; tp.ld = L.ld; tp.NQ = NQ;
         tp.scale = resolve_scale(shape);
+        if (pages) tp.pages = *pages;
         RecordCtx rc{events, 0, s};
         ScoreTcHook hook;
         hook.fn = record_hook;
@@ -223,6 +224,7 @@ tka_status decode_impl(const tka_shape *shape, const void *q, const void *k_cach
         sp.B = shape->B; sp.Q = shape->Q; sp.Hq = shape->Hq; sp.Hkv = shape->Hkv; sp.G = G;
         sp.L_max = shape->L_max; sp.ld = L.ld; sp.dtype = shape->dtype;
         sp.scale = resolve_scale(shape);
+        if (pages) sp.pages = *pages;
         if (launch_score(sp, dev->num_sms, s) != cudaSuccess) return TKA_ERR_CUDA;
     }
     if (record(events, 1, s) != cudaSuccess) return TKA_ERR_CUDA;
@@ -268,6 +270,7 @@ tka_status decode_impl(const tka_shape *shape, const void *q, const void *k_cach
     gp.counters = se.counters;
     gp.out = out;
     gp.kcount = cert ? cert->k_used : nullptr;
+    if (pages) gp.pages = *pages;
     // one wave of eight CTAs per SM (splits = floor(8 x SMs / rows), at least 1),
     // never fewer than kMinKeysPerSplit keys per CTA
     int splits = (dev->num_sms * 8) / rows;
@@ -290,6 +293,26 @@ tka_status topk_attn_decode_staged(const tka_shape *shape, const void *q, const 
                                    tka_stream_t stream, const tka_event_t events[4]) {
     return decode_impl(shape, q, k_cache, v_cache, seq_lens, k, out, idx, tail_mass, workspace, workspace_bytes,
                        stream, events, nullptr);
+}
+
+tka_status topk_attn_decode_paged(const tka_shape *shape, const void *q, const void *k_pages, const void *v_pages,
+                                  const int32_t *block_table, int32_t max_pages, int32_t num_pages,
+                                  int32_t page_size, const int32_t *seq_lens, int32_t k, float *out, int32_t *idx,
+                                  float *tail_mass, void *workspace, size_t workspace_bytes, tka_stream_t stream) {
+    if (!block_table || !aligned(block_table, 4)) return TKA_ERR_INVALID_ARG;
+    if (page_size < 16 || (page_size & (page_size - 1)) || max_pages < 1 || num_pages < 1)
+        return TKA_ERR_INVALID_ARG;
+    if (!shape) return TKA_ERR_INVALID_ARG;
+    if ((long long)max_pages * page_size < shape->L_max) return TKA_ERR_INVALID_ARG;
+    // rows of the paged cache are addressed with 32-bit row numbers
+    if ((long long)num_pages * shape->Hkv * page_size >= (1ll << 31)) return TKA_ERR_UNSUPPORTED;
+    PageTable pt;
+    pt.table = block_table;
+    pt.max_pages = max_pages;
+    pt.num_pages = num_pages;
+    pt.page_shift = __builtin_ctz((unsigned)page_size);
+    return decode_impl(shape, q, k_pages, v_pages, seq_lens, k, out, idx, tail_mass, workspace, workspace_bytes,
+                       stream, nullptr, nullptr, &pt);
 }
 
 tka_status topk_attn_decode_certified(const tka_shape *shape, const void *q, const void *k_cache,

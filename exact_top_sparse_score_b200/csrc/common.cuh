@@ -16,6 +16,25 @@ constexpr int kHeadDim = 128;
 // launch receives.
 __device__ __forceinline__ void raise_status(unsigned int *status, unsigned int bits) { atomicOr(status, bits); }
 
+// A paged cache: pages of 2^page_shift positions, [num_pages, Hkv, page, 128];
+// logical page j of sequence b is physical page table[b * max_pages + j].
+// A null table means the contiguous layout [B, Hkv, L_max, 128].
+struct PageTable {
+    const int32_t *table = nullptr;
+    int max_pages = 0, num_pages = 0, page_shift = 0;
+};
+
+// Row (of 128 elements) holding position pos of (b, kvh) in a paged cache.
+// A table entry out of range raises TKA_DEV_BAD_PAGE and reads page 0.
+__device__ __forceinline__ long long paged_row(const PageTable &pt, unsigned *status, int Hkv, int b, int kvh, int pos) {
+    int phys = __ldg(pt.table + (size_t)b * pt.max_pages + (pos >> pt.page_shift));
+    if ((unsigned)phys >= (unsigned)pt.num_pages) {
+        raise_status(status, TKA_DEV_BAD_PAGE);
+        phys = 0;
+    }
+    return ((long long)phys * Hkv + kvh) * (1ll << pt.page_shift) + (pos & ((1 << pt.page_shift) - 1));
+}
+
 // Rows are (b, qpos, h) in that order: row = (b * Q + qpos) * Hq + h.
 struct RowGeom {
     int B, Q, Hq, Hkv, G, L_max;

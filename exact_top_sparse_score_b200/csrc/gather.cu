@@ -48,7 +48,7 @@ __device__ __forceinline__ void fma_row(float (&acc)[16 / sizeof(T)], float wt, 
     }
 }
 
-template <typename T>
+template <typename T, bool kPaged>
 __global__ void __launch_bounds__(kGatherThreads, 8) gather_pv(GatherParams p) {
     constexpr int kPer = 16 / sizeof(T);              // elements per lane
     constexpr int kLanesPerRow = kHeadDim / kPer;     // 16 (bf16) or 32 (fp32)
@@ -72,8 +72,10 @@ __global__ void __launch_bounds__(kGatherThreads, 8) gather_pv(GatherParams p) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int slot = warp * kRowsPerWarp + lane / kLanesPerRow;
     const int c = lane % kLanesPerRow;  // this lane's 16-byte piece of a V row
-    const T *vbase = reinterpret_cast<const T *>(p.v) + ((size_t)b * p.Hkv + h / p.G) * p.L_max * kHeadDim +
-                     c * kPer;
+    // rows are counted from the (b, kv-head) block of a contiguous cache, or
+    // from the start of a paged one (staged below as physical row numbers)
+    const T *vbase = reinterpret_cast<const T *>(p.v) +
+                     (kPaged ? 0 : ((size_t)b * p.Hkv + h / p.G) * p.L_max * kHeadDim) + c * kPer;
     const int32_t *gidx = p.idx + (size_t)row * p.k;
     const float *gw = p.w + (size_t)row * p.k;
 
@@ -93,6 +95,7 @@ __global__ void __launch_bounds__(kGatherThreads, 8) gather_pv(GatherParams p) {
                 pos = 0;
                 wt = 0.f;
             }
+            if constexpr (kPaged) pos = (int32_t)paged_row(p.pages, p.status, p.Hkv, b, h / p.G, pos);
             s_idx[j] = pos;
             s_w[j] = wt;
         }
@@ -148,10 +151,18 @@ __global__ void __launch_bounds__(kGatherThreads, 8) gather_pv(GatherParams p) {
 cudaError_t launch_gather(const GatherParams &p, cudaStream_t stream) {
     const int rows = p.B * p.Q * p.Hq;
     const dim3 grid(p.splits, rows);
-    if (p.dtype == TKA_BF16)
-        gather_pv<__nv_bfloat16><<<grid, kGatherThreads, 0, stream>>>(p);
-    else
-        gather_pv<float><<<grid, kGatherThreads, 0, stream>>>(p);
+    const bool paged = p.pages.table != nullptr;
+    if (p.dtype == TKA_BF16) {
+        if (paged)
+            gather_pv<__nv_bfloat16, true><<<grid, kGatherThreads, 0, stream>>>(p);
+        else
+            gather_pv<__nv_bfloat16, false><<<grid, kGatherThreads, 0, stream>>>(p);
+    } else {
+        if (paged)
+            gather_pv<float, true><<<grid, kGatherThreads, 0, stream>>>(p);
+        else
+            gather_pv<float, false><<<grid, kGatherThreads, 0, stream>>>(p);
+    }
     return cudaGetLastError();
 }
 

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "common.cuh"
+
 namespace tka {
 
 constexpr int kMaxK = 8192;  // largest k (and k_max) the select and certify steps take
@@ -12,11 +14,12 @@ constexpr int kMaxK = 8192;  // largest k (and k_max) the select and certify ste
 struct ScoreParams {
     unsigned *status;         // device status word (TKA_DEV_* bits)
     const void *q;            // [B, Q, Hq, 128]
-    const void *k;            // [B, Hkv, L_max, 128]
+    const void *k;            // [B, Hkv, L_max, 128], or the paged cache
     const int32_t *seq_lens;  // [B]
     float *scores;            // [B*Q*Hq, ld]
     int B, Q, Hq, Hkv, G, L_max, ld, dtype;
     float scale;
+    PageTable pages;
 };
 
 struct ScoreTcParams {
@@ -25,6 +28,7 @@ struct ScoreTcParams {
     float *scores;            // [B*Q*Hq, ld]
     int B, Q, Hq, Hkv, G, L_max, ld, NQ;
     float scale;
+    PageTable pages;          // paged cache: the K tensor map covers [num_pages*Hkv*page, 128]
 };
 
 struct SelectParams {
@@ -52,6 +56,7 @@ struct GatherParams {
     float *out;               // [rows, 128]
     int splits, per_split;
     const int32_t *kcount;    // [rows] kept positions per row, or null: min(k, visible keys)
+    PageTable pages;          // v is the paged cache when pages.table is set
 };
 
 struct CertifyParams {

@@ -170,11 +170,14 @@ __global__ void __launch_bounds__(128) score_generic(ScoreParams p) {
         for (int kb = chunk * kChunkKeys + warp * 8; kb < (chunk + 1) * kChunkKeys; kb += 32) {
             const int key = kb + g;
             const bool ok = key < seq_len;
+            const T *krow = p.pages.table == nullptr || !ok
+                                ? kbase + (size_t)key * kHeadDim
+                                : reinterpret_cast<const T *>(p.k) +
+                                      (size_t)paged_row(p.pages, p.status, p.Hkv, b, kvh, key) * kHeadDim;
             float kv[kPieces][kPer];
 #pragma unroll
             for (int j = 0; j < kPieces; j++) {
-                const uint4 v = ok ? *reinterpret_cast<const uint4 *>(kbase + (size_t)key * kHeadDim +
-                                                                     kPer * (t + 4 * j))
+                const uint4 v = ok ? *reinterpret_cast<const uint4 *>(krow + kPer * (t + 4 * j))
                                    : make_uint4(0u, 0u, 0u, 0u);
                 if constexpr (sizeof(T) == 4) {
                     kv[j][0] = __uint_as_float(v.x);
@@ -216,7 +219,7 @@ cudaError_t launch_score(const ScoreParams &p, int num_sms, cudaStream_t stream)
     if (gx > chunks) gx = chunks;
     if (gx < 1) gx = 1;
     const dim3 grid(gx, units);
-    if (p.dtype == TKA_BF16 && NQ <= 64) {
+    if (p.dtype == TKA_BF16 && NQ <= 64 && p.pages.table == nullptr) {  // paged caches take score_generic
         if (NQ <= 8)
             score_bf16_mma<1><<<grid, 128, 0, stream>>>(p);
         else if (NQ <= 16)

@@ -161,9 +161,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (i >= S) ok = mbar_wait(&empty[s], ((i / S) - 1) & 1, abort);
                 if (!ok) break;
                 mbar_arrive_expect_tx(&full[s], kTileBytes);
-                const int row0 = w.bh * p.L_max + w.t * kTileKeys;
-                tma_load_2d_hint(stages + s * kTileBytes, &kmap, &full[s], 0, row0, evict_first);
-                tma_load_2d_hint(stages + s * kTileBytes + kKBlockBytes, &kmap, &full[s], 64, row0, evict_first);
+                if (p.pages.table == nullptr) {
+                    const int row0 = w.bh * p.L_max + w.t * kTileKeys;
+                    tma_load_2d_hint(stages + s * kTileBytes, &kmap, &full[s], 0, row0, evict_first);
+                    tma_load_2d_hint(stages + s * kTileBytes + kKBlockBytes, &kmap, &full[s], 64, row0, evict_first);
+                } else {
+                    // paged cache: the tile is box_rows-row pieces of one or
+                    // more pages; a piece past the sequence end rereads its
+                    // last page (those keys are never stored)
+                    const int box_rows = min(1 << p.pages.page_shift, kTileKeys);
+                    const int last = max(p.seq_lens[b] - 1, 0);
+                    for (int piece = 0; piece < kTileKeys / box_rows; piece++) {
+                        int pos = w.t * kTileKeys + piece * box_rows;
+                        if ((pos >> p.pages.page_shift) > (last >> p.pages.page_shift))
+                            pos = ((last >> p.pages.page_shift) << p.pages.page_shift) | (pos & ((1 << p.pages.page_shift) - 1));
+                        const int row0 = (int)paged_row(p.pages, p.status, p.Hkv, b, kvh, pos);
+                        uint8_t *dst = stages + s * kTileBytes + piece * box_rows * 128;
+                        tma_load_2d_hint(dst, &kmap, &full[s], 0, row0, evict_first);
+                        tma_load_2d_hint(dst + kKBlockBytes, &kmap, &full[s], 64, row0, evict_first);
+                    }
+                }
                 misc[2] = i + 1;
                 if (w.seg_last(i)) seg++;
                 w.next(p);
@@ -318,10 +335,14 @@ cudaError_t launch_score_tc(const ScoreTcParams &p, const void *q, const void *k
     if (!enc) return cudaErrorNotSupported;
     CUtensorMap km, qm;
     {
-        // K cache as rows of 128 bf16: [B*Hkv*L_max, 128]; boxes of 128 rows x 64 dims
-        const cuuint64_t dims[2] = {128, (cuuint64_t)p.B * p.Hkv * p.L_max};
+        // K cache as rows of 128 bf16: [B*Hkv*L_max, 128] (paged: [num_pages*Hkv*page, 128]);
+        // boxes of 128 rows (paged: min(page, 128) rows) x 64 dims
+        const bool paged = p.pages.table != nullptr;
+        const cuuint64_t nrows = paged ? (cuuint64_t)p.pages.num_pages * p.Hkv << p.pages.page_shift
+                                       : (cuuint64_t)p.B * p.Hkv * p.L_max;
+        const cuuint64_t dims[2] = {128, nrows};
         const cuuint64_t strides[1] = {256};
-        const cuuint32_t box[2] = {64, kTileKeys};
+        const cuuint32_t box[2] = {64, paged ? (cuuint32_t)min(1 << p.pages.page_shift, kTileKeys) : (cuuint32_t)kTileKeys};
         const cuuint32_t es[2] = {1, 1};
         if (enc(&km, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(k_cache), dims, strides, box, es,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,

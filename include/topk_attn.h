@@ -70,6 +70,7 @@ typedef enum { TKA_F32 = 0, TKA_BF16 = 1 } tka_dtype;
 #define TKA_DEV_BAD_SEQ_LEN 0x1u /* a seq_lens value was out of range; that sequence was skipped */
 #define TKA_DEV_INTERNAL 0x2u    /* an internal consistency check failed (a library bug) */
 #define TKA_DEV_TIMEOUT 0x4u     /* a bounded wait inside a kernel gave up; results are incomplete */
+#define TKA_DEV_BAD_PAGE 0x8u    /* a block-table entry names no page of the paged cache */
 
 /* cudaStream_t without pulling in the CUDA headers. */
 typedef struct CUstream_st *tka_stream_t;
@@ -107,6 +108,29 @@ tka_status topk_attn_decode_staged(const tka_shape *shape, const void *q, const 
                                    const void *v_cache, const int32_t *seq_lens, int32_t k, float *out,
                                    int32_t *idx, float *tail_mass, void *workspace, size_t workspace_bytes,
                                    tka_stream_t stream, const tka_event_t events[4]);
+
+/* topk_attn_decode over a paged KV cache ("Sparse Attention in LLM Inference:
+ * Practical Trade-Offs", section "Changes in Caching Strategy": the selected
+ * entries are read by index from the cache wherever they live).  The cache is
+ * a pool of pages of page_size positions:
+ *   k_pages, v_pages  [num_pages, Hkv, page_size, d] (cache dtype); each page
+ *                     holds page_size consecutive positions of every kv-head.
+ *   block_table       int32 [B, max_pages] device buffer: logical page j of
+ *                     sequence b (positions j*page_size .. (j+1)*page_size - 1)
+ *                     is physical page block_table[b * max_pages + j]; only
+ *                     the entries below ceil(seq_lens[b] / page_size) are read.
+ *   page_size         a power of two >= 16.
+ *   shape->L_max      the logical capacity, at most max_pages * page_size.
+ * Everything else (q, outputs, workspace = topk_attn_workspace_size(shape, k),
+ * results) is as topk_attn_decode, which gives the same out, idx and tail on
+ * the equivalent contiguous cache.  A table entry outside [0, num_pages)
+ * raises TKA_DEV_BAD_PAGE (page 0 is read instead).  num_pages * Hkv *
+ * page_size must stay below 2^31 (TKA_ERR_UNSUPPORTED otherwise). */
+tka_status topk_attn_decode_paged(const tka_shape *shape, const void *q, const void *k_pages,
+                                  const void *v_pages, const int32_t *block_table, int32_t max_pages,
+                                  int32_t num_pages, int32_t page_size, const int32_t *seq_lens, int32_t k,
+                                  float *out, int32_t *idx, float *tail_mass, void *workspace,
+                                  size_t workspace_bytes, tka_stream_t stream);
 
 /* Certified adaptive Top-k ("A Mathematical Theory of Top-k Sparse Attention
  * via Total Variation Distance", abstract: the Top-k truncation error in total
