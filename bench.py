@@ -55,6 +55,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch size (smaller cases for profiling)")
+    ap.add_argument("--paged", type=int, default=None, metavar="PAGE_SIZE",
+                    help="lay the cache out as shuffled pages of PAGE_SIZE positions (block tables)")
     ap.add_argument("--certified-eps", type=float, default=None,
                     help="certified adaptive Top-k: per row the smallest k (at most the workload's k) "
                          "whose discarded tail mass is <= EPS")
@@ -221,6 +223,25 @@ def make_inputs(cfg, rank, batch=None):
     return workloads.config_workload(cfg, seed=1000 + cfg + 7919 * rank, **over)
 
 
+def page_cache(kc, vc, page_size, rank):
+    """The contiguous caches [B, Hkv, L, d] as shuffled pages [num_pages, Hkv, page_size, d] and
+    the block table [B, L / page_size] that maps them back."""
+    B, Hkv, L, d = kc.shape
+    if L % page_size:
+        raise SystemExit("--paged: the page size must divide L_max")
+    npg = L // page_size
+    g = torch.Generator(device=kc.device).manual_seed(4242 + rank)
+    perm = torch.randperm(B * npg, generator=g, device=kc.device)
+    pages = []
+    for c in (kc, vc):
+        p = c.reshape(B, Hkv, npg, page_size, d).permute(0, 2, 1, 3, 4).reshape(B * npg, Hkv, page_size, d)
+        out = torch.empty_like(p)
+        out[perm] = p
+        pages.append(out)
+    table = perm.reshape(B, npg).to(torch.int32).contiguous()
+    return pages[0], pages[1], table
+
+
 def run_ours(args, world, rank, local):
     import exact_top_sparse_score_b200 as tka
     from exact_top_sparse_score_b200._binding import block_attn_workspace_size, make_shape
@@ -232,6 +253,7 @@ def run_ours(args, world, rank, local):
     rows = w.B * w.Q * w.Hq
     block = w.variant == "block"
     certified = args.certified_eps is not None and not block
+    paged = args.paged is not None and not block and not certified
     k = w.k
     if block:
         bk = tka.topk_block_pool_keys(kc, lens, w.block_size)
@@ -265,6 +287,17 @@ def run_ours(args, world, rank, local):
                     events[0].record()
                 tka.topk_attn_decode_certified(qq, kc, vc, lens, args.certified_eps, k, out=out, idx=idx,
                                                tail_mass=tail, k_used=k_used, workspace=ws)
+                if events:
+                    events[3].record()
+        elif paged:
+            kp, vp, table = page_cache(kc, vc, args.paged, rank)
+            launches_per_step = 3
+
+            def step(events=None, qq=q):
+                if events:
+                    events[0].record()
+                tka.topk_attn_decode_paged(qq, kp, vp, table, lens, k, out=out, idx=idx, tail_mass=tail,
+                                           workspace=ws)
                 if events:
                     events[3].record()
         else:
@@ -303,7 +336,7 @@ def run_ours(args, world, rank, local):
     if world > 1:
         torch.distributed.barrier()
     step_ms = [e[0].elapsed_time(e[3]) for e in evs]
-    stage_ms = None if block or certified else [[e[j].elapsed_time(e[j + 1]) for e in evs] for j in range(3)]
+    stage_ms = None if block or certified or paged else [[e[j].elapsed_time(e[j + 1]) for e in evs] for j in range(3)]
     total_ms = sum(step_ms)
 
     e2e_ms = None
@@ -331,6 +364,9 @@ def run_ours(args, world, rank, local):
             elif certified:
                 tka.topk_attn_decode_certified(q_step, kc, vc, lens_step, args.certified_eps, k, out=out,
                                                idx=idx, tail_mass=tail, k_used=k_used, workspace=ws)
+            elif paged:
+                tka.topk_attn_decode_paged(q_step, kp, vp, table, lens_step, k, out=out, idx=idx,
+                                           tail_mass=tail, workspace=ws)
             else:
                 tka.topk_attn_decode(q_step, kc, vc, lens_step, k, out=out, idx=idx, tail_mass=tail, workspace=ws)
             for h, t in zip(hosts, outs):
@@ -372,6 +408,7 @@ def run_ours(args, world, rank, local):
             "accumulate": "fp32", "parallelism": f"replica x{world} (independent sequences per GPU)",
             "l2": "flushed between timed steps (256 MiB write + 256 MiB read, outside the timed events)",
             **({"certified_eps": args.certified_eps, "k_max": k} if certified else {}),
+            **({"page_size": args.paged, "pages": "shuffled pool, block tables"} if paged else {}),
         },
         "us_per_step": ms * 1e3,
         "tokens_per_s": world * w.B * w.Q / (ms / 1e3),
@@ -382,6 +419,13 @@ def run_ours(args, world, rank, local):
         "gpu_launches": launches_per_step * K,
         "clocks": clocks.summary(),
     }
+    if paged:
+        # no per-kernel events on this path: the whole step against the copy peak
+        res["roofline"] = {"kernel": "whole step (paged: score + select + gather)", "bound": "hbm",
+                           "achieved": res["alg_gbs"], "peak": peak,
+                           "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
+                           else "fallback 6.65 TB/s", "unit": "GB/s", "frac": res["alg_gbs"] / peak,
+                           "traffic": None, "alg_bytes_per_launch": alg}
     if certified:
         ku = k_used.cpu().long()
         alg = alg_bytes_token(w, k, kept=int(ku.sum()))
