@@ -54,6 +54,8 @@ def _load():
         lib.oracle_topk_attn.restype = _i
         lib.oracle_certified_attn.argtypes = [_i] * 7 + [_d, _vp, _vp, _vp, _ip, _d, _i, _dp, _ip, _dp, _ip, _i]
         lib.oracle_certified_attn.restype = _i
+        lib.oracle_hisa_attn.argtypes = [_i] * 6 + [_d, _vp, _vp, _vp, _ip, _i, _i, _i, _dp, _ip, _ip, _dp, _i]
+        lib.oracle_hisa_attn.restype = _i
         lib.oracle_block_pool.argtypes = [_i] * 5 + [_vp, _ip, _i, _dp]
         lib.oracle_block_pool.restype = _i
         lib.oracle_block_attn.argtypes = [_i] * 6 + [_d, _vp, _vp, _vp, _ip, _i, _i, _dp, _ip, _dp, _dp, _i]
@@ -166,3 +168,25 @@ def block_attn(w, block_size: int, top_blocks: int, scale: float = 0.0, nthreads
     if rc:
         raise ValueError(f"oracle_block_attn failed with code {rc}")
     return dict(out=out, block_idx=bidx, tail=tail, kth=kth)
+
+
+def hisa_attn(w, block_size: int, top_blocks: int, k: int, scale: float = 0.0, nthreads: int = 0) -> dict:
+    """Hierarchical block -> token Top-k decode attention (one query per sequence).
+
+    Returns out [B,1,Hq,d] f64, block_idx [B,1,Hq,top_blocks] and idx [B,1,Hq,k]
+    (ascending, -1 padded) and tail [B,1,Hq] (discarded mass among the candidates).
+    """
+    if w.Q != 1:
+        raise ValueError("one query position per sequence")
+    lib = _load()
+    q, kc, vc, lens = _arr(w, w.q), _arr(w, w.k_cache), _arr(w, w.v_cache), _lens(w)
+    out = np.zeros((w.B, 1, w.Hq, w.d), np.float64)
+    bidx = np.zeros((w.B, 1, w.Hq, top_blocks), np.int32)
+    idx = np.zeros((w.B, 1, w.Hq, k), np.int32)
+    tail = np.zeros((w.B, 1, w.Hq), np.float64)
+    rc = lib.oracle_hisa_attn(w.B, w.Hq, w.Hkv, w.d, w.L_max, _code(w.dtype), scale,
+                              q.ctypes.data, kc.ctypes.data, vc.ctypes.data, lens,
+                              block_size, top_blocks, k, out, bidx, idx, tail, nthreads)
+    if rc:
+        raise ValueError(f"oracle_hisa_attn failed with code {rc}")
+    return dict(out=out, block_idx=bidx, idx=idx, tail=tail)

@@ -386,3 +386,97 @@ int oracle_block_attn(int B, int Hq, int Hkv, int d, int L_max, int dtype, doubl
     free(bk);
     return status;
 }
+
+/*
+ * Hierarchical block -> token selection ("Sparse Attention Landscape",
+ * section "Hierarchical Sparse Attention"), one query per sequence:
+ *   1. block scores r_j = scale * <q, mean key of block j> for every block j
+ *      of the sequence (the partial last block averaged over its tokens);
+ *   2. the top_blocks best blocks (r descending, block ascending) are kept;
+ *   3. token scores s_i = scale * <q, K_i> only for the tokens of the kept
+ *      blocks below seq_len (the candidates);
+ *   4. the top k candidates (s descending, position ascending) are kept and
+ *      attention runs over them: softmax over the kept tokens, P.V;
+ *   5. tail = the candidates' discarded softmax mass, relative to all
+ *      candidates (the method scores nothing else).
+ * block_idx [B, Hq, top_blocks] and idx [B, Hq, k] ascending, -1 padded.
+ */
+int oracle_hisa_attn(int B, int Hq, int Hkv, int d, int L_max, int dtype, double scale,
+                     const void *q, const void *k_cache, const void *v_cache, const int32_t *seq_lens,
+                     int block_size, int top_blocks, int k, double *out, int32_t *block_idx, int32_t *idx,
+                     double *tail, int nthreads) {
+    if (!check_shape(B, 1, Hq, Hkv, d, L_max, dtype) || block_size < 1 || top_blocks < 1 || k < 1)
+        return OR_BAD_ARG;
+    for (int b = 0; b < B; b++)
+        if (seq_lens[b] < 1 || seq_lens[b] > L_max) return OR_BAD_ARG;
+    const int G = Hq / Hkv;
+    const int nblk_max = (L_max + block_size - 1) / block_size;
+    double *bk = (double *)malloc(sizeof(double) * (size_t)B * Hkv * nblk_max * d);
+    if (!bk) return OR_NO_MEMORY;
+    int status = oracle_block_pool(B, Hkv, d, L_max, dtype, k_cache, seq_lens, block_size, bk);
+    if (status != OR_OK) { free(bk); return status; }
+    const double sc = resolve_scale(scale, d);
+    const long rows = (long)B * Hq;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+#pragma omp parallel
+    {
+        scored_pos *sb = (scored_pos *)malloc(sizeof(scored_pos) * (size_t)nblk_max);
+        scored_pos *sp = (scored_pos *)malloc(sizeof(scored_pos) * (size_t)L_max);
+        double *s = (double *)malloc(sizeof(double) * (size_t)L_max);
+        int32_t *kept = (int32_t *)malloc(sizeof(int32_t) * (size_t)nblk_max);
+        int32_t *sel = (int32_t *)malloc(sizeof(int32_t) * (size_t)L_max);
+        if (!sb || !sp || !s || !kept || !sel) {
+#pragma omp atomic write
+            status = OR_NO_MEMORY;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (long r = 0; r < rows; r++) {
+            if (!sb || !sp || !s || !kept || !sel) continue;
+            int h = (int)(r % Hq), b = (int)(r / Hq), kvh = h / G;
+            int Lb = seq_lens[b];
+            int nblk = (Lb + block_size - 1) / block_size;
+            size_t qoff = (size_t)r * d;
+            const double *bkh = bk + ((size_t)b * Hkv + kvh) * (size_t)nblk_max * d;
+            /* 1.-2. block scores of every block, the best top_blocks kept */
+            for (int j = 0; j < nblk; j++) {
+                double acc = 0.0;
+                for (int c = 0; c < d; c++) acc += load_elem(q, dtype, qoff + c) * bkh[(size_t)j * d + c];
+                sb[j].s = sc * acc;
+                sb[j].i = j;
+            }
+            qsort(sb, (size_t)nblk, sizeof(scored_pos), cmp_score_desc);
+            int nk = top_blocks < nblk ? top_blocks : nblk;
+            for (int j = 0; j < nk; j++) kept[j] = sb[j].i;
+            qsort(kept, (size_t)nk, sizeof(int32_t), cmp_int_asc);
+            int32_t *bi = block_idx + (size_t)r * top_blocks;
+            for (int j = 0; j < top_blocks; j++) bi[j] = j < nk ? kept[j] : -1;
+            /* 3. token scores of the candidates, in position order */
+            oracle_row_scores(B, 1, Hq, Hkv, d, L_max, dtype, scale, q, k_cache, seq_lens, b, 0, h, s);
+            int nc = 0;
+            for (int j = 0; j < nk; j++) {
+                int lo = kept[j] * block_size, hi = lo + block_size;
+                if (hi > Lb) hi = Lb;
+                for (int i = lo; i < hi; i++) {
+                    sp[nc].s = s[i];
+                    sp[nc].i = i;
+                    nc++;
+                }
+            }
+            /* 4.-5. top k of the candidates, attention over them, discarded candidate mass */
+            qsort(sp, (size_t)nc, sizeof(scored_pos), cmp_score_desc);
+            int kk = k < nc ? k : nc;
+            size_t voff = ((size_t)b * Hkv + kvh) * (size_t)L_max * d;
+            attend_prefix(sp, nc, kk, v_cache, dtype, voff, d, out + (size_t)r * d, tail ? tail + r : NULL,
+                          idx + (size_t)r * k, k, sel);
+        }
+        free(sb);
+        free(sp);
+        free(s);
+        free(kept);
+        free(sel);
+    }
+    free(bk);
+    return status;
+}

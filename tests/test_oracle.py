@@ -419,3 +419,45 @@ def test_certified_equals_fixed_k_at_the_chosen_k():
             np.testing.assert_array_equal(r["out"][0, qp, h], f["out"][0, qp, h])
             np.testing.assert_array_equal(r["idx"][0, qp, h, :ku], f["idx"][0, qp, h])
             assert r["tail"][0, qp, h] == f["tail"][0, qp, h]
+
+
+# ----------------------------------------------------------------------------- hierarchical block -> token
+
+def test_hisa_with_every_block_is_token_topk():
+    w = workloads.make_workload(2, 1, 8, 2, 700, dtype="bf16", seq_lens=[700, 260], seed=71)
+    h = oracle.hisa_attn(w, block_size=32, top_blocks=64, k=100)
+    t = oracle.topk_attn(w, k=100)
+    np.testing.assert_array_equal(h["idx"], t["idx"])
+    np.testing.assert_array_equal(h["out"], t["out"])
+    np.testing.assert_array_equal(h["tail"], t["tail"])
+
+
+@pytest.mark.parametrize("bs,top,k", [(16, 3, 20), (32, 4, 200), (64, 2, 7)])
+def test_hisa_brute_force(bs, top, k):
+    """Block means, block ranking, candidate ranking and attention recomputed
+    with torch and numpy lexsort."""
+    w = workloads.make_workload(2, 1, 4, 2, 400, dtype="bf16", seq_lens=[400, 150], k_mean_std=0.5, seed=72)
+    r = oracle.hisa_attn(w, block_size=bs, top_blocks=top, k=k)
+    s_all = torch_scores(w)
+    for b in range(2):
+        Lb = int(w.seq_lens[b])
+        nblk = -(-Lb // bs)
+        for h in range(4):
+            Kh = _f64(w.k_cache[b, h // 2, :Lb])
+            means = torch.stack([Kh[j * bs:min((j + 1) * bs, Lb)].mean(0) for j in range(nblk)])
+            rb = (means @ _f64(w.q[b, 0, h])).numpy() / math.sqrt(128)
+            kept_b = np.sort(np.lexsort((np.arange(nblk), -rb))[:min(top, nblk)])
+            got_b = r["block_idx"][b, 0, h]
+            assert np.array_equal(got_b[:len(kept_b)], kept_b) and np.all(got_b[len(kept_b):] == -1)
+            cand = np.concatenate([np.arange(j * bs, min((j + 1) * bs, Lb)) for j in kept_b])
+            sc = s_all[b, 0, h, cand]
+            order = np.lexsort((cand, -sc))
+            kk = min(k, len(cand))
+            sel = np.sort(cand[order[:kk]])
+            got = r["idx"][b, 0, h]
+            assert np.array_equal(got[:kk], sel) and np.all(got[kk:] == -1)
+            p = torch.softmax(torch.from_numpy(s_all[b, 0, h, sel]), dim=0).numpy()
+            want = (p[:, None] * _f64(w.v_cache[b, h // 2, sel]).numpy()).sum(0)
+            np.testing.assert_allclose(r["out"][b, 0, h], want, rtol=1e-12, atol=1e-12)
+            pc = torch.softmax(torch.from_numpy(sc), dim=0).numpy()
+            assert abs(r["tail"][b, 0, h] - (1.0 - pc[order[:kk]].sum())) < 1e-12

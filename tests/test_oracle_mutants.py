@@ -33,6 +33,10 @@ MUTANTS = {
     "certified_k_one_too_many": ("                    kk = j + 1;\n", "                    kk = j + 1 < cap ? j + 2 : cap;\n"),
     "certified_mass_of_capped_prefix": ("for (int j = 0; j < vis; j++) z += exp(sp[j].s - m);",
                                         "for (int j = 0; j < (k_max < vis ? k_max : vis); j++) z += exp(sp[j].s - m);"),
+    "hisa_first_blocks_not_best": ("for (int j = 0; j < nk; j++) kept[j] = sb[j].i;\n            qsort(kept, (size_t)nk",
+                                   "for (int j = 0; j < nk; j++) kept[j] = j;\n            qsort(kept, (size_t)nk"),
+    "hisa_candidates_all_blocks": ("            for (int j = 0; j < nk; j++) {\n                int lo = kept[j] * block_size, hi = lo + block_size;\n                if (hi > Lb) hi = Lb;\n                for (int i = lo; i < hi; i++) {\n                    sp[nc]",
+                                   "            for (int j = 0; j < nblk; j++) {\n                int lo = j * block_size, hi = lo + block_size;\n                if (hi > Lb) hi = Lb;\n                for (int i = lo; i < hi; i++) {\n                    sp[nc]"),
     "current_block_not_forced": ("kept[nk] = nblk - 1; /* the current block */",
                                  "kept[nk] = nk < nblk - 1 ? sp[nk].i : nblk - 1;"),
 }
