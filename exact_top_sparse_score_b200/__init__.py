@@ -27,4 +27,5 @@ from ._binding import (  # noqa: F401
     topk_attn_workspace_size,
     topk_block_attn_decode,
     topk_block_pool_keys,
+    topk_hisa_attn_decode,
 )

@@ -59,6 +59,11 @@ def load_library() -> ctypes.CDLL:
         lib.topk_attn_decode_paged.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _i32, _vp,
                                                _vp, _vp, _vp, _sz, _vp]
         lib.topk_attn_decode_paged.restype = ctypes.c_int
+        lib.topk_hisa_attn_workspace_size.argtypes = [_shape_p, _i32, _i32, _i32]
+        lib.topk_hisa_attn_workspace_size.restype = _sz
+        lib.topk_hisa_attn_decode.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp,
+                                              _vp, _vp, _sz, _vp]
+        lib.topk_hisa_attn_decode.restype = ctypes.c_int
         lib.topk_attn_static_workspace_capacity.argtypes = []
         lib.topk_attn_static_workspace_capacity.restype = _sz
         lib.topk_attn_decode_static.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp]
@@ -393,3 +398,51 @@ def topk_attn_device_status(stream=None) -> int:
     if rc:
         raise TopkAttnError("topk_attn_device_status", rc)
     return int(bits.value)
+
+
+def topk_hisa_attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_keys: torch.Tensor,
+                          seq_lens: torch.Tensor, block_size: int, top_blocks: int, k: int, *, scale: float = 0.0,
+                          out: Optional[torch.Tensor] = None, idx: Optional[torch.Tensor] = None,
+                          tail_mass: Optional[torch.Tensor] = None, block_idx: Optional[torch.Tensor] = None,
+                          workspace: Optional[torch.Tensor] = None, stream=None):
+    """Hierarchical block -> token Top-k decode attention (one query per sequence).
+
+    Returns (out fp32 [B,1,Hq,d], idx int32 [B,1,Hq,k], tail fp32 [B,1,Hq],
+    block_idx int32 [B,1,Hq,top_blocks])."""
+    lib = load_library()
+    shape = make_shape(q, k_cache, scale)
+    B, Q, Hq, d = q.shape
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, Q, Hq, d), dtype=torch.float32, device=dev)
+    if idx is None:
+        idx = torch.empty((B, Q, Hq, k), dtype=torch.int32, device=dev)
+    if tail_mass is None:
+        tail_mass = torch.empty((B, Q, Hq), dtype=torch.float32, device=dev)
+    if block_idx is None:
+        block_idx = torch.empty((B, Q, Hq, top_blocks), dtype=torch.int32, device=dev)
+    if seq_lens.dtype != torch.int32 or tuple(seq_lens.shape) != (B,):
+        raise TypeError("seq_lens must be int32 [B]")
+    if v_cache.dtype != k_cache.dtype or v_cache.shape != k_cache.shape:
+        raise TypeError("v_cache must match k_cache in dtype and shape")
+    _check_out("out", out, torch.float32, (B, Q, Hq, d))
+    _check_out("idx", idx, torch.int32, (B, Q, Hq, k))
+    _check_out("tail_mass", tail_mass, torch.float32, (B, Q, Hq))
+    _check_out("block_idx", block_idx, torch.int32, (B, Q, Hq, top_blocks))
+    _check_out("block_keys", block_keys, torch.float32, (B, k_cache.shape[1], -(-k_cache.shape[2] // block_size), d))
+    if workspace is not None and workspace.dtype != torch.uint8:
+        raise TypeError("workspace must be a uint8 tensor")
+    _check_cuda(q=q, k_cache=k_cache, v_cache=v_cache, block_keys=block_keys, seq_lens=seq_lens, out=out, idx=idx,
+                tail_mass=tail_mass, block_idx=block_idx, workspace=workspace)
+    nbytes = int(lib.topk_hisa_attn_workspace_size(ctypes.byref(shape), block_size, top_blocks, k))
+    if nbytes == 0:
+        raise TopkAttnError("topk_hisa_attn_workspace_size", 2)
+    sh = _stream(stream)
+    ws = _workspace(nbytes, dev, workspace, sh)
+    rc = lib.topk_hisa_attn_decode(ctypes.byref(shape), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                   block_keys.data_ptr(), seq_lens.data_ptr(), block_size, top_blocks, k,
+                                   out.data_ptr(), idx.data_ptr(), tail_mass.data_ptr(), block_idx.data_ptr(),
+                                   ws.data_ptr(), nbytes, sh)
+    if rc:
+        raise TopkAttnError("topk_hisa_attn_decode", rc)
+    return out, idx, tail_mass, block_idx

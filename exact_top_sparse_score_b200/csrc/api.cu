@@ -150,6 +150,54 @@ tka_status check_block_args(const tka_shape *s, int block_size, int top_blocks) 
     return TKA_OK;
 }
 
+// Workspace of topk_hisa_attn_decode, in order (256-byte aligned regions):
+//   bscore    fp32 [rows, nblk_max]   block scores
+//   block_idx int32 [rows, top]       (when the caller passes none)
+//   cscore    fp32 [rows, ldc]        candidate scores, ldc = top * bs rounded up to 64
+//   row_len   int32 [rows]            valid candidates per row
+//   weights   fp32 [rows, k], stats float4 [rows], partial fp32 [rows, k/64, d], counters uint32 [rows]
+struct HisaLayout {
+    size_t bscore, block_idx, cscore, row_len, weights, stats, partial, counters, total;
+    int ldc, max_splits;
+};
+
+HisaLayout hisa_layout(const tka_shape *s, int block_size, int top_blocks, int k) {
+    HisaLayout L;
+    const size_t rows = (size_t)s->B * s->Hq;
+    const size_t nblk_max = ((size_t)s->L_max + block_size - 1) / block_size;
+    L.ldc = (int)align_up((size_t)top_blocks * block_size, 64);
+    L.max_splits = (k + kMinKeysPerSplit - 1) / kMinKeysPerSplit;
+    size_t off = 0;
+    L.bscore = off;
+    off = align_up(off + rows * nblk_max * sizeof(float), 256);
+    L.block_idx = off;
+    off = align_up(off + rows * (size_t)top_blocks * sizeof(int32_t), 256);
+    L.cscore = off;
+    off = align_up(off + rows * (size_t)L.ldc * sizeof(float), 256);
+    L.row_len = off;
+    off = align_up(off + rows * sizeof(int32_t), 256);
+    L.weights = off;
+    off = align_up(off + rows * (size_t)k * sizeof(float), 256);
+    L.stats = off;
+    off = align_up(off + rows * sizeof(float4), 256);
+    L.partial = off;
+    off = align_up(off + rows * (size_t)L.max_splits * kHeadDim * sizeof(float), 256);
+    L.counters = off;
+    off = align_up(off + rows * sizeof(unsigned), 256);
+    L.total = off;
+    return L;
+}
+
+tka_status check_hisa_args(const tka_shape *s, int block_size, int top_blocks, int k) {
+    tka_status st = check_shape(s);
+    if (st != TKA_OK) return st;
+    if (block_size < 1 || top_blocks < 1 || k < 1) return TKA_ERR_INVALID_ARG;
+    if (block_size != 16 && block_size != 32 && block_size != 64 && block_size != 128) return TKA_ERR_UNSUPPORTED;
+    if (s->Q != 1 || top_blocks > 8192 || k > kMaxK) return TKA_ERR_UNSUPPORTED;
+    if ((s->L_max + block_size - 1) / block_size > 8192) return TKA_ERR_UNSUPPORTED;
+    return TKA_OK;
+}
+
 }  // namespace
 }  // namespace tka
 
@@ -408,6 +456,106 @@ tka_status topk_block_attn_decode(const tka_shape *shape, const void *q, const v
     ap.counters = counters;
     ap.out = out;
     if (launch_block_attn(ap, k_cache, dev->num_sms, s) != cudaSuccess) return TKA_ERR_CUDA;
+    return TKA_OK;
+}
+
+size_t topk_hisa_attn_workspace_size(const tka_shape *shape, int32_t block_size, int32_t top_blocks, int32_t k) {
+    if (check_hisa_args(shape, block_size, top_blocks, k) != TKA_OK) return 0;
+    return hisa_layout(shape, block_size, top_blocks, k).total;
+}
+
+tka_status topk_hisa_attn_decode(const tka_shape *shape, const void *q, const void *k_cache, const void *v_cache,
+                                 const float *block_keys, const int32_t *seq_lens, int32_t block_size,
+                                 int32_t top_blocks, int32_t k, float *out, int32_t *idx, float *tail_mass,
+                                 int32_t *block_idx, void *workspace, size_t workspace_bytes, tka_stream_t stream) {
+    tka_status st = check_hisa_args(shape, block_size, top_blocks, k);
+    if (st != TKA_OK) return st;
+    if (!q || !k_cache || !v_cache || !block_keys || !seq_lens || !out || !idx) return TKA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(block_keys, 16) ||
+        !aligned(out, 16) || !aligned(idx, 4) || !aligned(seq_lens, 4) || (tail_mass && !aligned(tail_mass, 4)) ||
+        (block_idx && !aligned(block_idx, 4)))
+        return TKA_ERR_INVALID_ARG;
+    const HisaLayout L = hisa_layout(shape, block_size, top_blocks, k);
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < L.total) return TKA_ERR_WORKSPACE;
+    DeviceInfo *dev = nullptr;
+    if (device_info(&dev) != cudaSuccess) return TKA_ERR_CUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    char *ws = static_cast<char *>(workspace);
+    const int G = shape->Hq / shape->Hkv;
+    const int rows = shape->B * shape->Hq;
+    const int nblk_max = (shape->L_max + block_size - 1) / block_size;
+    int32_t *bidx = block_idx ? block_idx : reinterpret_cast<int32_t *>(ws + L.block_idx);
+    int32_t *row_len = reinterpret_cast<int32_t *>(ws + L.row_len);
+    unsigned *counters = reinterpret_cast<unsigned *>(ws + L.counters);
+    const float scale = resolve_scale(shape);
+
+    // 1. blocks: every block competes for the top_blocks slots
+    BlockSelectParams bp;
+    bp.status = dev->status;
+    bp.q = q;
+    bp.block_keys = block_keys;
+    bp.seq_lens = seq_lens;
+    bp.B = shape->B; bp.Hq = shape->Hq; bp.Hkv = shape->Hkv; bp.G = G; bp.L_max = shape->L_max;
+    bp.block_size = block_size; bp.nblk_max = nblk_max; bp.top_blocks = top_blocks; bp.dtype = shape->dtype;
+    bp.scale = scale;
+    bp.bscore = reinterpret_cast<float *>(ws + L.bscore);
+    bp.block_idx = bidx;
+    bp.counters = nullptr;
+    bp.force_last = 0;
+    if (launch_block_select(bp, s) != cudaSuccess) return TKA_ERR_CUDA;
+
+    // 2. token scores inside the kept blocks
+    HisaScoreParams hp;
+    hp.status = dev->status;
+    hp.q = q; hp.k = k_cache;
+    hp.seq_lens = seq_lens;
+    hp.block_idx = bidx;
+    hp.B = shape->B; hp.Hq = shape->Hq; hp.Hkv = shape->Hkv; hp.G = G; hp.L_max = shape->L_max;
+    hp.block_size = block_size; hp.top_blocks = top_blocks; hp.ldc = L.ldc; hp.dtype = shape->dtype;
+    hp.scale = scale;
+    hp.cscore = reinterpret_cast<float *>(ws + L.cscore);
+    hp.row_len = row_len;
+    if (launch_hisa_scores(hp, s) != cudaSuccess) return TKA_ERR_CUDA;
+
+    // 3. the top k candidates (candidate order is position order)
+    SelectParams se;
+    se.status = dev->status;
+    se.scores = hp.cscore;
+    se.seq_lens = seq_lens;
+    se.B = shape->B; se.Q = 1; se.Hq = shape->Hq; se.L_max = shape->L_max; se.ld = L.ldc; se.k = k;
+    se.idx = idx;
+    se.w = reinterpret_cast<float *>(ws + L.weights);
+    se.stats = reinterpret_cast<float4 *>(ws + L.stats);
+    se.tail = tail_mass;
+    se.counters = counters;
+    se.row_len = row_len;
+    if (launch_select(se, s) != cudaSuccess) return TKA_ERR_CUDA;
+
+    // 4. softmax over the kept tokens and P.V; candidate indices become positions
+    GatherParams gp;
+    gp.status = dev->status;
+    gp.v = v_cache;
+    gp.seq_lens = seq_lens;
+    gp.B = shape->B; gp.Q = 1; gp.Hq = shape->Hq; gp.Hkv = shape->Hkv; gp.G = G;
+    gp.L_max = shape->L_max; gp.k = k; gp.dtype = shape->dtype;
+    gp.idx = idx;
+    gp.w = se.w;
+    gp.stats = se.stats;
+    gp.partial = reinterpret_cast<float *>(ws + L.partial);
+    gp.counters = counters;
+    gp.out = out;
+    gp.kcount = row_len;
+    gp.cblock = bidx;
+    gp.crow_len = row_len;
+    gp.idx_out = idx;
+    gp.cbs = block_size;
+    gp.cstride = top_blocks;
+    int splits = (dev->num_sms * 8) / rows;
+    if (splits > L.max_splits) splits = L.max_splits;
+    if (splits < 1) splits = 1;
+    gp.per_split = (k + splits - 1) / splits;
+    gp.splits = (k + gp.per_split - 1) / gp.per_split;
+    if (launch_gather(gp, s) != cudaSuccess) return TKA_ERR_CUDA;
     return TKA_OK;
 }
 

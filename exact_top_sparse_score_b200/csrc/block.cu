@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(kSelThreads) block_scores(BlockSelectParams p)
     const int bh = blockIdx.y, b = bh / p.Hkv, kvh = bh - b * p.Hkv;
     const int seq_len = p.seq_lens[b];
     if (seq_len < 1 || seq_len > p.L_max) return;  // block_topk raises the status
-    const int ncomp = (seq_len + p.block_size - 1) / p.block_size - 1;
+    const int ncomp = (seq_len + p.block_size - 1) / p.block_size - p.force_last;
     const int j0 = blockIdx.x * kScoreBlocks;
     if (j0 >= ncomp || ncomp <= p.top_blocks) return;  // nothing to rank here
     const T *q = reinterpret_cast<const T *>(p.q) + ((size_t)b * p.Hq + (size_t)kvh * p.G) * kHeadDim;
@@ -152,13 +152,14 @@ __global__ void __launch_bounds__(kSelThreads) block_topk(BlockSelectParams p) {
         if (threadIdx.x == 0) raise_status(p.status, TKA_DEV_BAD_SEQ_LEN);
         return;
     }
-    if (threadIdx.x == 0) p.counters[row] = 0u;
+    if (threadIdx.x == 0 && p.counters) p.counters[row] = 0u;
     const int nblk = (seq_len + p.block_size - 1) / p.block_size;
-    const int ncomp = nblk - 1;  // blocks competing for the top_blocks slots
+    const int ncomp = nblk - p.force_last;  // blocks competing for the top_blocks slots
     const int top = p.top_blocks;
-    int32_t *out = p.block_idx + (size_t)row * (top + 1);
+    const int width = top + p.force_last;
+    int32_t *out = p.block_idx + (size_t)row * width;
     if (ncomp <= top) {  // every block is kept: nothing to rank
-        for (int i = threadIdx.x; i <= top; i += kSelThreads) out[i] = i < nblk ? i : -1;
+        for (int i = threadIdx.x; i < width; i += kSelThreads) out[i] = i < nblk ? i : -1;
         return;
     }
     if (top == 0) {  // only the current block
@@ -204,7 +205,47 @@ __global__ void __launch_bounds__(kSelThreads) block_topk(BlockSelectParams p) {
         if (u == T) keep = eqr++ < need;
         if (keep) out[pos++] = j;
     }
-    if (threadIdx.x == 0) out[top] = nblk - 1;  // the current block has the highest index
+    if (threadIdx.x == 0 && p.force_last) out[top] = nblk - 1;  // the current block has the highest index
+}
+
+// ---------------------------------------------------------------- hisa_scores
+//
+// Hierarchical selection ("Sparse Attention Landscape", section "Hierarchical
+// Sparse Attention"): token scores only inside the kept blocks.  Grid (slot,
+// row): the CTA scores the tokens of the row's slot-th kept block into
+// cscore[row, slot * bs + t] (-inf past the sequence end); the kept blocks are
+// ascending and only the sequence's last block can be partial, so the valid
+// candidates are a prefix of the row, whose length slot 0 records.
+template <typename T>
+__global__ void __launch_bounds__(128) hisa_scores(HisaScoreParams p) {
+    const int slot = blockIdx.x, row = blockIdx.y, b = row / p.Hq, h = row - b * p.Hq;
+    const int seq_len = p.seq_lens[b];
+    if (seq_len < 1 || seq_len > p.L_max) return;  // block_topk raised the status
+    const int32_t *bi = p.block_idx + (size_t)row * p.top_blocks;
+    if (slot == 0 && threadIdx.x == 0) {
+        int len = 0;
+        for (int s2 = 0; s2 < p.top_blocks && bi[s2] >= 0; s2++)
+            len = s2 * p.block_size + min(p.block_size, seq_len - bi[s2] * p.block_size);
+        p.row_len[row] = len;
+    }
+    const int j = bi[slot];
+    float *dst = p.cscore + (size_t)row * p.ldc + (size_t)slot * p.block_size;
+    if (j < 0) {
+        for (int t = threadIdx.x; t < p.block_size; t += 128) dst[t] = -INFINITY;
+        return;
+    }
+    const int lo = j * p.block_size, n = min(p.block_size, seq_len - lo);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const float4 qv = load4(reinterpret_cast<const T *>(p.q) + (size_t)row * kHeadDim + 4 * lane);
+    const T *K = reinterpret_cast<const T *>(p.k) + (((size_t)b * p.Hkv + h / p.G) * p.L_max + lo) * kHeadDim;
+    for (int t = warp; t < p.block_size; t += 4) {
+        float s = -INFINITY;
+        if (t < n) {
+            const float4 kv = load4(K + (size_t)t * kHeadDim + 4 * lane);
+            s = warp_sum(qv.x * kv.x + qv.y * kv.y + qv.z * kv.z + qv.w * kv.w) * p.scale;
+        }
+        if (lane == 0) dst[t] = s;
+    }
 }
 
 // ---------------------------------------------------------------- block_attn
@@ -642,6 +683,15 @@ cudaError_t launch_block_select(const BlockSelectParams &p, cudaStream_t stream)
     const size_t ksmem = (size_t)p.nblk_max * sizeof(uint32_t);
     if ((e = allow_smem(block_topk, ksmem)) != cudaSuccess) return e;
     block_topk<<<p.B * p.Hq, kSelThreads, ksmem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_hisa_scores(const HisaScoreParams &p, cudaStream_t stream) {
+    const dim3 grid(p.top_blocks, p.B * p.Hq);
+    if (p.dtype == TKA_BF16)
+        hisa_scores<__nv_bfloat16><<<grid, 128, 0, stream>>>(p);
+    else
+        hisa_scores<float><<<grid, 128, 0, stream>>>(p);
     return cudaGetLastError();
 }
 

@@ -90,6 +90,14 @@ __global__ void __launch_bounds__(kGatherThreads, 8) gather_pv(GatherParams p) {
         for (int j = threadIdx.x; j < n; j += kGatherThreads) {
             int pos = __ldg(gidx + c0 + j);
             float wt = __ldg(gw + c0 + j);
+            if (p.cblock) {  // a candidate index: map it to its position, report the position
+                if ((unsigned)pos < (unsigned)p.crow_len[row]) {
+                    pos = p.cblock[(size_t)row * p.cstride + pos / p.cbs] * p.cbs + pos % p.cbs;
+                    p.idx_out[(size_t)row * p.k + c0 + j] = pos;
+                } else {
+                    pos = -1;
+                }
+            }
             if ((unsigned)pos >= (unsigned)vis) {  // never taken unless the select step is wrong
                 bad = true;
                 pos = 0;

@@ -41,6 +41,8 @@ struct SelectParams {
     float4 *stats;            // [rows] {m, Z_k, Z_tail, 0}
     float *tail;              // [rows] or null
     unsigned *counters;       // [rows], zeroed here for the combine step
+    const int32_t *row_len = nullptr;  // [rows] scores per row (compact candidate rows), or null:
+                                       // the visible keys of the row
 };
 
 struct GatherParams {
@@ -57,6 +59,24 @@ struct GatherParams {
     int splits, per_split;
     const int32_t *kcount;    // [rows] kept positions per row, or null: min(k, visible keys)
     PageTable pages;          // v is the paged cache when pages.table is set
+    // Candidate rows (hierarchical selection): idx holds indices into a row of
+    // candidates, slot-major over the kept blocks; position = cblock[row,
+    // c / cbs] * cbs + c % cbs.  The gather writes the positions back to idx.
+    const int32_t *cblock = nullptr;  // [rows, cstride]
+    const int32_t *crow_len = nullptr;  // [rows] valid candidates
+    int32_t *idx_out = nullptr;         // [rows, k] the same buffer as idx
+    int cbs = 0, cstride = 0;
+};
+
+struct HisaScoreParams {
+    unsigned *status;         // device status word (TKA_DEV_* bits)
+    const void *q, *k;        // q [B, 1, Hq, 128], K [B, Hkv, L_max, 128]
+    const int32_t *seq_lens;
+    const int32_t *block_idx; // [rows, top_blocks] ascending, -1 padded
+    int B, Hq, Hkv, G, L_max, block_size, top_blocks, ldc, dtype;
+    float scale;
+    float *cscore;            // [rows, ldc] candidate scores, slot-major
+    int32_t *row_len;         // [rows] valid candidates (a prefix of the row)
 };
 
 struct CertifyParams {
@@ -88,8 +108,10 @@ struct BlockSelectParams {
     int B, Hq, Hkv, G, L_max, block_size, nblk_max, top_blocks, dtype;
     float scale;
     float *bscore;            // [B*Hq, nblk_max] block scores of the competing blocks
-    int32_t *block_idx;       // [B*Hq, top_blocks + 1] (workspace or caller's)
-    unsigned *counters;       // [B*Hq], zeroed here for the attention step
+    int32_t *block_idx;       // [B*Hq, top_blocks + force_last] (workspace or caller's)
+    unsigned *counters;       // [B*Hq], zeroed here for the attention step (may be null)
+    int force_last = 1;       // 1: the current block is always kept and does not compete (MoBA);
+                              // 0: every block competes for the top_blocks slots
 };
 
 struct BlockAttnParams {
@@ -129,6 +151,7 @@ cudaError_t launch_gather(const GatherParams &p, cudaStream_t stream);
 cudaError_t launch_certify(const CertifyParams &p, cudaStream_t stream);
 cudaError_t launch_block_pool(const BlockPoolParams &p, cudaStream_t stream);
 cudaError_t launch_block_select(const BlockSelectParams &p, cudaStream_t stream);
+cudaError_t launch_hisa_scores(const HisaScoreParams &p, cudaStream_t stream);
 cudaError_t launch_block_attn(const BlockAttnParams &p, const void *k_cache, int num_sms, cudaStream_t stream);
 
 }  // namespace tka

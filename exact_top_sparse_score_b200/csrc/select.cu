@@ -253,7 +253,7 @@ __global__ void __launch_bounds__(kSelectThreads, kSelectCtasPerSm) select_topk(
         if (threadIdx.x == 0) raise_status(p.status, TKA_DEV_BAD_SEQ_LEN);
         return;
     }
-    const int vis = visible_keys(seq_len, p.Q, qpos);
+    const int vis = p.row_len ? p.row_len[row] : visible_keys(seq_len, p.Q, qpos);
     const int k = p.k;
     const float *s = p.scores + (size_t)row * p.ld;
     if (k >= vis) {  // every visible key is kept

@@ -195,6 +195,30 @@ tka_status topk_block_attn_decode(const tka_shape *shape, const void *q, const v
                                   float *out, int32_t *block_idx, void *workspace,
                                   size_t workspace_bytes, tka_stream_t stream);
 
+/* Hierarchical block -> token Top-k ("Sparse Attention Landscape", section
+ * "Hierarchical Sparse Attention"), one query per sequence (shape->Q == 1).
+ * With nblk = ceil(seq_lens[b] / block_size): every block j < nblk scores
+ * r_j = scale * <q, block_keys[b, h/G, j, :]> (the mean keys of
+ * topk_block_pool_keys); the best top_blocks blocks (ties to the lower j) are
+ * kept; exact token scores are computed only for the tokens of the kept
+ * blocks (the candidates); the top k candidates (ties to the lower position)
+ * are kept and out is softmax attention over them.
+ *   idx        int32 [B, 1, Hq, k] ascending positions, -1 padded when fewer
+ *              than k candidates exist.
+ *   tail_mass  (nullable) the candidates' discarded softmax mass, relative to
+ *              all candidates.
+ *   block_idx  (nullable) int32 [B, 1, Hq, top_blocks] ascending, -1 padded.
+ *   workspace  topk_hisa_attn_workspace_size(shape, block_size, top_blocks, k)
+ *              bytes (0 on unsupported arguments).
+ * Supported: block_size in {16, 32, 64, 128}, 1 <= top_blocks <= 8192,
+ * 1 <= k <= 8192, ceil(L_max / block_size) <= 8192. */
+size_t topk_hisa_attn_workspace_size(const tka_shape *shape, int32_t block_size, int32_t top_blocks, int32_t k);
+tka_status topk_hisa_attn_decode(const tka_shape *shape, const void *q, const void *k_cache,
+                                 const void *v_cache, const float *block_keys, const int32_t *seq_lens,
+                                 int32_t block_size, int32_t top_blocks, int32_t k, float *out, int32_t *idx,
+                                 float *tail_mass, int32_t *block_idx, void *workspace,
+                                 size_t workspace_bytes, tka_stream_t stream);
+
 /* Synchronises `stream`, returns the device status word of the current device
  * (TKA_DEV_* bits raised by kernels since the last read) in *bits and clears it. */
 tka_status topk_attn_device_status(tka_stream_t stream, uint32_t *bits);

@@ -183,3 +183,60 @@ def check_certified(w, eps, k_max, out, idx, tail, k_used, ref, scale=0.0, rows_
         assert _close(out[b, qp, h], vo, atol, rtol).all(), f"{where}: out invalid for its own set"
         assert abs(tail[b, qp, h] - vt) <= TAIL_TOL, f"{where}: tail invalid for its own set"
     return n_diff
+
+
+def check_hisa(w, block_size, top_blocks, k, out, idx, tail, bidx, ref, scale=0.0):
+    """Asserts parity of topk_hisa_attn_decode with oracle.hisa_attn output `ref`.
+
+    Kept blocks equal the oracle's except blocks whose fp64 block score lies
+    within BAND of the oracle's top_blocks-th; kept tokens equal the top k of
+    the GPU's own candidates except positions within BAND of the k-th
+    candidate score; out and tail match the oracle where the sets agree and an
+    fp64 evaluation over the GPU's own sets otherwise.  Returns the number of
+    rows checked through the band."""
+    out = out.detach().cpu().double().numpy()
+    idx = idx.detach().cpu().numpy()
+    tail = tail.detach().cpu().double().numpy()
+    bidx = bidx.detach().cpu().numpy()
+    atol, rtol = out_tol(w.dtype)
+    bk = None
+    n_band = 0
+    for b in range(w.B):
+        Lb = int(w.seq_lens[b])
+        nblk = -(-Lb // block_size)
+        nk = min(top_blocks, nblk)
+        for h in range(w.Hq):
+            where = f"row (b={b}, h={h})"
+            gb, ob = bidx[b, 0, h], ref["block_idx"][b, 0, h]
+            assert np.all(gb[nk:] == -1) and np.all(np.diff(gb[:nk]) > 0) and gb[0] >= 0, f"{where}: block list"
+            s = oracle.row_scores(w, b, 0, h, scale)
+            if not np.array_equal(gb[:nk], ob[:nk]):
+                n_band += 1
+                if bk is None:
+                    bk = oracle.block_pool(w, block_size)
+                r = oracle_block_scores(w, bk, b, h, scale)[:nblk]
+                kth = np.sort(r)[::-1][nk - 1]
+                diff = np.setxor1d(gb[:nk], ob[:nk])
+                assert np.all(np.abs(r[diff] - kth) <= BAND), f"{where}: blocks differ outside the tie band"
+            cand = np.concatenate([np.arange(j * block_size, min((j + 1) * block_size, Lb)) for j in gb[:nk]])
+            kk = min(k, len(cand))
+            g = idx[b, 0, h]
+            assert np.all(g[kk:] == -1), f"{where}: padding"
+            gs = g[:kk]
+            assert np.all(np.isin(gs, cand)) and np.all(np.diff(gs) > 0), f"{where}: kept tokens"
+            order = np.lexsort((cand, -s[cand]))
+            top = np.sort(cand[order[:kk]])
+            kth_s = s[cand[order[kk - 1]]]
+            assert np.all(np.abs(s[np.setxor1d(gs, top)] - kth_s) <= BAND), f"{where}: tokens outside the tie band"
+            if np.array_equal(gb[:nk], ob[:nk]) and np.array_equal(gs, ref["idx"][b, 0, h, :kk]):
+                assert _close(out[b, 0, h], ref["out"][b, 0, h], atol, rtol).all(), f"{where}: out"
+                assert abs(tail[b, 0, h] - ref["tail"][b, 0, h]) <= TAIL_TOL, f"{where}: tail"
+                continue
+            n_band += 1
+            e_all = np.exp(s[cand] - s[cand].max())
+            e = np.exp(s[gs] - s[gs].max())
+            V = w.v_cache[b, h // w.G].double().numpy()[gs]
+            assert _close(out[b, 0, h], (e[:, None] * V).sum(0) / e.sum(), atol, rtol).all(), f"{where}: out invalid"
+            kept_mass = np.exp(s[gs] - s[cand].max()).sum() / e_all.sum()
+            assert abs(tail[b, 0, h] - (1.0 - kept_mass)) <= TAIL_TOL, f"{where}: tail invalid"
+    return n_band
