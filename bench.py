@@ -57,6 +57,9 @@ def parse_args():
                     help="override the workload's batch size (smaller cases for profiling)")
     ap.add_argument("--paged", type=int, default=None, metavar="PAGE_SIZE",
                     help="lay the cache out as shuffled pages of PAGE_SIZE positions (block tables)")
+    ap.add_argument("--hisa", type=str, default=None, metavar="BLOCK_SIZE,TOP_BLOCKS",
+                    help="hierarchical block -> token Top-k: score only the tokens of the best TOP_BLOCKS "
+                         "blocks of BLOCK_SIZE (one-query workloads)")
     ap.add_argument("--certified-eps", type=float, default=None,
                     help="certified adaptive Top-k: per row the smallest k (at most the workload's k) "
                          "whose discarded tail mass is <= EPS")
@@ -254,6 +257,9 @@ def run_ours(args, world, rank, local):
     block = w.variant == "block"
     certified = args.certified_eps is not None and not block
     paged = args.paged is not None and not block and not certified
+    hisa = args.hisa is not None and not block and not certified and not paged
+    if hisa:
+        h_bs, h_top = (int(x) for x in args.hisa.split(","))
     k = w.k
     if block:
         bk = tka.topk_block_pool_keys(kc, lens, w.block_size)
@@ -287,6 +293,20 @@ def run_ours(args, world, rank, local):
                     events[0].record()
                 tka.topk_attn_decode_certified(qq, kc, vc, lens, args.certified_eps, k, out=out, idx=idx,
                                                tail_mass=tail, k_used=k_used, workspace=ws)
+                if events:
+                    events[3].record()
+        elif hisa:
+            h_bk = tka.topk_block_pool_keys(kc, lens, h_bs)
+            h_bidx = torch.empty((w.B, 1, w.Hq, h_top), dtype=torch.int32, device=dev)
+            ws = torch.empty(tka._binding.load_library().topk_hisa_attn_workspace_size(
+                make_shape(q, kc), h_bs, h_top, k), dtype=torch.uint8, device=dev)
+            launches_per_step = 5  # block_scores, block_topk, hisa_scores, select, gather
+
+            def step(events=None, qq=q):
+                if events:
+                    events[0].record()
+                tka.topk_hisa_attn_decode(qq, kc, vc, h_bk, lens, h_bs, h_top, k, out=out, idx=idx,
+                                          tail_mass=tail, block_idx=h_bidx, workspace=ws)
                 if events:
                     events[3].record()
         elif paged:
@@ -336,7 +356,7 @@ def run_ours(args, world, rank, local):
     if world > 1:
         torch.distributed.barrier()
     step_ms = [e[0].elapsed_time(e[3]) for e in evs]
-    stage_ms = None if block or certified or paged else [[e[j].elapsed_time(e[j + 1]) for e in evs] for j in range(3)]
+    stage_ms = None if block or certified or paged or hisa else [[e[j].elapsed_time(e[j + 1]) for e in evs] for j in range(3)]
     total_ms = sum(step_ms)
 
     e2e_ms = None
@@ -367,6 +387,9 @@ def run_ours(args, world, rank, local):
             elif paged:
                 tka.topk_attn_decode_paged(q_step, kp, vp, table, lens_step, k, out=out, idx=idx,
                                            tail_mass=tail, workspace=ws)
+            elif hisa:
+                tka.topk_hisa_attn_decode(q_step, kc, vc, h_bk, lens_step, h_bs, h_top, k, out=out, idx=idx,
+                                          tail_mass=tail, block_idx=h_bidx, workspace=ws)
             else:
                 tka.topk_attn_decode(q_step, kc, vc, lens_step, k, out=out, idx=idx, tail_mass=tail, workspace=ws)
             for h, t in zip(hosts, outs):
@@ -409,6 +432,7 @@ def run_ours(args, world, rank, local):
             "l2": "flushed between timed steps (256 MiB write + 256 MiB read, outside the timed events)",
             **({"certified_eps": args.certified_eps, "k_max": k} if certified else {}),
             **({"page_size": args.paged, "pages": "shuffled pool, block tables"} if paged else {}),
+            **({"hisa_block_size": h_bs, "hisa_top_blocks": h_top} if hisa else {}),
         },
         "us_per_step": ms * 1e3,
         "tokens_per_s": world * w.B * w.Q / (ms / 1e3),
@@ -419,6 +443,20 @@ def run_ours(args, world, rank, local):
         "gpu_launches": launches_per_step * K,
         "clocks": clocks.summary(),
     }
+    if hisa:
+        # algorithmic bytes: block keys + the kept blocks' K rows + the k kept V rows + q/out/idx
+        row = w.d * elem_bytes(w)
+        nblk = -(-w.L_max // h_bs)
+        alg = rows * (nblk * w.d * 4 // w.G + h_top * h_bs * row + k * row) + rows * w.d * (elem_bytes(w) + 4) + rows * 4 * (k + 1)
+        res["alg_bytes_per_step"] = alg
+        res["alg_gbs"] = alg / (ms / 1e3) / 1e9
+        res["alg_frac_of_spec_8tbs"] = res["alg_gbs"] / SPEC_HBM_GBS
+        res["alg_frac_of_measured_hbm"] = res["alg_gbs"] / peak
+        res["roofline"] = {"kernel": "whole step (hierarchical: blocks + candidates + select + gather)",
+                           "bound": "hbm", "achieved": res["alg_gbs"], "peak": peak,
+                           "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
+                           else "fallback 6.65 TB/s", "unit": "GB/s", "frac": res["alg_gbs"] / peak,
+                           "traffic": None, "alg_bytes_per_launch": alg}
     if paged:
         # no per-kernel events on this path: the whole step against the copy peak
         res["roofline"] = {"kernel": "whole step (paged: score + select + gather)", "bound": "hbm",
