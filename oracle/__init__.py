@@ -56,6 +56,10 @@ def _load():
         lib.oracle_certified_attn.restype = _i
         lib.oracle_hisa_attn.argtypes = [_i] * 6 + [_d, _vp, _vp, _vp, _ip, _i, _i, _i, _dp, _ip, _ip, _dp, _i]
         lib.oracle_hisa_attn.restype = _i
+        lib.oracle_indexer_attn.argtypes = [_i] * 7 + [_d, _vp, _vp, _vp, _ip, _i, _i, _vp,
+                                                       np.ctypeslib.ndpointer(dtype=np.float32, flags="C_CONTIGUOUS"),
+                                                       _vp, _i, _dp, _ip, _dp, _i]
+        lib.oracle_indexer_attn.restype = _i
         lib.oracle_block_pool.argtypes = [_i] * 5 + [_vp, _ip, _i, _dp]
         lib.oracle_block_pool.restype = _i
         lib.oracle_block_attn.argtypes = [_i] * 6 + [_d, _vp, _vp, _vp, _ip, _i, _i, _dp, _ip, _dp, _dp, _i]
@@ -190,3 +194,27 @@ def hisa_attn(w, block_size: int, top_blocks: int, k: int, scale: float = 0.0, n
     if rc:
         raise ValueError(f"oracle_hisa_attn failed with code {rc}")
     return dict(out=out, block_idx=bidx, idx=idx, tail=tail)
+
+
+def indexer_attn(w, q_idx, w_idx, k_idx, k: int, scale: float = 0.0, nthreads: int = 0) -> dict:
+    """Token selection by a lightning indexer, then exact attention per head.
+
+    q_idx [B,Q,H_I,d_I] and k_idx [B,L_max,d_I] in the cache dtype (torch
+    tensors), w_idx [B,Q,H_I] fp32.  Returns out [B,Q,Hq,d] f64, idx [B,Q,k]
+    (ascending, -1 padded, shared by all heads of a query position) and kth
+    [B,Q] (the smallest kept indexer score).
+    """
+    lib = _load()
+    B, Q, H_I, d_I = q_idx.shape
+    q, kc, vc, lens = _arr(w, w.q), _arr(w, w.k_cache), _arr(w, w.v_cache), _lens(w)
+    qi, ki = _arr(w, q_idx), _arr(w, k_idx)
+    wi = np.ascontiguousarray(w_idx.numpy().astype(np.float32))
+    out = np.zeros((w.B, w.Q, w.Hq, w.d), np.float64)
+    idx = np.zeros((w.B, w.Q, k), np.int32)
+    kth = np.zeros((w.B, w.Q), np.float64)
+    rc = lib.oracle_indexer_attn(w.B, w.Q, w.Hq, w.Hkv, w.d, w.L_max, _code(w.dtype), scale,
+                                 q.ctypes.data, kc.ctypes.data, vc.ctypes.data, lens, H_I, d_I,
+                                 qi.ctypes.data, wi, ki.ctypes.data, k, out, idx, kth, nthreads)
+    if rc:
+        raise ValueError(f"oracle_indexer_attn failed with code {rc}")
+    return dict(out=out, idx=idx, kth=kth)

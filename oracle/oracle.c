@@ -480,3 +480,85 @@ int oracle_hisa_attn(int B, int Hq, int Hkv, int d, int L_max, int dtype, double
     free(bk);
     return status;
 }
+
+/*
+ * Token selection by a lightning indexer ("Sparse Attention Landscape",
+ * section "Token Sparse Attention", DeepSeek Sparse Attention): the indexer
+ * scores every visible token of a query position with its own small heads,
+ *   I_i = sum_j w[j] * ReLU(<q_idx[j], k_idx[i]>),   j < H_I,
+ * where q_idx [B, Q, H_I, d_I], w_idx [B, Q, H_I] (fp32) and k_idx
+ * [B, L_max, d_I] are the indexer's projected queries, head weights and keys
+ * (inputs here); the top k tokens by I (descending, position ascending) are
+ * kept for the query position, shared by all attention heads; then every
+ * head h attends over them with its exact scores:
+ *   out = sum_{i kept} softmax_i(scale * <q_h, K[b, h / G, i, :]>) V[b, h / G, i, :].
+ * idx [B, Q, k] ascending, -1 padded; kth_index [B, Q] the smallest kept I.
+ */
+int oracle_indexer_attn(int B, int Q, int Hq, int Hkv, int d, int L_max, int dtype, double scale,
+                        const void *q, const void *k_cache, const void *v_cache, const int32_t *seq_lens,
+                        int H_I, int d_I, const void *q_idx, const float *w_idx, const void *k_idx, int k,
+                        double *out, int32_t *idx, double *kth_index, int nthreads) {
+    if (!check_shape(B, Q, Hq, Hkv, d, L_max, dtype) || H_I < 1 || d_I < 1 || k < 1) return OR_BAD_ARG;
+    for (int b = 0; b < B; b++)
+        if (seq_lens[b] > L_max || visible(seq_lens[b], Q, 0) < 1) return OR_BAD_ARG;
+    const int G = Hq / Hkv;
+    const long units = (long)B * Q;
+    int status = OR_OK;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+#pragma omp parallel
+    {
+        scored_pos *sp = (scored_pos *)malloc(sizeof(scored_pos) * (size_t)L_max);
+        scored_pos *kept = (scored_pos *)malloc(sizeof(scored_pos) * (size_t)L_max);
+        double *s = (double *)malloc(sizeof(double) * (size_t)L_max);
+        int32_t *sel = (int32_t *)malloc(sizeof(int32_t) * 2 * (size_t)L_max);  /* kept positions + scratch */
+        if (!sp || !kept || !s || !sel) {
+#pragma omp atomic write
+            status = OR_NO_MEMORY;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (long u = 0; u < units; u++) {
+            if (!sp || !kept || !s || !sel) continue;
+            int qpos = (int)(u % Q), b = (int)(u / Q);
+            int vis = visible(seq_lens[b], Q, qpos);
+            /* indexer scores of every visible token */
+            for (int i = 0; i < vis; i++) {
+                double acc = 0.0;
+                for (int j = 0; j < H_I; j++) {
+                    double dot = 0.0;
+                    size_t qo = ((size_t)u * H_I + j) * d_I, ko = ((size_t)b * L_max + i) * d_I;
+                    for (int c = 0; c < d_I; c++) dot += load_elem(q_idx, dtype, qo + c) * load_elem(k_idx, dtype, ko + c);
+                    acc += (double)w_idx[(size_t)u * H_I + j] * (dot > 0.0 ? dot : 0.0);
+                }
+                sp[i].s = acc;
+                sp[i].i = i;
+            }
+            qsort(sp, (size_t)vis, sizeof(scored_pos), cmp_score_desc);
+            int kk = k < vis ? k : vis;
+            if (kth_index) kth_index[u] = sp[kk - 1].s;
+            for (int j = 0; j < kk; j++) sel[j] = sp[j].i;
+            qsort(sel, (size_t)kk, sizeof(int32_t), cmp_int_asc);
+            int32_t *ir = idx + (size_t)u * k;
+            for (int j = 0; j < k; j++) ir[j] = j < kk ? sel[j] : -1;
+            /* every head attends over the kept tokens with its exact scores */
+            for (int h = 0; h < Hq; h++) {
+                int kvh = h / G;
+                oracle_row_scores(B, Q, Hq, Hkv, d, L_max, dtype, scale, q, k_cache, seq_lens, b, qpos, h, s);
+                for (int j = 0; j < kk; j++) {
+                    kept[j].s = s[sel[j]];
+                    kept[j].i = sel[j];
+                }
+                qsort(kept, (size_t)kk, sizeof(scored_pos), cmp_score_desc);
+                size_t voff = ((size_t)b * Hkv + kvh) * (size_t)L_max * d;
+                size_t r = (size_t)u * Hq + h;
+                attend_prefix(kept, kk, kk, v_cache, dtype, voff, d, out + r * d, NULL, sel + kk, 0, sel + kk);
+            }
+        }
+        free(sp);
+        free(kept);
+        free(s);
+        free(sel);
+    }
+    return status;
+}

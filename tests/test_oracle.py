@@ -461,3 +461,39 @@ def test_hisa_brute_force(bs, top, k):
             np.testing.assert_allclose(r["out"][b, 0, h], want, rtol=1e-12, atol=1e-12)
             pc = torch.softmax(torch.from_numpy(sc), dim=0).numpy()
             assert abs(r["tail"][b, 0, h] - (1.0 - pc[order[:kk]].sum())) < 1e-12
+
+
+# ----------------------------------------------------------------------------- lightning indexer
+
+def _torch_index_scores(w, q_idx, w_idx, k_idx):
+    """Sum_j w_j ReLU(<q_idx_j, k_idx_i>) in fp64 via torch, [B, Q, L] (-inf where not visible)."""
+    dots = torch.einsum("bqjc,blc->bqjl", _f64(q_idx), _f64(torch.nan_to_num(k_idx.float())))
+    s = (w_idx.double()[..., None] * torch.relu(dots)).sum(2)
+    return s.masked_fill(~_visible_mask(w)[:, 0], -math.inf).numpy()
+
+
+@pytest.mark.parametrize("Q,H_I,d_I,k", [(1, 4, 64, 40), (3, 8, 32, 100), (2, 1, 128, 7)])
+def test_indexer_selection_and_attention_brute_force(Q, H_I, d_I, k):
+    w = workloads.make_workload(2, Q, 8, 2, 300, dtype="bf16", seq_lens=[300, 140], seed=81)
+    qi, wi, ki = workloads.make_indexer_inputs(w, H_I, d_I)
+    r = oracle.indexer_attn(w, qi, wi, ki, k)
+    I = _torch_index_scores(w, qi, wi, ki)
+    s = torch_scores(w)
+    for b in range(2):
+        for qp in range(Q):
+            vis = int(w.seq_lens[b]) - Q + qp + 1
+            sel = lexsort_topk(I[b, qp], k)
+            got = r["idx"][b, qp]
+            assert np.array_equal(got[:len(sel)], sel) and np.all(got[len(sel):] == -1)
+            for h in range(8):
+                p = torch.softmax(torch.from_numpy(s[b, qp, h, sel]), dim=0).numpy()
+                want = (p[:, None] * _f64(w.v_cache[b, h // 4, sel]).numpy()).sum(0)
+                np.testing.assert_allclose(r["out"][b, qp, h], want, rtol=1e-12, atol=1e-12)
+            assert vis >= 1
+
+
+def test_indexer_keeping_every_token_is_dense_attention():
+    w = workloads.make_workload(2, 2, 8, 4, 120, dtype="f32", seq_lens=[120, 33], seed=82)
+    qi, wi, ki = workloads.make_indexer_inputs(w, 4, 64)
+    r = oracle.indexer_attn(w, qi, wi, ki, 120)
+    np.testing.assert_allclose(r["out"], dense_sdpa(w), rtol=1e-12, atol=1e-12)

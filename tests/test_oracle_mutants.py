@@ -37,6 +37,9 @@ MUTANTS = {
                                    "for (int j = 0; j < nk; j++) kept[j] = j;\n            qsort(kept, (size_t)nk"),
     "hisa_candidates_all_blocks": ("            for (int j = 0; j < nk; j++) {\n                int lo = kept[j] * block_size, hi = lo + block_size;\n                if (hi > Lb) hi = Lb;\n                for (int i = lo; i < hi; i++) {\n                    sp[nc]",
                                    "            for (int j = 0; j < nblk; j++) {\n                int lo = j * block_size, hi = lo + block_size;\n                if (hi > Lb) hi = Lb;\n                for (int i = lo; i < hi; i++) {\n                    sp[nc]"),
+    "indexer_relu_dropped": ("(dot > 0.0 ? dot : 0.0)", "dot"),
+    "indexer_weights_ignored": ("acc += (double)w_idx[(size_t)u * H_I + j] * (dot > 0.0 ? dot : 0.0);",
+                                "acc += (dot > 0.0 ? dot : 0.0);"),
     "current_block_not_forced": ("kept[nk] = nblk - 1; /* the current block */",
                                  "kept[nk] = nk < nblk - 1 ? sp[nk].i : nblk - 1;"),
 }

@@ -36,7 +36,7 @@ import numpy as np
 import torch
 
 # stream ids inside a seed
-_T_Q, _T_K, _T_V, _T_KMEAN, _T_PLANT_POS, _T_PLANT_NOISE, _T_SEQ = range(7)
+_T_Q, _T_K, _T_V, _T_KMEAN, _T_PLANT_POS, _T_PLANT_NOISE, _T_SEQ, _T_IQ, _T_IW, _T_IK = range(10)
 
 
 @dataclass
@@ -217,3 +217,23 @@ def config_workload(cfg_id: int, seed: Optional[int] = None, plant_scale: Option
     if seed is None:
         seed = 1000 + cfg_id
     return make_workload(seed=seed, **spec)
+
+
+def make_indexer_inputs(w: "Workload", H_I: int = 16, d_I: int = 128, seed: Optional[int] = None):
+    """Synthetic lightning-indexer inputs for workload ``w``: projected indexer
+    queries q_idx [B, Q, H_I, d_I] and keys k_idx [B, L_max, d_I] (N(0, 1),
+    rounded to the cache dtype; keys past a sequence's end NaN) and head
+    weights w_idx [B, Q, H_I] (uniform on [0, 1), fp32).  No trained weights
+    exist here: the inputs have the shapes, not the statistics, of a trained
+    indexer."""
+    seed = w.seed if seed is None else seed
+    qi = np.stack([_normal(seed, (_T_IQ, b), w.Q * H_I * d_I).reshape(w.Q, H_I, d_I) for b in range(w.B)])
+    wi = np.stack([_rng(seed, _T_IW, b).random((w.Q, H_I), dtype=np.float32) for b in range(w.B)])
+    ki = np.stack([_normal(seed, (_T_IK, b), w.L_max * d_I).reshape(w.L_max, d_I) for b in range(w.B)])
+    q_idx = _to_dtype(np.ascontiguousarray(qi), w.dtype)
+    k_idx = _to_dtype(np.ascontiguousarray(ki), w.dtype)
+    for b in range(w.B):
+        Lb = int(w.seq_lens[b])
+        if Lb < w.L_max:
+            k_idx[b, Lb:] = float("nan")
+    return q_idx, torch.from_numpy(np.ascontiguousarray(wi)), k_idx
