@@ -28,4 +28,5 @@ from ._binding import (  # noqa: F401
     topk_block_attn_decode,
     topk_block_pool_keys,
     topk_hisa_attn_decode,
+    topk_indexer_attn_decode,
 )

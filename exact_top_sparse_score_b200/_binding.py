@@ -64,6 +64,11 @@ def load_library() -> ctypes.CDLL:
         lib.topk_hisa_attn_decode.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp,
                                               _vp, _vp, _sz, _vp]
         lib.topk_hisa_attn_decode.restype = ctypes.c_int
+        lib.topk_indexer_attn_workspace_size.argtypes = [_shape_p, _i32, _i32, _i32]
+        lib.topk_indexer_attn_workspace_size.restype = _sz
+        lib.topk_indexer_attn_decode.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _i32,
+                                                 _vp, _vp, _vp, _sz, _vp]
+        lib.topk_indexer_attn_decode.restype = ctypes.c_int
         lib.topk_attn_static_workspace_capacity.argtypes = []
         lib.topk_attn_static_workspace_capacity.restype = _sz
         lib.topk_attn_decode_static.argtypes = [_shape_p, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp]
@@ -446,3 +451,47 @@ def topk_hisa_attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch
     if rc:
         raise TopkAttnError("topk_hisa_attn_decode", rc)
     return out, idx, tail_mass, block_idx
+
+
+def topk_indexer_attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, q_idx: torch.Tensor,
+                             w_idx: torch.Tensor, k_idx: torch.Tensor, seq_lens: torch.Tensor, k: int, *,
+                             scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                             idx: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                             stream=None):
+    """Lightning-indexer token selection, then exact attention per head.
+
+    Returns (out fp32 [B,Q,Hq,d], idx int32 [B,Q,k])."""
+    lib = load_library()
+    shape = make_shape(q, k_cache, scale)
+    B, Q, Hq, d = q.shape
+    if q_idx.dim() != 4 or tuple(q_idx.shape[:2]) != (B, Q):
+        raise ValueError("q_idx must be [B,Q,H_I,d_I]")
+    H_I, d_I = q_idx.shape[2], q_idx.shape[3]
+    if tuple(k_idx.shape) != (B, k_cache.shape[2], d_I) or tuple(w_idx.shape) != (B, Q, H_I):
+        raise ValueError("k_idx must be [B,L_max,d_I] and w_idx [B,Q,H_I]")
+    if q_idx.dtype != k_cache.dtype or k_idx.dtype != k_cache.dtype or w_idx.dtype != torch.float32:
+        raise TypeError("q_idx and k_idx take the cache dtype, w_idx fp32")
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, Q, Hq, d), dtype=torch.float32, device=dev)
+    if idx is None:
+        idx = torch.empty((B, Q, k), dtype=torch.int32, device=dev)
+    if seq_lens.dtype != torch.int32 or tuple(seq_lens.shape) != (B,):
+        raise TypeError("seq_lens must be int32 [B]")
+    _check_out("out", out, torch.float32, (B, Q, Hq, d))
+    _check_out("idx", idx, torch.int32, (B, Q, k))
+    if workspace is not None and workspace.dtype != torch.uint8:
+        raise TypeError("workspace must be a uint8 tensor")
+    _check_cuda(q=q, k_cache=k_cache, v_cache=v_cache, q_idx=q_idx, w_idx=w_idx, k_idx=k_idx, seq_lens=seq_lens,
+                out=out, idx=idx, workspace=workspace)
+    nbytes = int(lib.topk_indexer_attn_workspace_size(ctypes.byref(shape), H_I, d_I, k))
+    if nbytes == 0:
+        raise TopkAttnError("topk_indexer_attn_workspace_size", 2)
+    sh = _stream(stream)
+    ws = _workspace(nbytes, dev, workspace, sh)
+    rc = lib.topk_indexer_attn_decode(ctypes.byref(shape), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                      q_idx.data_ptr(), w_idx.data_ptr(), k_idx.data_ptr(), H_I, d_I,
+                                      seq_lens.data_ptr(), k, out.data_ptr(), idx.data_ptr(), ws.data_ptr(), nbytes, sh)
+    if rc:
+        raise TopkAttnError("topk_indexer_attn_decode", rc)
+    return out, idx

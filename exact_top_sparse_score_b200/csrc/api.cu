@@ -188,6 +188,48 @@ HisaLayout hisa_layout(const tka_shape *s, int block_size, int top_blocks, int k
     return L;
 }
 
+// Workspace of topk_indexer_attn_decode (256-byte aligned regions):
+//   iscores fp32 [B*Q, ld], weights fp32 [B*Q, k], stats float4 [B*Q],
+//   sel counters uint32 [B*Q], part_ml float4 [B*Q*Hq, k/64],
+//   part_acc fp32 [B*Q*Hq, k/64, d], attn counters uint32 [B*Q*Hkv]
+struct IndexerLayout {
+    size_t iscores, weights, stats, sel_counters, part_ml, part_acc, attn_counters, total;
+    int ld, max_splits;
+};
+
+IndexerLayout indexer_layout(const tka_shape *s, int k) {
+    IndexerLayout L;
+    const size_t units = (size_t)s->B * s->Q, rows = units * s->Hq;
+    L.ld = (int)align_up((size_t)s->L_max, 64);
+    L.max_splits = (k + kMinKeysPerSplit - 1) / kMinKeysPerSplit;
+    size_t off = 0;
+    L.iscores = off;
+    off = align_up(off + units * L.ld * sizeof(float), 256);
+    L.weights = off;
+    off = align_up(off + units * (size_t)k * sizeof(float), 256);
+    L.stats = off;
+    off = align_up(off + units * sizeof(float4), 256);
+    L.sel_counters = off;
+    off = align_up(off + units * sizeof(unsigned), 256);
+    L.part_ml = off;
+    off = align_up(off + rows * L.max_splits * sizeof(float4), 256);
+    L.part_acc = off;
+    off = align_up(off + rows * L.max_splits * kHeadDim * sizeof(float), 256);
+    L.attn_counters = off;
+    off = align_up(off + units * s->Hkv * sizeof(unsigned), 256);
+    L.total = off;
+    return L;
+}
+
+tka_status check_indexer_args(const tka_shape *s, int H_I, int d_I, int k) {
+    tka_status st = check_shape(s);
+    if (st != TKA_OK) return st;
+    if (H_I < 1 || d_I < 1 || k < 1) return TKA_ERR_INVALID_ARG;
+    if (!indexer_supported(s->Hq / s->Hkv, d_I) || H_I > 64 || s->Q * H_I > 256 || k > kMaxK)
+        return TKA_ERR_UNSUPPORTED;
+    return TKA_OK;
+}
+
 tka_status check_hisa_args(const tka_shape *s, int block_size, int top_blocks, int k) {
     tka_status st = check_shape(s);
     if (st != TKA_OK) return st;
@@ -556,6 +598,77 @@ tka_status topk_hisa_attn_decode(const tka_shape *shape, const void *q, const vo
     gp.per_split = (k + splits - 1) / splits;
     gp.splits = (k + gp.per_split - 1) / gp.per_split;
     if (launch_gather(gp, s) != cudaSuccess) return TKA_ERR_CUDA;
+    return TKA_OK;
+}
+
+size_t topk_indexer_attn_workspace_size(const tka_shape *shape, int32_t H_I, int32_t d_I, int32_t k) {
+    if (check_indexer_args(shape, H_I, d_I, k) != TKA_OK) return 0;
+    return indexer_layout(shape, k).total;
+}
+
+tka_status topk_indexer_attn_decode(const tka_shape *shape, const void *q, const void *k_cache, const void *v_cache,
+                                    const void *q_idx, const float *w_idx, const void *k_idx, int32_t H_I,
+                                    int32_t d_I, const int32_t *seq_lens, int32_t k, float *out, int32_t *idx,
+                                    void *workspace, size_t workspace_bytes, tka_stream_t stream) {
+    tka_status st = check_indexer_args(shape, H_I, d_I, k);
+    if (st != TKA_OK) return st;
+    if (!q || !k_cache || !v_cache || !q_idx || !w_idx || !k_idx || !seq_lens || !out || !idx)
+        return TKA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(q_idx, 16) ||
+        !aligned(k_idx, 16) || !aligned(w_idx, 4) || !aligned(out, 16) || !aligned(idx, 4) || !aligned(seq_lens, 4))
+        return TKA_ERR_INVALID_ARG;
+    const IndexerLayout L = indexer_layout(shape, k);
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < L.total) return TKA_ERR_WORKSPACE;
+    DeviceInfo *dev = nullptr;
+    if (device_info(&dev) != cudaSuccess) return TKA_ERR_CUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    char *ws = static_cast<char *>(workspace);
+    const int G = shape->Hq / shape->Hkv;
+    const int units = shape->B * shape->Q;
+
+    // 1. indexer scores of every visible token, per query position
+    IndexerScoreParams ip;
+    ip.status = dev->status;
+    ip.q_idx = q_idx; ip.w_idx = w_idx; ip.k_idx = k_idx;
+    ip.seq_lens = seq_lens;
+    ip.B = shape->B; ip.Q = shape->Q; ip.Hkv = shape->Hkv; ip.L_max = shape->L_max;
+    ip.H_I = H_I; ip.d_I = d_I; ip.ld = L.ld; ip.dtype = shape->dtype;
+    ip.scores = reinterpret_cast<float *>(ws + L.iscores);
+    ip.attn_counters = reinterpret_cast<unsigned *>(ws + L.attn_counters);
+    if (launch_indexer_scores(ip, dev->num_sms, s) != cudaSuccess) return TKA_ERR_CUDA;
+
+    // 2. the top k tokens of each query position (one row per position)
+    SelectParams se;
+    se.status = dev->status;
+    se.scores = ip.scores;
+    se.seq_lens = seq_lens;
+    se.B = shape->B; se.Q = shape->Q; se.Hq = 1; se.L_max = shape->L_max; se.ld = L.ld; se.k = k;
+    se.idx = idx;
+    se.w = reinterpret_cast<float *>(ws + L.weights);
+    se.stats = reinterpret_cast<float4 *>(ws + L.stats);
+    se.tail = nullptr;
+    se.counters = reinterpret_cast<unsigned *>(ws + L.sel_counters);
+    if (launch_select(se, s) != cudaSuccess) return TKA_ERR_CUDA;
+
+    // 3. every head attends over its position's kept tokens with exact scores
+    IndexerAttnParams ap;
+    ap.status = dev->status;
+    ap.q = q; ap.kc = k_cache; ap.vc = v_cache;
+    ap.seq_lens = seq_lens;
+    ap.idx = idx;
+    ap.B = shape->B; ap.Q = shape->Q; ap.Hq = shape->Hq; ap.Hkv = shape->Hkv; ap.G = G;
+    ap.L_max = shape->L_max; ap.k = k; ap.dtype = shape->dtype;
+    ap.scale = resolve_scale(shape);
+    ap.part_ml = reinterpret_cast<float4 *>(ws + L.part_ml);
+    ap.part_acc = reinterpret_cast<float *>(ws + L.part_acc);
+    ap.counters = ip.attn_counters;
+    ap.out = out;
+    int splits = (dev->num_sms * 8) / (units * shape->Hkv);
+    if (splits > L.max_splits) splits = L.max_splits;
+    if (splits < 1) splits = 1;
+    ap.per_split = (k + splits - 1) / splits;
+    ap.splits = (k + ap.per_split - 1) / ap.per_split;
+    if (launch_indexer_attn(ap, s) != cudaSuccess) return TKA_ERR_CUDA;
     return TKA_OK;
 }
 

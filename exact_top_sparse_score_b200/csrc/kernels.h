@@ -92,6 +92,31 @@ struct CertifyParams {
     int32_t *k_used;          // [rows]
 };
 
+struct IndexerScoreParams {
+    unsigned *status;         // device status word (TKA_DEV_* bits)
+    const void *q_idx;        // [B, Q, H_I, d_I] indexer queries
+    const float *w_idx;       // [B, Q, H_I] indexer head weights
+    const void *k_idx;        // [B, L_max, d_I] indexer keys
+    const int32_t *seq_lens;
+    int B, Q, Hkv, L_max, H_I, d_I, ld, dtype;
+    float *scores;            // [B*Q, ld] indexer scores
+    unsigned *attn_counters;  // [B*Q*Hkv], zeroed here for the attention step
+};
+
+struct IndexerAttnParams {
+    unsigned *status;         // device status word (TKA_DEV_* bits)
+    const void *q, *kc, *vc;  // q [B, Q, Hq, 128]; caches [B, Hkv, L_max, 128]
+    const int32_t *seq_lens;
+    const int32_t *idx;       // [B*Q, k] kept positions, ascending
+    int B, Q, Hq, Hkv, G, L_max, k, dtype;
+    float scale;
+    float4 *part_ml;          // [B*Q*Hq, splits] {m, l}
+    float *part_acc;          // [B*Q*Hq, splits, 128]
+    unsigned *counters;       // [B*Q*Hkv]
+    float *out;               // [B*Q*Hq, 128]
+    int splits, per_split;
+};
+
 struct BlockPoolParams {
     unsigned *status;         // device status word (TKA_DEV_* bits)
     const void *k;
@@ -149,6 +174,9 @@ cudaError_t launch_select(const SelectParams &p, cudaStream_t stream);
 size_t select_smem_bytes(int k);
 cudaError_t launch_gather(const GatherParams &p, cudaStream_t stream);
 cudaError_t launch_certify(const CertifyParams &p, cudaStream_t stream);
+bool indexer_supported(int G, int d_I);
+cudaError_t launch_indexer_scores(const IndexerScoreParams &p, int num_sms, cudaStream_t stream);
+cudaError_t launch_indexer_attn(const IndexerAttnParams &p, cudaStream_t stream);
 cudaError_t launch_block_pool(const BlockPoolParams &p, cudaStream_t stream);
 cudaError_t launch_block_select(const BlockSelectParams &p, cudaStream_t stream);
 cudaError_t launch_hisa_scores(const HisaScoreParams &p, cudaStream_t stream);

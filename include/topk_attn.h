@@ -195,6 +195,26 @@ tka_status topk_block_attn_decode(const tka_shape *shape, const void *q, const v
                                   float *out, int32_t *block_idx, void *workspace,
                                   size_t workspace_bytes, tka_stream_t stream);
 
+/* Lightning-indexer token selection ("Sparse Attention Landscape", section
+ * "Token Sparse Attention", DeepSeek Sparse Attention): per query position,
+ *   I_i = sum_j w_idx[j] * ReLU(<q_idx[j], k_idx[i]>)   (j < H_I)
+ * over its visible tokens; the top k tokens by I (ties to the lower position)
+ * are kept for the position, shared by all its Hq heads, and every head
+ * attends over them with its exact scores: out = softmax(scale * q.K) V over
+ * the kept tokens.  No tail mass: the method scores the tokens with I only.
+ *   q_idx   [B, Q, H_I, d_I], k_idx [B, L_max, d_I]: the indexer's projected
+ *           queries and keys, in the cache dtype; w_idx fp32 [B, Q, H_I].
+ *   idx     int32 [B, Q, k] ascending, -1 padded.
+ *   workspace topk_indexer_attn_workspace_size(shape, H_I, d_I, k) bytes.
+ * Supported: d_I in {64, 128}, 1 <= H_I <= 64, Q * H_I <= 256,
+ * G = Hq / Hkv in {1, 2, 4, 8, 16}, 1 <= k <= 8192. */
+size_t topk_indexer_attn_workspace_size(const tka_shape *shape, int32_t H_I, int32_t d_I, int32_t k);
+tka_status topk_indexer_attn_decode(const tka_shape *shape, const void *q, const void *k_cache,
+                                    const void *v_cache, const void *q_idx, const float *w_idx,
+                                    const void *k_idx, int32_t H_I, int32_t d_I, const int32_t *seq_lens,
+                                    int32_t k, float *out, int32_t *idx, void *workspace,
+                                    size_t workspace_bytes, tka_stream_t stream);
+
 /* Hierarchical block -> token Top-k ("Sparse Attention Landscape", section
  * "Hierarchical Sparse Attention"), one query per sequence (shape->Q == 1).
  * With nblk = ceil(seq_lens[b] / block_size): every block j < nblk scores

@@ -240,3 +240,55 @@ def check_hisa(w, block_size, top_blocks, k, out, idx, tail, bidx, ref, scale=0.
             kept_mass = np.exp(s[gs] - s[cand].max()).sum() / e_all.sum()
             assert abs(tail[b, 0, h] - (1.0 - kept_mass)) <= TAIL_TOL, f"{where}: tail invalid"
     return n_band
+
+
+def index_scores_f64(w, q_idx, w_idx, k_idx):
+    """sum_j w_j ReLU(<q_idx_j, k_idx_i>) in fp64 [B, Q, L_max] (positions past a sequence's end: -inf)."""
+    dots = torch.einsum("bqjc,blc->bqjl", q_idx.double(), torch.nan_to_num(k_idx.float()).double())
+    s = (w_idx.double()[..., None] * torch.relu(dots)).sum(2).numpy()
+    for b in range(w.B):
+        for qp in range(w.Q):
+            s[b, qp, _vis(w, b, qp):] = -np.inf
+    return s
+
+
+def check_indexer(w, k, out, idx, ref, I, scale=0.0):
+    """Asserts parity of topk_indexer_attn_decode with oracle.indexer_attn output `ref`.
+
+    Kept tokens equal the oracle's except positions whose fp64 indexer score
+    lies within BAND (relative to its scale) of the oracle's k-th; out matches
+    the oracle where the sets agree, else an fp64 evaluation over the GPU's
+    own set.  I: fp64 indexer scores [B, Q, L_max].  Returns the number of
+    positions checked through the band."""
+    out = out.detach().cpu().double().numpy()
+    idx = idx.detach().cpu().numpy()
+    atol, rtol = out_tol(w.dtype)
+    n_band = 0
+    for b in range(w.B):
+        for qp in range(w.Q):
+            where = f"position (b={b}, q={qp})"
+            vis = _vis(w, b, qp)
+            kk = min(k, vis)
+            g = idx[b, qp]
+            assert np.all(g[kk:] == -1), f"{where}: padding"
+            gs = g[:kk]
+            assert np.all(gs >= 0) and np.all(gs < vis) and np.all(np.diff(gs) > 0), f"{where}: kept list"
+            o = ref["idx"][b, qp, :kk]
+            same = np.array_equal(gs, o)
+            if not same:
+                n_band += 1
+                kth = ref["kth"][b, qp]
+                tol = BAND * max(1.0, abs(kth))
+                diff = np.setxor1d(gs, o)
+                assert np.all(np.abs(I[b, qp, diff] - kth) <= tol), f"{where}: set differs outside the tie band"
+            for h in range(w.Hq):
+                if same:
+                    ok = _close(out[b, qp, h], ref["out"][b, qp, h], atol, rtol)
+                    assert ok.all(), f"{where}, head {h}: out"
+                else:
+                    s = oracle.row_scores(w, b, qp, h, scale)
+                    e = np.exp(s[gs] - s[gs].max())
+                    V = w.v_cache[b, h // w.G].double().numpy()[gs]
+                    assert _close(out[b, qp, h], (e[:, None] * V).sum(0) / e.sum(), atol, rtol).all(), \
+                        f"{where}, head {h}: out invalid for its own set"
+    return n_band

@@ -33,7 +33,8 @@ def test_header_declares_the_entry_points():
     for n in ["topk_attn_decode", "topk_attn_workspace_size", "topk_block_attn_decode",
               "topk_block_pool_keys", "topk_block_attn_workspace_size", "topk_attn_device_status",
               "topk_attn_status_string", "topk_attn_decode_certified",
-              "topk_attn_decode_paged", "topk_hisa_attn_decode", "topk_hisa_attn_workspace_size"]:
+              "topk_attn_decode_paged", "topk_hisa_attn_decode", "topk_hisa_attn_workspace_size",
+              "topk_indexer_attn_decode", "topk_indexer_attn_workspace_size"]:
         assert n in names
 
 
