@@ -57,6 +57,9 @@ def parse_args():
                     help="override the workload's batch size (smaller cases for profiling)")
     ap.add_argument("--paged", type=int, default=None, metavar="PAGE_SIZE",
                     help="lay the cache out as shuffled pages of PAGE_SIZE positions (block tables)")
+    ap.add_argument("--indexer", type=str, default=None, metavar="H_I,D_I",
+                    help="lightning-indexer token selection with H_I indexer heads of D_I dims "
+                         "(synthetic indexer inputs)")
     ap.add_argument("--hisa", type=str, default=None, metavar="BLOCK_SIZE,TOP_BLOCKS",
                     help="hierarchical block -> token Top-k: score only the tokens of the best TOP_BLOCKS "
                          "blocks of BLOCK_SIZE (one-query workloads)")
@@ -258,6 +261,10 @@ def run_ours(args, world, rank, local):
     certified = args.certified_eps is not None and not block
     paged = args.paged is not None and not block and not certified
     hisa = args.hisa is not None and not block and not certified and not paged
+    indexer = args.indexer is not None and not block and not certified and not paged and not hisa
+    if indexer:
+        i_h, i_d = (int(x) for x in args.indexer.split(","))
+        i_q, i_w, i_k = (t.to(dev) for t in workloads.make_indexer_inputs(w, i_h, i_d))
     if hisa:
         h_bs, h_top = (int(x) for x in args.hisa.split(","))
     k = w.k
@@ -293,6 +300,18 @@ def run_ours(args, world, rank, local):
                     events[0].record()
                 tka.topk_attn_decode_certified(qq, kc, vc, lens, args.certified_eps, k, out=out, idx=idx,
                                                tail_mass=tail, k_used=k_used, workspace=ws)
+                if events:
+                    events[3].record()
+        elif indexer:
+            i_idx = torch.empty((w.B, w.Q, k), dtype=torch.int32, device=dev)
+            ws = torch.empty(tka._binding.load_library().topk_indexer_attn_workspace_size(
+                make_shape(q, kc), i_h, i_d, k), dtype=torch.uint8, device=dev)
+            launches_per_step = 3  # indexer_scores, select, indexer_attn
+
+            def step(events=None, qq=q):
+                if events:
+                    events[0].record()
+                tka.topk_indexer_attn_decode(qq, kc, vc, i_q, i_w, i_k, lens, k, out=out, idx=i_idx, workspace=ws)
                 if events:
                     events[3].record()
         elif hisa:
@@ -356,7 +375,7 @@ def run_ours(args, world, rank, local):
     if world > 1:
         torch.distributed.barrier()
     step_ms = [e[0].elapsed_time(e[3]) for e in evs]
-    stage_ms = None if block or certified or paged or hisa else [[e[j].elapsed_time(e[j + 1]) for e in evs] for j in range(3)]
+    stage_ms = None if block or certified or paged or hisa or indexer else [[e[j].elapsed_time(e[j + 1]) for e in evs] for j in range(3)]
     total_ms = sum(step_ms)
 
     e2e_ms = None
@@ -368,7 +387,8 @@ def run_ours(args, world, rank, local):
         lens_host = w.seq_lens.pin_memory()
         q_step = torch.empty_like(q)
         lens_step = torch.empty_like(lens)
-        outs = [out, bidx] if block else ([out, idx, tail, k_used] if certified else [out, idx, tail])
+        outs = [out, bidx] if block else ([out, idx, tail, k_used] if certified else
+                                          ([out, i_idx] if indexer else [out, idx, tail]))
         hosts = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
         h2d = q_host.numel() * q_host.element_size() + lens_host.numel() * 4
         d2h = sum(t.numel() * t.element_size() for t in outs)
@@ -390,6 +410,9 @@ def run_ours(args, world, rank, local):
             elif hisa:
                 tka.topk_hisa_attn_decode(q_step, kc, vc, h_bk, lens_step, h_bs, h_top, k, out=out, idx=idx,
                                           tail_mass=tail, block_idx=h_bidx, workspace=ws)
+            elif indexer:
+                tka.topk_indexer_attn_decode(q_step, kc, vc, i_q, i_w, i_k, lens_step, k, out=out, idx=i_idx,
+                                             workspace=ws)
             else:
                 tka.topk_attn_decode(q_step, kc, vc, lens_step, k, out=out, idx=idx, tail_mass=tail, workspace=ws)
             for h, t in zip(hosts, outs):
@@ -433,6 +456,7 @@ def run_ours(args, world, rank, local):
             **({"certified_eps": args.certified_eps, "k_max": k} if certified else {}),
             **({"page_size": args.paged, "pages": "shuffled pool, block tables"} if paged else {}),
             **({"hisa_block_size": h_bs, "hisa_top_blocks": h_top} if hisa else {}),
+            **({"indexer_heads": i_h, "indexer_dims": i_d, "indexer_inputs": "synthetic"} if indexer else {}),
         },
         "us_per_step": ms * 1e3,
         "tokens_per_s": world * w.B * w.Q / (ms / 1e3),
@@ -443,6 +467,21 @@ def run_ours(args, world, rank, local):
         "gpu_launches": launches_per_step * K,
         "clocks": clocks.summary(),
     }
+    if indexer:
+        # algorithmic bytes: index keys once per sequence + the k kept K and V rows per kv-head + q/out/idx
+        row = w.d * elem_bytes(w)
+        kept = sum(min(k, visible(w, b, qp)) for b in range(w.B) for qp in range(w.Q))
+        alg = (k_bytes(w) // (w.Hkv * w.d) * i_d) + kept * w.Hkv * 2 * row + rows * w.d * (elem_bytes(w) + 4) \
+            + w.B * w.Q * k * 4
+        res["alg_bytes_per_step"] = alg
+        res["alg_gbs"] = alg / (ms / 1e3) / 1e9
+        res["alg_frac_of_spec_8tbs"] = res["alg_gbs"] / SPEC_HBM_GBS
+        res["alg_frac_of_measured_hbm"] = res["alg_gbs"] / peak
+        res["roofline"] = {"kernel": "whole step (indexer scores + select + attention)", "bound": "hbm",
+                           "achieved": res["alg_gbs"], "peak": peak,
+                           "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
+                           else "fallback 6.65 TB/s", "unit": "GB/s", "frac": res["alg_gbs"] / peak,
+                           "traffic": None, "alg_bytes_per_launch": alg}
     if hisa:
         # algorithmic bytes: block keys + the kept blocks' K rows + the k kept V rows + q/out/idx
         row = w.d * elem_bytes(w)

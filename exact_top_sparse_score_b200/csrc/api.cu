@@ -193,11 +193,17 @@ HisaLayout hisa_layout(const tka_shape *s, int block_size, int top_blocks, int k
 //   sel counters uint32 [B*Q], part_ml float4 [B*Q*Hq, k/64],
 //   part_acc fp32 [B*Q*Hq, k/64, d], attn counters uint32 [B*Q*Hkv]
 struct IndexerLayout {
-    size_t iscores, weights, stats, sel_counters, part_ml, part_acc, attn_counters, total;
+    size_t iscores, weights, stats, sel_counters, part_ml, part_acc, attn_counters, raw, total;
     int ld, max_splits;
 };
 
-IndexerLayout indexer_layout(const tka_shape *s, int k) {
+// tensor-core indexer dots: bf16 128-dim index keys, all heads of a sequence as query rows of one kv-head
+bool indexer_tc(const tka_shape *s, int H_I, int d_I) {
+    return d_I == 128 && s->dtype == TKA_BF16 && score_tc_supported(TKA_BF16, s->Q * H_I) &&
+           (long long)s->B * s->L_max < (1ll << 31);
+}
+
+IndexerLayout indexer_layout(const tka_shape *s, int k, int H_I, int d_I) {
     IndexerLayout L;
     const size_t units = (size_t)s->B * s->Q, rows = units * s->Hq;
     L.ld = (int)align_up((size_t)s->L_max, 64);
@@ -217,6 +223,8 @@ IndexerLayout indexer_layout(const tka_shape *s, int k) {
     off = align_up(off + rows * L.max_splits * kHeadDim * sizeof(float), 256);
     L.attn_counters = off;
     off = align_up(off + units * s->Hkv * sizeof(unsigned), 256);
+    L.raw = off;  // per-head dots of the tensor-core path: fp32 [B*Q*H_I, ld]
+    if (indexer_tc(s, H_I, d_I)) off = align_up(off + units * H_I * (size_t)L.ld * sizeof(float), 256);
     L.total = off;
     return L;
 }
@@ -603,7 +611,7 @@ tka_status topk_hisa_attn_decode(const tka_shape *shape, const void *q, const vo
 
 size_t topk_indexer_attn_workspace_size(const tka_shape *shape, int32_t H_I, int32_t d_I, int32_t k) {
     if (check_indexer_args(shape, H_I, d_I, k) != TKA_OK) return 0;
-    return indexer_layout(shape, k).total;
+    return indexer_layout(shape, k, H_I, d_I).total;
 }
 
 tka_status topk_indexer_attn_decode(const tka_shape *shape, const void *q, const void *k_cache, const void *v_cache,
@@ -617,7 +625,7 @@ tka_status topk_indexer_attn_decode(const tka_shape *shape, const void *q, const
     if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(q_idx, 16) ||
         !aligned(k_idx, 16) || !aligned(w_idx, 4) || !aligned(out, 16) || !aligned(idx, 4) || !aligned(seq_lens, 4))
         return TKA_ERR_INVALID_ARG;
-    const IndexerLayout L = indexer_layout(shape, k);
+    const IndexerLayout L = indexer_layout(shape, k, H_I, d_I);
     if (!workspace || !aligned(workspace, 256) || workspace_bytes < L.total) return TKA_ERR_WORKSPACE;
     DeviceInfo *dev = nullptr;
     if (device_info(&dev) != cudaSuccess) return TKA_ERR_CUDA;
@@ -635,7 +643,19 @@ tka_status topk_indexer_attn_decode(const tka_shape *shape, const void *q, const
     ip.H_I = H_I; ip.d_I = d_I; ip.ld = L.ld; ip.dtype = shape->dtype;
     ip.scores = reinterpret_cast<float *>(ws + L.iscores);
     ip.attn_counters = reinterpret_cast<unsigned *>(ws + L.attn_counters);
-    if (launch_indexer_scores(ip, dev->num_sms, s) != cudaSuccess) return TKA_ERR_CUDA;
+    if (indexer_tc(shape, H_I, d_I)) {
+        ScoreTcParams tp;
+        tp.status = dev->status;
+        tp.seq_lens = seq_lens;
+        tp.scores = reinterpret_cast<float *>(ws + L.raw);
+        tp.B = shape->B; tp.Q = shape->Q; tp.Hq = H_I; tp.Hkv = 1; tp.G = H_I;
+        tp.L_max = shape->L_max; tp.ld = L.ld; tp.NQ = shape->Q * H_I;
+        tp.scale = 1.f;
+        if (launch_score_tc(tp, q_idx, k_idx, dev->num_sms, s, ScoreTcHook{}) != cudaSuccess) return TKA_ERR_CUDA;
+        if (launch_indexer_combine(ip, tp.scores, s) != cudaSuccess) return TKA_ERR_CUDA;
+    } else if (launch_indexer_scores(ip, dev->num_sms, s) != cudaSuccess) {
+        return TKA_ERR_CUDA;
+    }
 
     // 2. the top k tokens of each query position (one row per position)
     SelectParams se;

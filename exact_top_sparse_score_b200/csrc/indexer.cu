@@ -9,7 +9,10 @@
 //   indexer_scores  grid (key chunks, b): a quad of lanes per index key, each
 //                   lane a quarter of the dims; every (query position, indexer
 //                   head) dot is reduced in the quad, ReLU'd, weighted and
-//                   summed; one score per (query position, key).
+//                   summed; one score per (query position, key).  With bf16
+//                   128-dim index keys the dots run on the tensor cores instead
+//                   (the score kernel with the indexer heads as query rows of
+//                   one kv-head) and indexer_combine forms the weighted sum.
 //   (the select step keeps the top k per query position)
 //   indexer_attn    grid (splits, b * Q * Hkv): a slice of the kept tokens for
 //                   the G heads of one kv-head; every K and V row is read once
@@ -93,6 +96,28 @@ __global__ void __launch_bounds__(128) indexer_scores(IndexerScoreParams p) {
             }
         }
     }
+}
+
+// I = sum_j w_j ReLU(raw_j) from the raw per-head dots the tensor-core scorer
+// wrote ([B*Q*H_I, ld], head-minor rows): grid (key chunks of 256, b * Q).
+__global__ void __launch_bounds__(256) indexer_combine(IndexerScoreParams p, const float *raw) {
+    __shared__ float ws[256];
+    const int bq = blockIdx.y, b = bq / p.Q, qpos = bq - b * p.Q;
+    const int seq_len = p.seq_lens[b];
+    if (!seq_len_ok(seq_len, p.Q, p.L_max)) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) raise_status(p.status, TKA_DEV_BAD_SEQ_LEN);
+        return;
+    }
+    if (blockIdx.x == 0 && qpos == 0)  // the attention step's tickets for this sequence's units
+        for (int u = threadIdx.x; u < p.Q * p.Hkv; u += blockDim.x) p.attn_counters[(size_t)b * p.Q * p.Hkv + u] = 0u;
+    for (int j = threadIdx.x; j < p.H_I; j += blockDim.x) ws[j] = p.w_idx[(size_t)bq * p.H_I + j];
+    __syncthreads();
+    const int key = blockIdx.x * 256 + threadIdx.x;
+    if (key >= visible_keys(seq_len, p.Q, qpos)) return;
+    const float *r = raw + (size_t)bq * p.H_I * p.ld + key;
+    float I = 0.f;
+    for (int j = 0; j < p.H_I; j++) I = fmaf(ws[j], fmaxf(__ldcg(r + (size_t)j * p.ld), 0.f), I);
+    p.scores[(size_t)bq * p.ld + key] = I;
 }
 
 constexpr int kAttnWarps = 4;
@@ -255,6 +280,12 @@ bool indexer_supported(int G, int d_I) { return (d_I == 64 || d_I == 128) && (G 
 
 cudaError_t launch_indexer_scores(const IndexerScoreParams &p, int num_sms, cudaStream_t stream) {
     return p.d_I == 64 ? launch_scores_di<64>(p, num_sms, stream) : launch_scores_di<128>(p, num_sms, stream);
+}
+
+cudaError_t launch_indexer_combine(const IndexerScoreParams &p, const float *raw, cudaStream_t stream) {
+    const dim3 grid((p.L_max + 255) / 256, p.B * p.Q);
+    indexer_combine<<<grid, 256, 0, stream>>>(p, raw);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_indexer_attn(const IndexerAttnParams &p, cudaStream_t stream) {

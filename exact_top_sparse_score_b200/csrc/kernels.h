@@ -177,6 +177,7 @@ cudaError_t launch_certify(const CertifyParams &p, cudaStream_t stream);
 bool indexer_supported(int G, int d_I);
 cudaError_t launch_indexer_scores(const IndexerScoreParams &p, int num_sms, cudaStream_t stream);
 cudaError_t launch_indexer_attn(const IndexerAttnParams &p, cudaStream_t stream);
+cudaError_t launch_indexer_combine(const IndexerScoreParams &p, const float *raw, cudaStream_t stream);
 cudaError_t launch_block_pool(const BlockPoolParams &p, cudaStream_t stream);
 cudaError_t launch_block_select(const BlockSelectParams &p, cudaStream_t stream);
 cudaError_t launch_hisa_scores(const HisaScoreParams &p, cudaStream_t stream);
