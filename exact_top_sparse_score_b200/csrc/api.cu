@@ -270,6 +270,140 @@ struct CertArgs {
     int32_t *k_used;
 };
 
+// Everything decode_impl resolved before the launches.
+struct DecodeArgs {
+    const tka_shape *shape;
+    const void *q, *k_cache, *v_cache;
+    const int32_t *seq_lens;
+    int k, G;
+    float *out, *tail;
+    int32_t *idx;
+    char *ws;
+    TokenLayout L;
+    DeviceInfo *dev;
+    const CertArgs *cert;
+    const PageTable *pages;
+    bool tc;
+};
+
+size_t elem_bytes(const tka_shape *s) { return s->dtype == TKA_BF16 ? 2 : 4; }
+
+// Score of sequences [b0, b1) on s (every per-sequence array offset to b0).
+tka_status launch_score_part(const DecodeArgs &a, int b0, int b1, cudaStream_t s, const tka_event_t *events) {
+    const tka_shape *sh = a.shape;
+    const size_t row0 = (size_t)b0 * sh->Q * sh->Hq, eb = elem_bytes(sh);
+    const char *q = static_cast<const char *>(a.q) + row0 * kHeadDim * eb;
+    const char *kc = static_cast<const char *>(a.k_cache);
+    PageTable pt;
+    if (a.pages) {
+        pt = *a.pages;
+        pt.table += (size_t)b0 * pt.max_pages;
+    } else {
+        kc += (size_t)b0 * sh->Hkv * sh->L_max * kHeadDim * eb;
+    }
+    float *scores = reinterpret_cast<float *>(a.ws + a.L.scores) + row0 * a.L.ld;
+    if (a.tc) {
+        ScoreTcParams tp;
+        tp.status = a.dev->status;
+        tp.seq_lens = a.seq_lens + b0;
+        tp.scores = scores;
+        tp.B = b1 - b0; tp.Q = sh->Q; tp.Hq = sh->Hq; tp.Hkv = sh->Hkv; tp.G = a.G;
+        tp.L_max = sh->L_max; tp.ld = a.L.ld; tp.NQ = sh->Q * a.G;
+        tp.scale = resolve_scale(sh);
+        tp.pages = pt;
+        RecordCtx rc{events, 0, s};
+        ScoreTcHook hook;
+        hook.fn = record_hook;
+        hook.ctx = &rc;
+        if (launch_score_tc(tp, q, kc, a.dev->num_sms, s, hook) != cudaSuccess) return TKA_ERR_CUDA;
+    } else {
+        if (record(events, 0, s) != cudaSuccess) return TKA_ERR_CUDA;
+        ScoreParams sp;
+        sp.status = a.dev->status;
+        sp.q = q;
+        sp.k = kc;
+        sp.seq_lens = a.seq_lens + b0;
+        sp.scores = scores;
+        sp.B = b1 - b0; sp.Q = sh->Q; sp.Hq = sh->Hq; sp.Hkv = sh->Hkv; sp.G = a.G;
+        sp.L_max = sh->L_max; sp.ld = a.L.ld; sp.dtype = sh->dtype;
+        sp.scale = resolve_scale(sh);
+        sp.pages = pt;
+        if (launch_score(sp, a.dev->num_sms, s) != cudaSuccess) return TKA_ERR_CUDA;
+    }
+    return TKA_OK;
+}
+
+// Select (k) -> [certify] -> gather of sequences [b0, b1) on s.
+tka_status launch_rest_part(const DecodeArgs &a, int b0, int b1, cudaStream_t s, int select_threads,
+                            const tka_event_t *events) {
+    const tka_shape *sh = a.shape;
+    const size_t row0 = (size_t)b0 * sh->Q * sh->Hq, eb = elem_bytes(sh);
+    const int rows = (b1 - b0) * sh->Q * sh->Hq;
+    const float *scores = reinterpret_cast<const float *>(a.ws + a.L.scores) + row0 * a.L.ld;
+    int32_t *idx = a.idx + row0 * a.k;
+    float *w = reinterpret_cast<float *>(a.ws + a.L.weights) + row0 * a.k;
+    float4 *stats = reinterpret_cast<float4 *>(a.ws + a.L.stats) + row0;
+    unsigned *counters = reinterpret_cast<unsigned *>(a.ws + a.L.counters) + row0;
+    float *tail = a.tail ? a.tail + row0 : nullptr;
+    int32_t *k_used = a.cert ? a.cert->k_used + row0 : nullptr;
+
+    SelectParams se;
+    se.status = a.dev->status;
+    se.scores = scores;
+    se.seq_lens = a.seq_lens + b0;
+    se.B = b1 - b0; se.Q = sh->Q; se.Hq = sh->Hq; se.L_max = sh->L_max; se.ld = a.L.ld; se.k = a.k;
+    se.idx = idx;
+    se.w = w;
+    se.stats = stats;
+    se.tail = tail;
+    se.counters = counters;
+    if (launch_select(se, s, select_threads) != cudaSuccess) return TKA_ERR_CUDA;
+    if (a.cert) {
+        CertifyParams cp;
+        cp.status = a.dev->status;
+        cp.scores = scores;
+        cp.seq_lens = a.seq_lens + b0;
+        cp.B = b1 - b0; cp.Q = sh->Q; cp.Hq = sh->Hq; cp.L_max = sh->L_max; cp.ld = a.L.ld;
+        cp.k_max = a.k;
+        cp.eps = a.cert->eps;
+        cp.idx = idx;
+        cp.w = w;
+        cp.stats = stats;
+        cp.tail = tail;
+        cp.k_used = k_used;
+        if (launch_certify(cp, s) != cudaSuccess) return TKA_ERR_CUDA;
+    }
+    if (record(events, 2, s) != cudaSuccess) return TKA_ERR_CUDA;
+
+    GatherParams gp;
+    gp.status = a.dev->status;
+    gp.v = a.pages ? a.v_cache
+                   : static_cast<const char *>(a.v_cache) + (size_t)b0 * sh->Hkv * sh->L_max * kHeadDim * eb;
+    gp.seq_lens = a.seq_lens + b0;
+    gp.B = b1 - b0; gp.Q = sh->Q; gp.Hq = sh->Hq; gp.Hkv = sh->Hkv; gp.G = a.G;
+    gp.L_max = sh->L_max; gp.k = a.k; gp.dtype = sh->dtype;
+    gp.idx = idx;
+    gp.w = w;
+    gp.stats = stats;
+    gp.partial = reinterpret_cast<float *>(a.ws + a.L.partial) + row0 * a.L.max_splits * kHeadDim;
+    gp.counters = counters;
+    gp.out = a.out + row0 * kHeadDim;
+    gp.kcount = k_used;
+    if (a.pages) {
+        gp.pages = *a.pages;
+        gp.pages.table += (size_t)b0 * gp.pages.max_pages;
+    }
+    // one wave of eight CTAs per SM (splits = floor(8 x SMs / rows), at least 1),
+    // never fewer than kMinKeysPerSplit keys per CTA
+    int splits = (a.dev->num_sms * 8) / rows;
+    if (splits > a.L.max_splits) splits = a.L.max_splits;
+    if (splits < 1) splits = 1;
+    gp.per_split = (a.k + splits - 1) / splits;
+    gp.splits = (a.k + gp.per_split - 1) / gp.per_split;
+    if (launch_gather(gp, s) != cudaSuccess) return TKA_ERR_CUDA;
+    return TKA_OK;
+}
+
 // Score -> select (k) -> [certify] -> gather on `stream`.
 tka_status decode_impl(const tka_shape *shape, const void *q, const void *k_cache, const void *v_cache,
                        const int32_t *seq_lens, int32_t k, float *out, int32_t *idx, float *tail_mass,
@@ -283,100 +417,37 @@ tka_status decode_impl(const tka_shape *shape, const void *q, const void *k_cach
     if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
         !aligned(idx, 4) || !aligned(seq_lens, 4) || (tail_mass && !aligned(tail_mass, 4)))
         return TKA_ERR_INVALID_ARG;
-    const TokenLayout L = token_layout(shape, k);
-    if (!workspace || !aligned(workspace, 256) || workspace_bytes < L.total) return TKA_ERR_WORKSPACE;
-    DeviceInfo *dev = nullptr;
-    if (device_info(&dev) != cudaSuccess) return TKA_ERR_CUDA;
+    DecodeArgs a;
+    a.shape = shape;
+    a.q = q;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.seq_lens = seq_lens;
+    a.k = k;
+    a.G = shape->Hq / shape->Hkv;
+    a.out = out;
+    a.tail = tail_mass;
+    a.idx = idx;
+    a.L = token_layout(shape, k);
+    a.cert = cert;
+    a.pages = pages;
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < a.L.total) return TKA_ERR_WORKSPACE;
+    a.ws = static_cast<char *>(workspace);
+    if (device_info(&a.dev) != cudaSuccess) return TKA_ERR_CUDA;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    char *ws = static_cast<char *>(workspace);
-    const int G = shape->Hq / shape->Hkv;
-    const int rows = shape->B * shape->Q * shape->Hq;
-
-    float *scores = reinterpret_cast<float *>(ws + L.scores);
-    const int NQ = shape->Q * G;
     // the tensor map addresses cache rows with int32 coordinates
-    const bool tc = score_tc_supported(shape->dtype, NQ) &&
-                    (pages || (long long)shape->B * shape->Hkv * shape->L_max < (1LL << 31));
-    if (tc) {
-        ScoreTcParams tp;
-        tp.status = dev->status;
-        tp.seq_lens = seq_lens;
-        tp.scores = scores;
-        tp.B = shape->B; tp.Q = shape->Q; tp.Hq = shape->Hq; tp.Hkv = shape->Hkv; tp.G = G;
-        tp.L_max = shape->L_max; tp.ld = L.ld; tp.NQ = NQ;
-        tp.scale = resolve_scale(shape);
-        if (pages) tp.pages = *pages;
-        RecordCtx rc{events, 0, s};
-        ScoreTcHook hook;
-        hook.fn = record_hook;
-        hook.ctx = &rc;
-        if (launch_score_tc(tp, q, k_cache, dev->num_sms, s, hook) != cudaSuccess) return TKA_ERR_CUDA;
-    } else {
-        if (record(events, 0, s) != cudaSuccess) return TKA_ERR_CUDA;
-        ScoreParams sp;
-        sp.status = dev->status;
-        sp.q = q;
-        sp.k = k_cache;
-        sp.seq_lens = seq_lens;
-        sp.scores = scores;
-        sp.B = shape->B; sp.Q = shape->Q; sp.Hq = shape->Hq; sp.Hkv = shape->Hkv; sp.G = G;
-        sp.L_max = shape->L_max; sp.ld = L.ld; sp.dtype = shape->dtype;
-        sp.scale = resolve_scale(shape);
-        if (pages) sp.pages = *pages;
-        if (launch_score(sp, dev->num_sms, s) != cudaSuccess) return TKA_ERR_CUDA;
-    }
+    a.tc = score_tc_supported(shape->dtype, shape->Q * a.G) &&
+           (pages || (long long)shape->B * shape->Hkv * shape->L_max < (1LL << 31));
+
+    st = launch_score_part(a, 0, shape->B, s, events);
+    if (st != TKA_OK) return st;
     if (record(events, 1, s) != cudaSuccess) return TKA_ERR_CUDA;
-
-    SelectParams se;
-    se.status = dev->status;
-    se.scores = scores;
-    se.seq_lens = seq_lens;
-    se.B = shape->B; se.Q = shape->Q; se.Hq = shape->Hq; se.L_max = shape->L_max; se.ld = L.ld; se.k = k;
-    se.idx = idx;
-    se.w = reinterpret_cast<float *>(ws + L.weights);
-    se.stats = reinterpret_cast<float4 *>(ws + L.stats);
-    se.tail = tail_mass;
-    se.counters = reinterpret_cast<unsigned *>(ws + L.counters);
-    if (launch_select(se, s) != cudaSuccess) return TKA_ERR_CUDA;
-    if (cert) {
-        CertifyParams cp;
-        cp.status = dev->status;
-        cp.scores = scores;
-        cp.seq_lens = seq_lens;
-        cp.B = shape->B; cp.Q = shape->Q; cp.Hq = shape->Hq; cp.L_max = shape->L_max; cp.ld = L.ld;
-        cp.k_max = k;
-        cp.eps = cert->eps;
-        cp.idx = idx;
-        cp.w = se.w;
-        cp.stats = se.stats;
-        cp.tail = tail_mass;
-        cp.k_used = cert->k_used;
-        if (launch_certify(cp, s) != cudaSuccess) return TKA_ERR_CUDA;
-    }
-    if (record(events, 2, s) != cudaSuccess) return TKA_ERR_CUDA;
-
-    GatherParams gp;
-    gp.status = dev->status;
-    gp.v = v_cache;
-    gp.seq_lens = seq_lens;
-    gp.B = shape->B; gp.Q = shape->Q; gp.Hq = shape->Hq; gp.Hkv = shape->Hkv; gp.G = G;
-    gp.L_max = shape->L_max; gp.k = k; gp.dtype = shape->dtype;
-    gp.idx = idx;
-    gp.w = se.w;
-    gp.stats = se.stats;
-    gp.partial = reinterpret_cast<float *>(ws + L.partial);
-    gp.counters = se.counters;
-    gp.out = out;
-    gp.kcount = cert ? cert->k_used : nullptr;
-    if (pages) gp.pages = *pages;
-    // one wave of eight CTAs per SM (splits = floor(8 x SMs / rows), at least 1),
-    // never fewer than kMinKeysPerSplit keys per CTA
-    int splits = (dev->num_sms * 8) / rows;
-    if (splits > L.max_splits) splits = L.max_splits;
-    if (splits < 1) splits = 1;
-    gp.per_split = (k + splits - 1) / splits;
-    gp.splits = (k + gp.per_split - 1) / gp.per_split;
-    if (launch_gather(gp, s) != cudaSuccess) return TKA_ERR_CUDA;
+    // more rows than SMs: 512-thread select CTAs, two rows per SM at a time
+    // (a 1024-thread CTA takes a whole SM's registers, and the rows would run
+    // in waves of one per SM); otherwise 1024 threads per row
+    const int rows = shape->B * shape->Q * shape->Hq;
+    st = launch_rest_part(a, 0, shape->B, s, rows > a.dev->num_sms ? 512 : 1024, events);
+    if (st != TKA_OK) return st;
     if (record(events, 3, s) != cudaSuccess) return TKA_ERR_CUDA;
     return TKA_OK;
 }

@@ -190,6 +190,48 @@ __device__ inline void warp_find_bin(const uint32_t *hist, uint32_t need, uint32
     }
 }
 
+// The same search spread over the whole block, for two targets at once: the
+// bins holding the need_a-th and the need_b-th largest element (1 <= need <=
+// total count).  Thread t sums the NB / blockDim.x bins below the top
+// t NB / blockDim.x, a block-wide prefix sum over the threads (warp scans plus
+// one word per warp in `wtot`, >= 32 words) locates the thread holding each
+// target, and that thread scans its few bins.  out[0], out[1] = bin and count
+// above it for need_a; out[2], out[3] for need_b.  The histogram must be
+// complete when the block enters (the first barrier here does not wait for
+// it), and every thread reads `out` after the call.
+template <int NB>
+__device__ inline void block_find_bins(const uint32_t *hist, uint32_t need_a, uint32_t need_b, uint32_t *wtot,
+                                       uint32_t *out) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int per = NB / (int)blockDim.x;  // >= 1: NB >= blockDim.x, both powers of two
+    const int top = NB - 1 - (int)threadIdx.x * per;
+    uint32_t local = 0u;
+    for (int j = 0; j < per; j++) local += hist[top - j];
+    const uint32_t incl = warp_incl_scan(local);
+    if (lane == 31) wtot[warp] = incl;
+    __syncthreads();
+    const uint32_t wt = lane < nw ? wtot[lane] : 0u;
+    const uint32_t winc = warp_incl_scan(wt);
+    const uint32_t before = __shfl_sync(0xffffffffu, winc - wt, warp) + incl - local;
+#pragma unroll
+    for (int t = 0; t < 2; t++) {
+        const uint32_t need = t == 0 ? need_a : need_b;
+        if (before < need && before + local >= need) {
+            uint32_t c = before;
+            for (int j = 0; j < per; j++) {
+                const uint32_t h = hist[top - j];
+                if (c + h >= need) {
+                    out[2 * t] = (uint32_t)(top - j);
+                    out[2 * t + 1] = c;
+                    break;
+                }
+                c += h;
+            }
+        }
+    }
+    __syncthreads();
+}
+
 // The same search for the whole block: the block first meets at a barrier
 // (so the histogram is complete and the results of a previous call have been
 // read), warp 0 searches and writes the results, and the block meets again.

@@ -170,8 +170,9 @@ struct ScoreTcHook {
 };
 cudaError_t launch_score_tc(const ScoreTcParams &p, const void *q, const void *k_cache, int num_sms,
                             cudaStream_t stream, const ScoreTcHook &hook);
-cudaError_t launch_select(const SelectParams &p, cudaStream_t stream);
-size_t select_smem_bytes(int k);
+// threads: 1024 (one CTA per SM) or 512 (shares an SM with a scorer CTA)
+cudaError_t launch_select(const SelectParams &p, cudaStream_t stream, int threads = 1024);
+size_t select_smem_bytes(int threads);
 cudaError_t launch_gather(const GatherParams &p, cudaStream_t stream);
 cudaError_t launch_certify(const CertifyParams &p, cudaStream_t stream);
 bool indexer_supported(int G, int d_I);

@@ -7,8 +7,8 @@
 // the discarded mass is the Top-k tail mass of "A Mathematical Theory of
 // Top-k Sparse Attention via Total Variation Distance" (abstract).
 //
-// One CTA (32 warps) per row; every warp owns a contiguous segment of the
-// row, lane l holding positions l, l + 32, ... of it, so a warp compacts 32
+// One CTA (16 or 32 warps) per row; every warp owns a contiguous segment of
+// the row, lane l holding positions l, l + 32, ... of it, so a warp compacts 32
 // consecutive positions at a time with one ballot.  A segment is streamed in
 // batches of 32 x 32 positions with all loads of a batch in flight together
 // (a segment that fits one batch is read once and kept in registers for all
@@ -20,9 +20,10 @@
 //           holds the k-th key with high probability;
 //   pass 2  scores above the range are counted, keys inside it are collected
 //           (unordered) into per-warp candidate lists;
-//   exact radix selection over the candidates' full keys (11 + 11 + 10 bits)
-//           yields the k-th key T and how many of the keys equal to T are
-//           kept (the lowest positions);
+//   exact radix selection over the candidates' keys, in levels of up to 11
+//           bits over the key range the band spans, yields the k-th key T
+//           and how many of the keys equal to T are kept (the lowest
+//           positions); the bins are searched by the whole block;
 //   pass 3  every score is tested against that exact rule and the kept
 //           positions are written straight to their ascending slots (warp
 //           prefix sums plus per-warp offsets), while Z_k = sum_kept e^{s-m}
@@ -38,10 +39,12 @@ namespace tka {
 
 namespace {
 
-constexpr int kSelectThreads = 1024;
-constexpr int kWarps = kSelectThreads / 32;  // <= 32: per-warp words are reduced by one warp, lane w reading warp w's
-constexpr int kSelectCtasPerSm = 1024 / kSelectThreads;
-constexpr int kWarpCand = 256;                  // candidates per warp held in shared memory
+// A row is taken by one CTA of kThreads threads: 1024 when the select runs
+// alone (one CTA per SM), 512 when it shares the SMs with the scorer of the
+// next batch chunk (a 512-thread CTA and a scorer CTA fit one SM's registers
+// and shared memory together).  Up to 32 warps: per-warp words are reduced by
+// one warp, lane w reading warp w's.
+constexpr int kCandWords = 8192;  // candidate keys held in shared memory per row, split evenly over the warps
 constexpr int kHeld = 32;                       // scores per lane held in registers per batch
 constexpr int kSampleMinLen = 16384;            // rows this long histogram a 1/8 sample in pass 1
 
@@ -154,7 +157,8 @@ __device__ void select_multipass(const SelectParams &p, int row, int vis, const 
     });
     m = block_max(m, sm.red);
     __syncthreads();
-    find_bin(hist, 2048, (uint32_t)k, sm.tmp, &sm.scal[0], &sm.scal[1]);
+    __syncthreads();  // the histogram is complete
+    block_find_bins<2048>(hist, (uint32_t)k, (uint32_t)k, sm.tmp, sm.scal);
     const uint32_t b1 = sm.scal[0];
     uint32_t above = sm.scal[1];
     for (int i = threadIdx.x; i < 2048; i += blockDim.x) hist[i] = 0u;
@@ -164,7 +168,8 @@ __device__ void select_multipass(const SelectParams &p, int row, int vis, const 
         if ((key >> 21) == b1) atomicAdd(&hist[(key >> 10) & 0x7ffu], 1u);
     });
     __syncthreads();
-    find_bin(hist, 2048, (uint32_t)k - above, sm.tmp, &sm.scal[0], &sm.scal[1]);
+    __syncthreads();  // the histogram is complete
+    block_find_bins<2048>(hist, (uint32_t)k - above, (uint32_t)k - above, sm.tmp, sm.scal);
     const uint32_t b2 = sm.scal[0];
     above += sm.scal[1];
     const uint32_t pre = (b1 << 11) | b2;
@@ -175,7 +180,8 @@ __device__ void select_multipass(const SelectParams &p, int row, int vis, const 
         if ((key >> 10) == pre) atomicAdd(&hist[key & 0x3ffu], 1u);
     });
     __syncthreads();
-    find_bin(hist, 1024, (uint32_t)k - above, sm.tmp, &sm.scal[0], &sm.scal[1]);
+    __syncthreads();  // the histogram is complete
+    block_find_bins<1024>(hist, (uint32_t)k - above, (uint32_t)k - above, sm.tmp, sm.scal);
     const uint32_t b3 = sm.scal[0];
     above += sm.scal[1];
     const uint32_t T = (pre << 10) | b3, n_eq = hist[b3], r_eq = (uint32_t)k - above;
@@ -235,7 +241,13 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
     return m;
 }
 
-__global__ void __launch_bounds__(kSelectThreads, kSelectCtasPerSm) select_topk(SelectParams p) {
+__host__ __device__ constexpr size_t smem_words(int warps) { return 2048 + 104 + warps * 8 + kCandWords + 2048; }
+
+template <int kThreads>
+__global__ void __launch_bounds__(kThreads, 1024 / kThreads) select_topk(SelectParams p) {
+    constexpr int kWarps = kThreads / 32;
+    static_assert(kWarps <= 32 && kThreads % 32 == 0, "at most 32 whole warps");
+    constexpr int kWarpCand = kCandWords / kWarps;  // a warp's candidate list
     extern __shared__ __align__(16) uint32_t dyn[];
     SelectSmem sm;
     sm.hist = dyn;                                                   // [2048]
@@ -283,7 +295,7 @@ __global__ void __launch_bounds__(kSelectThreads, kSelectCtasPerSm) select_topk(
     // pass 1: the row maximum, and the histogram of the top 11 key bits of a
     // sample: every eighth group of 32 consecutive positions (every position
     // on short rows) -- the threshold is looked for there
-    for (int i = threadIdx.x; i < 2048; i += kSelectThreads) sm.hist[i] = 0u;
+    for (int i = threadIdx.x; i < 2048; i += kThreads) sm.hist[i] = 0u;
     __syncthreads();
     const bool sampled = vis >= kSampleMinLen;
     float m = -INFINITY;
@@ -322,23 +334,15 @@ __global__ void __launch_bounds__(kSelectThreads, kSelectCtasPerSm) select_topk(
     // widened by 4 binomial standard deviations each way and checked exactly
     // below.  As floats: x >= hi_t is above, lo_t <= x < hi_t a candidate.
     float hi_t, lo_t;
+    uint32_t b_hi, b_lo;
     {
         const float ks = (float)k * (float)total_sample / (float)vis;
         const float margin = sampled ? 4.f * sqrtf(ks) + 4.f : 0.f;
         const uint32_t need_hi = (uint32_t)fmaxf(1.f, floorf(ks - margin));
         const uint32_t need_lo = (uint32_t)fminf((float)total_sample, ceilf(ks + margin));
-        __syncthreads();
-        if (warp == 0) {
-            uint32_t bh, bl, unused;
-            warp_find_bin<2048>(sm.hist, need_hi, bh, unused);
-            warp_find_bin<2048>(sm.hist, max(need_lo, need_hi), bl, unused);
-            if (lane == 0) {
-                sm.scal[0] = bh;
-                sm.scal[1] = bl;
-            }
-        }
-        __syncthreads();
-        const uint32_t b_hi = sm.scal[0], b_lo = sm.scal[1];
+        block_find_bins<2048>(sm.hist, need_hi, max(need_lo, need_hi), sm.tmp, sm.scal);
+        b_hi = sm.scal[0];
+        b_lo = sm.scal[2];
         // a NaN threshold compares false: nothing above bin 2044 (+inf) or below bin 4 (-FLT_MAX)
         hi_t = b_hi >= 2044u ? __uint_as_float(0x7fc00000u) : key_float((b_hi + 1u) << 21);
         lo_t = key_float(b_lo << 21);
@@ -376,48 +380,48 @@ __global__ void __launch_bounds__(kSelectThreads, kSelectCtasPerSm) select_topk(
         return;
     }
 
-    // exact radix selection over the candidates' full 32-bit keys (11 + 11 +
-    // 10 bits): r of them are kept
+    // exact radix selection over the candidates' keys.  They lie in the
+    // band's key range [base, base + 2^rem) (bins b_lo..b_hi of 2^21 keys;
+    // with no upper threshold, everything up to the top key), so every level
+    // splits the current range into at most 2048 bins and the candidates
+    // spread over the bins instead of piling into the few bins of the band
+    // (few conflicting atomics); two levels reach a single key unless the
+    // band spans more than two bins.
     const uint32_t need = (uint32_t)k - above;
-    uint32_t pre = 0u, gt = 0u, T = 0u;
+    uint32_t gt = 0u, base = b_lo << 21;
+    int rem;
+    {
+        const uint32_t nb = (b_hi >= 2044u ? 2047u : b_hi) - b_lo + 1u;  // >= 1
+        rem = 21 + (nb > 1u ? 32 - __clz(nb - 1u) : 0);                // <= 32
+    }
     // two histograms: level L counts into sm.hist (L even) or hist2 (L odd)
     // while the other one is cleared for level L + 1; warp 0 searches between
     // two barriers
-    for (int i = threadIdx.x; i < 2048; i += kSelectThreads) {
+    for (int i = threadIdx.x; i < 2048; i += kThreads) {
         sm.hist[i] = 0u;
         hist2[i] = 0u;
     }
     __syncthreads();
-    for (int level = 0; level < 3; level++) {
-        const int shift = level == 0 ? 21 : (level == 1 ? 10 : 0);
-        const uint32_t nbm = level == 2 ? 1023u : 2047u;
+    const uint32_t my_cand = wstat[warp * 8 + 1];
+    for (int level = 0; rem > 0; level++) {
+        const int sh = rem > 11 ? rem - 11 : 0;
         uint32_t *h = (level & 1) ? hist2 : sm.hist;
-        for (uint32_t i = lane; i < wstat[warp * 8 + 1]; i += 32) {  // this warp's own list
+        const unsigned long long span = 1ull << rem;
+        for (uint32_t i = lane; i < my_cand; i += 32) {  // this warp's own list
             const uint32_t key = canon_key(__uint_as_float(my_key[i]));
-            if (level == 0 || (key >> (shift + (level == 1 ? 11 : 10))) == pre) atomicAdd(&h[(key >> shift) & nbm], 1u);
+            if (key >= base && (unsigned long long)(key - base) < span) atomicAdd(&h[(key - base) >> sh], 1u);
         }
-        if (level == 1)
-            for (int i = threadIdx.x; i < 2048; i += kSelectThreads) sm.hist[i] = 0u;
-        __syncthreads();
-        if (warp == 0) {
-            uint32_t bin, above_bin;
-            if (level == 2)
-                warp_find_bin<1024>(h, need - gt, bin, above_bin);
-            else
-                warp_find_bin<2048>(h, need - gt, bin, above_bin);
-            if (lane == 0) {
-                sm.scal[0] = bin;
-                sm.scal[1] = above_bin;
-            }
+        if (level >= 1) {  // the previous level's histogram, for the next level
+            uint32_t *hn = (level & 1) ? sm.hist : hist2;
+            for (int i = threadIdx.x; i < 2048; i += kThreads) hn[i] = 0u;
         }
-        __syncthreads();
-        const uint32_t bin = sm.scal[0];
+        __syncthreads();  // the histogram is complete
+        block_find_bins<2048>(h, need - gt, need - gt, sm.tmp, sm.scal);
         gt += sm.scal[1];
-        if (level < 2)
-            pre = (pre << (level == 0 ? 0 : 11)) | bin;
-        else
-            T = (pre << 10) | bin;
+        base += sm.scal[0] << sh;
+        rem = sh;
     }
+    const uint32_t T = base;
     // keys equal to T: the first r_eq of them (by position) are kept
     const uint32_t r_eq = need - gt;
 
@@ -505,24 +509,31 @@ __global__ void __launch_bounds__(kSelectThreads, kSelectCtasPerSm) select_topk(
 
 }  // namespace
 
-size_t select_smem_bytes(int) {
-    return (size_t)(2048 + 104 + kWarps * 8) * 4 + (size_t)kWarps * kWarpCand * 4 + 2048 * 4;
-}
+size_t select_smem_bytes(int threads) { return smem_words(threads / 32) * 4; }
 
-cudaError_t launch_select(const SelectParams &p, cudaStream_t stream) {
+namespace {
+
+template <int kThreads>
+cudaError_t launch_n(const SelectParams &p, cudaStream_t stream) {
     const int rows = p.B * p.Q * p.Hq;
-    const size_t smem = select_smem_bytes(p.k);
+    const size_t smem = select_smem_bytes(kThreads);
     static bool attr_set[64] = {};  // per device: the shared-memory opt-in is a function attribute
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (smem > 48 * 1024 && (dev < 0 || dev >= 64 || !attr_set[dev])) {
-        e = cudaFuncSetAttribute(select_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        e = cudaFuncSetAttribute(select_topk<kThreads>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
-    select_topk<<<rows, kSelectThreads, smem, stream>>>(p);
+    select_topk<kThreads><<<rows, kThreads, smem, stream>>>(p);
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_select(const SelectParams &p, cudaStream_t stream, int threads) {
+    return threads == 512 ? launch_n<512>(p, stream) : launch_n<1024>(p, stream);
 }
 
 }  // namespace tka

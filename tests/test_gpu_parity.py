@@ -48,6 +48,9 @@ TOKEN_CASES = [
     ("bf16", 1, 1, 8, 2, 256, None, 256),              # k = visible keys
     ("bf16", 1, 1, 8, 8, 10000, None, 8192),           # largest k
     ("bf16", 1, 3, 4, 4, 700, None, 30),               # G = 1 (multi-head), Q = 3
+    ("bf16", 5, 1, 32, 8, 20000, [20000, 19001, 16384, 17777, 20000], 1024),  # more rows than SMs: 512-thread
+                                                       # select, sampled band, segments streamed in two batches
+    ("bf16", 1, 1, 8, 2, 40000, None, 2048),           # 1024-thread select, segments streamed in two batches
 ]
 
 
