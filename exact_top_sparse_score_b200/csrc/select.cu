@@ -45,6 +45,7 @@ namespace {
 // and shared memory together).  Up to 32 warps: per-warp words are reduced by
 // one warp, lane w reading warp w's.
 constexpr int kCandWords = 8192;  // candidate keys held in shared memory per row, split evenly over the warps
+constexpr int kPlusWords = 6144;  // (score, position) pairs of the scores at or above the band, split likewise
 constexpr int kHeld = 32;                       // scores per lane held in registers per batch
 constexpr int kSampleMinLen = 16384;            // rows this long histogram a 1/8 sample in pass 1
 
@@ -116,7 +117,7 @@ __device__ __forceinline__ void finish_row(const SelectParams &p, int row, float
         }
         __syncthreads();
         zk = warp_sum(lane < nw ? sm.red[2 * lane] : 0.f);
-        zt = warp_sum(lane < nw ? sm.red[2 * lane + 1] : 0.f);
+        zt = fmaxf(warp_sum(lane < nw ? sm.red[2 * lane + 1] : 0.f), 0.f);  // formed as total - kept: >= 0
     }
     if (threadIdx.x == 0) {
         if (written != kept) raise_status(p.status, TKA_DEV_INTERNAL);
@@ -241,7 +242,9 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
     return m;
 }
 
-__host__ __device__ constexpr size_t smem_words(int warps) { return 2048 + 104 + warps * 8 + kCandWords + 2048; }
+__host__ __device__ constexpr size_t smem_words(int warps) {
+    return 2048 + 104 + warps * 8 + kCandWords + 2048 + 2 * kPlusWords;
+}
 
 template <int kThreads>
 __global__ void __launch_bounds__(kThreads, 1024 / kThreads) select_topk(SelectParams p) {
@@ -257,6 +260,9 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads) select_topk(SelectP
     uint32_t *wstat = dyn + 2048 + 104;                              // [kWarps][8]
     uint32_t *wc_key = wstat + kWarps * 8;                           // [kWarps][kWarpCand]
     uint32_t *hist2 = wc_key + kWarps * kWarpCand;                   // [2048] second radix histogram
+    constexpr int kPlusCap = kPlusWords / kWarps;                    // a warp's list of scores >= the band
+    float *plus_x = reinterpret_cast<float *>(hist2 + 2048);         // [kWarps][kPlusCap]
+    int32_t *plus_pos = reinterpret_cast<int32_t *>(plus_x + kPlusWords);  // [kWarps][kPlusCap]
 
     const int row = blockIdx.x;
     const int b = row / (p.Q * p.Hq), qpos = (row / p.Hq) % p.Q;
@@ -349,20 +355,39 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads) select_topk(SelectP
     }
 
     // pass 2: count the positions above the range; collect the keys inside it
-    // (in any order: only their values matter) into this warp's candidate list
-    uint32_t nwin = 0u;
+    // (in any order: only their values matter) into this warp's candidate
+    // list; append every score at or above the range, with its position, to
+    // this warp's ordered list (one ballot per round keeps position order);
+    // sum e^{s-m} over all positions
+    uint32_t nwin = 0u, nplus = 0u;
     uint32_t *my_key = wc_key + warp * kWarpCand;
+    float *my_px = plus_x + warp * kPlusCap;
+    int32_t *my_pp = plus_pos + warp * kPlusCap;
+    const float m_l2e = m * kLog2e;
+    float zall = 0.f;
     for (int bi = 0; bi < nbatch; bi++) {
         if (!resident) load_batch(bi);
+        const int p0 = lo + bi * 32 * kHeld + lane;
 #pragma unroll
         for (int r = 0; r < kHeld; r++) {
             const float xv = x[r];
+            zall += exp2_approx(fmaf(xv, kLog2e, -m_l2e));
             const bool above = xv >= hi_t;
             nwin += above;
-            if (xv >= lo_t && !above) {
-                const uint32_t slot = atomicAdd(&wstat[warp * 8 + 1], 1u);
-                if (slot < (uint32_t)kWarpCand) my_key[slot] = __float_as_uint(xv);  // converted when ranked
+            const bool plus = xv >= lo_t;
+            const uint32_t pb = __ballot_sync(0xffffffffu, plus);
+            if (plus) {
+                const uint32_t slot = nplus + __popc(pb & lt);
+                if (slot < (uint32_t)kPlusCap) {
+                    my_px[slot] = xv;
+                    my_pp[slot] = p0 + 32 * r;
+                }
+                if (!above) {
+                    const uint32_t cs = atomicAdd(&wstat[warp * 8 + 1], 1u);
+                    if (cs < (uint32_t)kWarpCand) my_key[cs] = __float_as_uint(xv);  // converted when ranked
+                }
             }
+            nplus += __popc(pb);
         }
     }
     nwin = warp_sum(nwin);
@@ -460,9 +485,11 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads) select_topk(SelectP
     // pass 3: the exact rule -- s > T, or s == T among the first r_eq ties
     // (s >= T when every tie is kept) -- written straight to the final
     // ascending positions, with the softmax sums of kept and dropped scores.
-    // As float comparisons: canon_key order is float order.
+    // As float comparisons: canon_key order is float order.  A warp whose
+    // ordered list is complete takes its kept positions from the list (every
+    // kept score is at or above the range) and its dropped mass as the total
+    // less the kept; a warp whose list overflowed streams its segment again.
     const float T_f = key_float(T);
-    const float m_l2e = m * kLog2e;
     int32_t *idx = p.idx + (size_t)row * k;
     float *wv = p.w + (size_t)row * k;
     float zk = 0.f, zt = 0.f;
@@ -480,24 +507,53 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads) select_topk(SelectP
         }
         out_run += __popc(sb);
     };
-    for (int bi = 0; bi < nbatch; bi++) {
-        if (!resident) load_batch(bi);
-        const int p0 = lo + bi * 32 * kHeld + lane;
-        if (rank_ties) {
-#pragma unroll
-            for (int r = 0; r < kHeld; r++) {
-                const float xv = x[r];
+    if (nplus <= (uint32_t)kPlusCap) {
+        for (uint32_t i0 = 0; i0 < nplus; i0 += 32) {
+            const uint32_t i = i0 + lane;
+            const float xv = i < nplus ? my_px[i] : -INFINITY;
+            bool sel;
+            if (rank_ties) {
                 const bool tie = xv == T_f;
                 const uint32_t tb = __ballot_sync(0xffffffffu, tie);
-                const bool sel = xv > T_f || (tie && tie_run + __popc(tb & lt) < r_eq);
+                sel = xv > T_f || (tie && tie_run + __popc(tb & lt) < r_eq);
                 tie_run += __popc(tb);
-                emit(sel, exp2_approx(fmaf(xv, kLog2e, -m_l2e)), p0 + 32 * r);
+            } else {
+                sel = xv >= T_f;
             }
-        } else {
+            const uint32_t sb = __ballot_sync(0xffffffffu, sel);
+            if (sel) {
+                const float e = exp2_approx(fmaf(xv, kLog2e, -m_l2e));
+                const uint32_t o = out_run + __popc(sb & lt);
+                if (o < (uint32_t)k) {  // always true unless the counts above are wrong
+                    idx[o] = my_pp[i];
+                    wv[o] = e;
+                }
+                zk += e;
+            }
+            out_run += __popc(sb);
+        }
+        // dropped = all - kept, per warp (the warp's lanes sum to its totals)
+        zt = zall - zk;
+    } else {
+        for (int bi = 0; bi < nbatch; bi++) {
+            if (!resident) load_batch(bi);
+            const int p0 = lo + bi * 32 * kHeld + lane;
+            if (rank_ties) {
 #pragma unroll
-            for (int r = 0; r < kHeld; r++) {
-                const float xv = x[r];
-                emit(xv >= T_f, exp2_approx(fmaf(xv, kLog2e, -m_l2e)), p0 + 32 * r);
+                for (int r = 0; r < kHeld; r++) {
+                    const float xv = x[r];
+                    const bool tie = xv == T_f;
+                    const uint32_t tb = __ballot_sync(0xffffffffu, tie);
+                    const bool sel = xv > T_f || (tie && tie_run + __popc(tb & lt) < r_eq);
+                    tie_run += __popc(tb);
+                    emit(sel, exp2_approx(fmaf(xv, kLog2e, -m_l2e)), p0 + 32 * r);
+                }
+            } else {
+#pragma unroll
+                for (int r = 0; r < kHeld; r++) {
+                    const float xv = x[r];
+                    emit(xv >= T_f, exp2_approx(fmaf(xv, kLog2e, -m_l2e)), p0 + 32 * r);
+                }
             }
         }
     }

@@ -87,6 +87,21 @@ def test_planted_heavy_tail(cuda_device):
     check_token(w, 256, out, idx, tail, oracle.topk_attn(w, 256))
 
 
+@pytest.mark.parametrize("rise", [1.5, 6.0, 30.0])
+def test_scores_rising_with_position(rise, cuda_device):
+    # a recency-like pattern: keys drift along their group's mean query
+    # direction with position, so the kept positions crowd into the last
+    # segments of each row (more per warp than its ordered list holds)
+    B, Hq, Hkv, L = 5, 32, 8, 20000
+    w = workloads.make_workload(B, 1, Hq, Hkv, L, dtype="bf16", seed=7)
+    u = w.q.float().reshape(B, Hkv, Hq // Hkv, 128).mean(2)
+    u = u / u.norm(dim=-1, keepdim=True)
+    ramp = torch.linspace(0.0, rise, L)
+    w.k_cache[:] = (w.k_cache.float() + ramp[None, None, :, None] * u[:, :, None, :]).to(w.k_cache.dtype)
+    out, idx, tail = run_token(w, 1024)
+    check_token(w, 1024, out, idx, tail, oracle.topk_attn(w, 1024))
+
+
 def test_repeat_calls_are_bitwise_identical(cuda_device):
     w = workloads.make_workload(2, 1, 32, 8, 3000, dtype="bf16", seed=6)
     q, kc, vc, lens = to_device(w)
