@@ -32,6 +32,8 @@
 // If the sampled range misses the k-th key, or a warp collects more
 // candidates than fit, the row falls back to three exact histogram passes and
 // an ordered compaction pass over the row.
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -46,7 +48,8 @@ namespace {
 // one warp, lane w reading warp w's.
 constexpr int kCandWords = 8192;  // candidate keys held in shared memory per row, split evenly over the warps
 constexpr int kPlusWords = 6144;  // (score, position) pairs of the scores at or above the band, split likewise
-constexpr int kHeld = 32;                       // scores per lane held in registers per batch
+constexpr int kHeld = 32;  // scores per lane held in registers (a resident segment: 32 x 32 positions)
+constexpr int kStep = 16;  // scores per lane per step of a streamed segment (half the registers)
 constexpr int kSampleMinLen = 16384;            // rows this long histogram a 1/8 sample in pass 1
 
 constexpr int kBatch = 8;  // float4 loads in flight per thread
@@ -284,45 +287,84 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads) select_topk(SelectP
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint32_t lt = lanemask_lt();
     // this warp's contiguous segment; lane l holds positions lo + 32 r + l of
-    // each batch of 32 * kHeld positions, -inf past the segment's end (so the
-    // passes below need no bounds tests: -inf is never kept and weighs 0)
+    // it, -inf past the segment's end (so the passes below need no bounds
+    // tests: -inf is never kept and weighs 0).  A segment of up to 32 kHeld
+    // positions is loaded once and kept in registers for every pass; a longer
+    // one is streamed in steps of 32 kStep positions through the two halves
+    // of the same registers, the loads of the next step in flight while the
+    // current one is processed.
     const int seg = (((vis + kWarps - 1) / kWarps) + 31) & ~31;
     const int lo = min(vis, warp * seg), hi = min(vis, lo + seg);
-    const int nbatch = (hi - lo + 32 * kHeld - 1) / (32 * kHeld);
-    const bool resident = nbatch <= 1;  // the whole segment fits in registers
+    const bool resident = hi - lo <= 32 * kHeld;
+    const int nstep = (hi - lo + 32 * kStep - 1) / (32 * kStep);
     float x[kHeld];
-    auto load_batch = [&](int bi) {
-        const int p0 = lo + bi * 32 * kHeld + lane;
+    // positions lo + 32 (n0 + r) + lane into x[off + r], r < cnt
+    auto load_into = [&](auto off_c, auto cnt_c, int n0) {
+        constexpr int off = decltype(off_c)::value, cnt = decltype(cnt_c)::value;
+        const int p0 = lo + 32 * n0 + lane;
 #pragma unroll
-        for (int r = 0; r < kHeld; r++) x[r] = p0 + 32 * r < hi ? __ldcg(s + p0 + 32 * r) : -INFINITY;
+        for (int r = 0; r < cnt; r++) x[off + r] = p0 + 32 * r < hi ? __ldcg(s + p0 + 32 * r) : -INFINITY;
     };
-    if (resident) load_batch(0);
+    using C0 = std::integral_constant<int, 0>;
+    using CS = std::integral_constant<int, kStep>;
+    using CH = std::integral_constant<int, kHeld>;
+    // calls f(off_c, cnt_c, p0) on every part of the segment held in x
+    auto for_segment = [&](auto &&f) {
+        if (resident) {
+            f(C0{}, CH{}, lo + lane);
+            return;
+        }
+        load_into(C0{}, CS{}, 0);
+        for (int st = 0; st < nstep; st += 2) {
+            if (st + 1 < nstep) load_into(CS{}, CS{}, (st + 1) * kStep);
+            f(C0{}, CS{}, lo + 32 * st * kStep + lane);
+            if (st + 1 < nstep) {
+                if (st + 2 < nstep) load_into(C0{}, CS{}, (st + 2) * kStep);
+                f(CS{}, CS{}, lo + 32 * (st + 1) * kStep + lane);
+            }
+        }
+    };
+    if (resident) load_into(C0{}, CH{}, 0);
 
-    // pass 1: the row maximum, and the histogram of the top 11 key bits of a
-    // sample: every eighth group of 32 consecutive positions (every position
-    // on short rows) -- the threshold is looked for there
+    // pass 1: the histogram of the top 11 key bits of a sample: every eighth
+    // group of 32 consecutive positions (every position on short rows) -- the
+    // threshold is looked for there.  A streamed segment reads just its
+    // sample here.
     for (int i = threadIdx.x; i < 2048; i += kThreads) sm.hist[i] = 0u;
     __syncthreads();
-    const bool sampled = vis >= kSampleMinLen;
-    float m = -INFINITY;
+    const bool sampled = vis >= kSampleMinLen;  // always so for a streamed segment
     uint32_t nsample = 0u;
-    for (int bi = 0; bi < nbatch; bi++) {
-        if (!resident) load_batch(bi);
-        const int p0 = lo + bi * 32 * kHeld + lane;
-#pragma unroll
-        for (int r = 0; r < kHeld; r++) m = fmaxf(m, x[r]);
+    if (resident) {
         if (sampled) {
 #pragma unroll
             for (int r = 0; r < kHeld; r += 8) {
-                if (p0 + 32 * r < hi) {
+                if (lo + lane + 32 * r < hi) {
                     atomicAdd(&sm.hist[canon_key(x[r]) >> 21], 1u);
                     nsample++;
                 }
             }
         } else {
-            for (int r = 0; r < kHeld; r++) {  // short rows: every position (not unrolled: rare)
-                if (p0 + 32 * r < hi) {
+#pragma unroll
+            for (int r = 0; r < kHeld; r++) {
+                if (lo + lane + 32 * r < hi) {
                     atomicAdd(&sm.hist[canon_key(x[r]) >> 21], 1u);
+                    nsample++;
+                }
+            }
+        }
+    } else {
+        // groups 0, 8, 16, ... of the segment, four loads in flight
+        for (int g0 = 0; lo + 32 * g0 < hi; g0 += 32) {
+            float v[4];
+#pragma unroll
+            for (int u = 0; u < 4; u++) {
+                const int pos = lo + 32 * (g0 + 8 * u) + lane;
+                v[u] = pos < hi ? __ldcg(s + pos) : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; u++) {
+                if (lo + 32 * (g0 + 8 * u) + lane < hi) {
+                    atomicAdd(&sm.hist[canon_key(v[u]) >> 21], 1u);
                     nsample++;
                 }
             }
@@ -331,7 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads) select_topk(SelectP
     if (lane == 0) wstat[warp * 8 + 1] = 0u;  // this warp's candidate count, for pass 2
     nsample = warp_sum(nsample);
     if (lane == 0) wstat[warp * 8 + 6] = nsample;
-    m = block_max(m, sm.red);  // contains __syncthreads
+    __syncthreads();  // the histogram and the sample counts are complete
     // word f of the lane-th warp (0 past the last warp), for warp-wide reductions
     auto wword = [&](int f) { return lane < kWarps ? wstat[lane * 8 + f] : 0u; };
     const uint32_t total_sample = warp_sum(wword(6));
@@ -354,24 +396,31 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads) select_topk(SelectP
         lo_t = key_float(b_lo << 21);
     }
 
-    // pass 2: count the positions above the range; collect the keys inside it
-    // (in any order: only their values matter) into this warp's candidate
-    // list; append every score at or above the range, with its position, to
-    // this warp's ordered list (one ballot per round keeps position order);
-    // sum e^{s-m} over all positions
+    // pass 2: the row maximum; count the positions above the range; collect
+    // the keys inside it (in any order: only their values matter) into this
+    // warp's candidate list; append every score at or above the range, with
+    // its position, to this warp's ordered list (one ballot per round keeps
+    // position order); sum e^{s - m_lane} over this lane's positions against
+    // a running lane maximum m_lane (rescaled when it grows)
     uint32_t nwin = 0u, nplus = 0u;
     uint32_t *my_key = wc_key + warp * kWarpCand;
     float *my_px = plus_x + warp * kPlusCap;
     int32_t *my_pp = plus_pos + warp * kPlusCap;
-    const float m_l2e = m * kLog2e;
-    float zall = 0.f;
-    for (int bi = 0; bi < nbatch; bi++) {
-        if (!resident) load_batch(bi);
-        const int p0 = lo + bi * 32 * kHeld + lane;
+    float m_lane = -INFINITY, zall = 0.f;
+    for_segment([&](auto off_c, auto cnt_c, int p0) {
+        constexpr int off = decltype(off_c)::value, cnt = decltype(cnt_c)::value;
+        float bm = x[off];
 #pragma unroll
-        for (int r = 0; r < kHeld; r++) {
-            const float xv = x[r];
-            zall += exp2_approx(fmaf(xv, kLog2e, -m_l2e));
+        for (int r = 1; r < cnt; r++) bm = fmaxf(bm, x[off + r]);
+        if (bm > m_lane) {  // never true for a part with no position (all -inf)
+            zall *= exp2_approx((m_lane - bm) * kLog2e);
+            m_lane = bm;
+        }
+        const float ml = m_lane == -INFINITY ? 0.f : m_lane * kLog2e;
+#pragma unroll
+        for (int r = 0; r < cnt; r++) {
+            const float xv = x[off + r];
+            zall += exp2_approx(fmaf(xv, kLog2e, -ml));
             const bool above = xv >= hi_t;
             nwin += above;
             const bool plus = xv >= lo_t;
@@ -389,10 +438,16 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads) select_topk(SelectP
             }
             nplus += __popc(pb);
         }
-    }
+    });
+    float m = warp_max(m_lane);
+    if (lane == 0) wstat[warp * 8 + 5] = __float_as_uint(m);
     nwin = warp_sum(nwin);
     if (lane == 0) wstat[warp * 8 + 0] = nwin;
     __syncthreads();
+    m = warp_max(lane < kWarps ? __uint_as_float(wstat[lane * 8 + 5]) : -INFINITY);  // the row maximum
+    const float m_l2e = m * kLog2e;
+    // this lane's sum against the row maximum
+    zall = m_lane == -INFINITY ? 0.f : zall * exp2_approx((m_lane - m) * kLog2e);
     // block totals, every warp reducing the per-warp words (lane w reads warp w's)
     const uint32_t above = warp_sum(wword(0));
     const uint32_t ncand = warp_sum(wword(1));
@@ -535,27 +590,21 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads) select_topk(SelectP
         // dropped = all - kept, per warp (the warp's lanes sum to its totals)
         zt = zall - zk;
     } else {
-        for (int bi = 0; bi < nbatch; bi++) {
-            if (!resident) load_batch(bi);
-            const int p0 = lo + bi * 32 * kHeld + lane;
-            if (rank_ties) {
+        for_segment([&](auto off_c, auto cnt_c, int p0) {
+            constexpr int off = decltype(off_c)::value, cnt = decltype(cnt_c)::value;
 #pragma unroll
-                for (int r = 0; r < kHeld; r++) {
-                    const float xv = x[r];
+            for (int r = 0; r < cnt; r++) {
+                const float xv = x[off + r];
+                bool sel = xv >= T_f;
+                if (rank_ties) {
                     const bool tie = xv == T_f;
                     const uint32_t tb = __ballot_sync(0xffffffffu, tie);
-                    const bool sel = xv > T_f || (tie && tie_run + __popc(tb & lt) < r_eq);
+                    sel = xv > T_f || (tie && tie_run + __popc(tb & lt) < r_eq);
                     tie_run += __popc(tb);
-                    emit(sel, exp2_approx(fmaf(xv, kLog2e, -m_l2e)), p0 + 32 * r);
                 }
-            } else {
-#pragma unroll
-                for (int r = 0; r < kHeld; r++) {
-                    const float xv = x[r];
-                    emit(xv >= T_f, exp2_approx(fmaf(xv, kLog2e, -m_l2e)), p0 + 32 * r);
-                }
+                emit(sel, exp2_approx(fmaf(xv, kLog2e, -m_l2e)), p0 + 32 * r);
             }
-        }
+        });
     }
     if (lane == 0) wstat[warp * 8 + 4] = out_run - out_begin;
     __syncthreads();
