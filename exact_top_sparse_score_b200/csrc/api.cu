@@ -315,7 +315,7 @@ tka_status launch_score_part(const DecodeArgs &a, int b0, int b1, cudaStream_t s
         ScoreTcHook hook;
         hook.fn = record_hook;
         hook.ctx = &rc;
-        if (launch_score_tc(tp, q, kc, a.dev->num_sms, s, hook) != cudaSuccess) return TKA_ERR_CUDA;
+        if (launch_score_tc(tp, q, kc, a.dev->num_sms, s, hook, events == nullptr) != cudaSuccess) return TKA_ERR_CUDA;
     } else {
         if (record(events, 0, s) != cudaSuccess) return TKA_ERR_CUDA;
         ScoreParams sp;
@@ -357,7 +357,9 @@ tka_status launch_rest_part(const DecodeArgs &a, int b0, int b1, cudaStream_t s,
     se.stats = stats;
     se.tail = tail;
     se.counters = counters;
-    if (launch_select(se, s, select_threads) != cudaSuccess) return TKA_ERR_CUDA;
+    // with no stage events between them, each kernel may start behind the one before
+    const bool pdl = events == nullptr;
+    if (launch_select(se, s, select_threads, pdl) != cudaSuccess) return TKA_ERR_CUDA;
     if (a.cert) {
         CertifyParams cp;
         cp.status = a.dev->status;
@@ -371,7 +373,7 @@ tka_status launch_rest_part(const DecodeArgs &a, int b0, int b1, cudaStream_t s,
         cp.stats = stats;
         cp.tail = tail;
         cp.k_used = k_used;
-        if (launch_certify(cp, s) != cudaSuccess) return TKA_ERR_CUDA;
+        if (launch_certify(cp, s, pdl) != cudaSuccess) return TKA_ERR_CUDA;
     }
     if (record(events, 2, s) != cudaSuccess) return TKA_ERR_CUDA;
 
@@ -400,7 +402,7 @@ tka_status launch_rest_part(const DecodeArgs &a, int b0, int b1, cudaStream_t s,
     if (splits < 1) splits = 1;
     gp.per_split = (a.k + splits - 1) / splits;
     gp.splits = (a.k + gp.per_split - 1) / gp.per_split;
-    if (launch_gather(gp, s) != cudaSuccess) return TKA_ERR_CUDA;
+    if (launch_gather(gp, s, pdl) != cudaSuccess) return TKA_ERR_CUDA;
     return TKA_OK;
 }
 

@@ -105,6 +105,8 @@ __global__ void __launch_bounds__(kMaxThreads) certify_topk(CertifyParams p) {
     __shared__ unsigned long long s_mass;
     __shared__ uint32_t s_bin, s_cnt;
     __shared__ uint32_t s_kmin[32], s_kmax[32];
+    pdl_wait();  // the selection comes from the kernel before
+    pdl_trigger();
 
     const int row = blockIdx.x;
     const int b = row / (p.Q * p.Hq), qpos = (row / p.Hq) % p.Q;
@@ -288,14 +290,13 @@ __global__ void __launch_bounds__(kMaxThreads) certify_topk(CertifyParams p) {
 
 }  // namespace
 
-cudaError_t launch_certify(const CertifyParams &p, cudaStream_t stream) {
+cudaError_t launch_certify(const CertifyParams &p, cudaStream_t stream, bool pdl) {
     if (p.k_max > kMaxK) return cudaErrorInvalidValue;
     const int threads = max(64, min(kCertThreads, (p.k_max + kCertPer * 32 - 1) / (kCertPer * 32) * 32));
     if (threads <= 256)
-        certify_topk<256><<<p.B * p.Q * p.Hq, threads, 0, stream>>>(p);
+        return launch_k(pdl, certify_topk<256>, dim3(p.B * p.Q * p.Hq), dim3(threads), 0, stream, p);
     else
-        certify_topk<kCertThreads><<<p.B * p.Q * p.Hq, threads, 0, stream>>>(p);
-    return cudaGetLastError();
+        return launch_k(pdl, certify_topk<kCertThreads>, dim3(p.B * p.Q * p.Hq), dim3(threads), 0, stream, p);
 }
 
 }  // namespace tka

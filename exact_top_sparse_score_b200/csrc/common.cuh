@@ -58,6 +58,15 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 // a == b iff key(a) == key(b).
 __device__ __forceinline__ uint32_t canon_key(float f) { return order_key(__fadd_rn(f, 0.f)); }
 
+// Programmatic dependent launch.  A kernel launched with launch_pdl may be
+// started while the kernel before it on the stream is still running: it must
+// call pdl_wait() before it reads anything that kernel (or any earlier work)
+// wrote -- the wait returns once the earlier grid has completed and its
+// writes are visible, and at once for a kernel launched without the
+// attribute.  pdl_trigger() lets the launch of the next kernel begin.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
 // 2^t by the hardware approximation (PTX ex2.approx.ftz.f32).
 __device__ __forceinline__ float exp2_approx(float t) {
     float r;

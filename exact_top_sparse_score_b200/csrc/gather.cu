@@ -61,6 +61,8 @@ __global__ void __launch_bounds__(kGatherThreads, 8) gather_pv(GatherParams p) {
     __shared__ unsigned s_ticket;
 
     const int row = blockIdx.y, split = blockIdx.x;
+    pdl_wait();  // the kept positions and weights come from the kernel before
+    pdl_trigger();
     const int b = row / (p.Q * p.Hq), qpos = (row / p.Hq) % p.Q, h = row % p.Hq;
     const int seq_len = p.seq_lens[b];
     if (!seq_len_ok(seq_len, p.Q, p.L_max)) return;  // the select step raised the status
@@ -156,22 +158,21 @@ __global__ void __launch_bounds__(kGatherThreads, 8) gather_pv(GatherParams p) {
 
 }  // namespace
 
-cudaError_t launch_gather(const GatherParams &p, cudaStream_t stream) {
+cudaError_t launch_gather(const GatherParams &p, cudaStream_t stream, bool pdl) {
     const int rows = p.B * p.Q * p.Hq;
     const dim3 grid(p.splits, rows);
     const bool paged = p.pages.table != nullptr;
     if (p.dtype == TKA_BF16) {
         if (paged)
-            gather_pv<__nv_bfloat16, true><<<grid, kGatherThreads, 0, stream>>>(p);
+            return launch_k(pdl, gather_pv<__nv_bfloat16, true>, grid, dim3(kGatherThreads), 0, stream, p);
         else
-            gather_pv<__nv_bfloat16, false><<<grid, kGatherThreads, 0, stream>>>(p);
+            return launch_k(pdl, gather_pv<__nv_bfloat16, false>, grid, dim3(kGatherThreads), 0, stream, p);
     } else {
         if (paged)
-            gather_pv<float, true><<<grid, kGatherThreads, 0, stream>>>(p);
+            return launch_k(pdl, gather_pv<float, true>, grid, dim3(kGatherThreads), 0, stream, p);
         else
-            gather_pv<float, false><<<grid, kGatherThreads, 0, stream>>>(p);
+            return launch_k(pdl, gather_pv<float, false>, grid, dim3(kGatherThreads), 0, stream, p);
     }
-    return cudaGetLastError();
 }
 
 }  // namespace tka

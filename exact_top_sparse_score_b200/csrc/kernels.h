@@ -154,6 +154,25 @@ struct BlockAttnParams {
     uint32_t stage_bytes;
 };
 
+// Launches kernel<<<grid, block, smem, stream>>>(args...), allowed to start
+// early behind the previous kernel on the stream when pdl is set (the kernel
+// calls pdl_wait() before reading earlier results).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                     Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // cuTensorMapEncodeTiled, fetched from the driver once (null if unavailable).
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
@@ -169,12 +188,12 @@ struct ScoreTcHook {
     void *ctx = nullptr;
 };
 cudaError_t launch_score_tc(const ScoreTcParams &p, const void *q, const void *k_cache, int num_sms,
-                            cudaStream_t stream, const ScoreTcHook &hook);
+                            cudaStream_t stream, const ScoreTcHook &hook, bool pdl = false);
 // threads: 1024 (one CTA per SM) or 512 (shares an SM with a scorer CTA)
-cudaError_t launch_select(const SelectParams &p, cudaStream_t stream, int threads = 1024);
+cudaError_t launch_select(const SelectParams &p, cudaStream_t stream, int threads = 1024, bool pdl = false);
 size_t select_smem_bytes(int threads);
-cudaError_t launch_gather(const GatherParams &p, cudaStream_t stream);
-cudaError_t launch_certify(const CertifyParams &p, cudaStream_t stream);
+cudaError_t launch_gather(const GatherParams &p, cudaStream_t stream, bool pdl = false);
+cudaError_t launch_certify(const CertifyParams &p, cudaStream_t stream, bool pdl = false);
 bool indexer_supported(int G, int d_I);
 cudaError_t launch_indexer_scores(const IndexerScoreParams &p, int num_sms, cudaStream_t stream);
 cudaError_t launch_indexer_attn(const IndexerAttnParams &p, cudaStream_t stream);

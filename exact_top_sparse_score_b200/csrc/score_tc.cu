@@ -108,6 +108,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int *abort = reinterpret_cast<volatile int *>(&misc[1]);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_wait();  // the queries, the cache and the lengths may come from the kernel before
+    pdl_trigger();
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; s++) {
             mbar_init(&full[s], 1);
@@ -294,7 +296,7 @@ size_t smem_bytes() {
 
 template <int N>
 cudaError_t launch_n(const CUtensorMap &km, const CUtensorMap &qm, const ScoreTcParams &p, int num_sms,
-                     cudaStream_t stream, const ScoreTcHook &hook) {
+                     cudaStream_t stream, const ScoreTcHook &hook, bool pdl) {
     const size_t smem = smem_bytes<N>();
     static bool attr_set[64] = {};  // per device: the shared-memory opt-in is a function attribute
     int dev = 0;
@@ -309,8 +311,7 @@ cudaError_t launch_n(const CUtensorMap &km, const CUtensorMap &qm, const ScoreTc
         e = hook.fn(hook.ctx);  // e.g. a timing event, right before the launch
         if (e != cudaSuccess) return e;
     }
-    score_tc<N><<<num_sms, kThreads, smem, stream>>>(km, qm, p);
-    return cudaGetLastError();
+    return launch_k(pdl, score_tc<N>, dim3(num_sms), dim3(kThreads), smem, stream, km, qm, p);
 }
 
 }  // namespace
@@ -330,7 +331,7 @@ EncodeTiledFn encode_fn() {
 bool score_tc_supported(int dtype, int NQ) { return dtype == TKA_BF16 && NQ <= 128 && encode_fn() != nullptr; }
 
 cudaError_t launch_score_tc(const ScoreTcParams &p, const void *q, const void *k_cache, int num_sms,
-                            cudaStream_t stream, const ScoreTcHook &hook) {
+                            cudaStream_t stream, const ScoreTcHook &hook, bool pdl) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return cudaErrorNotSupported;
     CUtensorMap km, qm;
@@ -361,10 +362,10 @@ cudaError_t launch_score_tc(const ScoreTcParams &p, const void *q, const void *k
             return cudaErrorInvalidValue;
     }
     const int NQ = p.NQ;
-    if (NQ <= 16) return launch_n<16>(km, qm, p, num_sms, stream, hook);
-    if (NQ <= 32) return launch_n<32>(km, qm, p, num_sms, stream, hook);
-    if (NQ <= 64) return launch_n<64>(km, qm, p, num_sms, stream, hook);
-    return launch_n<128>(km, qm, p, num_sms, stream, hook);
+    if (NQ <= 16) return launch_n<16>(km, qm, p, num_sms, stream, hook, pdl);
+    if (NQ <= 32) return launch_n<32>(km, qm, p, num_sms, stream, hook, pdl);
+    if (NQ <= 64) return launch_n<64>(km, qm, p, num_sms, stream, hook, pdl);
+    return launch_n<128>(km, qm, p, num_sms, stream, hook, pdl);
 }
 
 }  // namespace tka

@@ -268,6 +268,8 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads) select_topk(SelectP
     int32_t *plus_pos = reinterpret_cast<int32_t *>(plus_x + kPlusWords);  // [kWarps][kPlusCap]
 
     const int row = blockIdx.x;
+    pdl_wait();  // the scores come from the kernel before
+    pdl_trigger();
     const int b = row / (p.Q * p.Hq), qpos = (row / p.Hq) % p.Q;
     const int seq_len = p.seq_lens[b];
     if (!seq_len_ok(seq_len, p.Q, p.L_max)) {
@@ -619,7 +621,7 @@ size_t select_smem_bytes(int threads) { return smem_words(threads / 32) * 4; }
 namespace {
 
 template <int kThreads>
-cudaError_t launch_n(const SelectParams &p, cudaStream_t stream) {
+cudaError_t launch_n(const SelectParams &p, cudaStream_t stream, bool pdl) {
     const int rows = p.B * p.Q * p.Hq;
     const size_t smem = select_smem_bytes(kThreads);
     static bool attr_set[64] = {};  // per device: the shared-memory opt-in is a function attribute
@@ -631,14 +633,13 @@ cudaError_t launch_n(const SelectParams &p, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
-    select_topk<kThreads><<<rows, kThreads, smem, stream>>>(p);
-    return cudaGetLastError();
+    return launch_k(pdl, select_topk<kThreads>, dim3(rows), dim3(kThreads), smem, stream, p);
 }
 
 }  // namespace
 
-cudaError_t launch_select(const SelectParams &p, cudaStream_t stream, int threads) {
-    return threads == 512 ? launch_n<512>(p, stream) : launch_n<1024>(p, stream);
+cudaError_t launch_select(const SelectParams &p, cudaStream_t stream, int threads, bool pdl) {
+    return threads == 512 ? launch_n<512>(p, stream, pdl) : launch_n<1024>(p, stream, pdl);
 }
 
 }  // namespace tka
