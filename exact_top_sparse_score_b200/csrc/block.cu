@@ -71,6 +71,8 @@ __device__ __forceinline__ float load1s(const T *p) {
 
 template <typename T>
 __global__ void __launch_bounds__(128) block_pool(BlockPoolParams p) {
+    pdl_wait();  // inputs may come from the kernel before
+    pdl_trigger();
     const int j = blockIdx.x, bh = blockIdx.y, b = bh / p.Hkv;
     const int seq_len = p.seq_lens[b];
     if (seq_len < 1 || seq_len > p.L_max) {
@@ -94,6 +96,8 @@ constexpr int kSelThreads = 256;
 // a thread keeps both of its blocks' loads in flight before any arithmetic.
 template <typename T>
 __global__ void __launch_bounds__(kSelThreads) block_scores(BlockSelectParams p) {
+    pdl_wait();  // inputs may come from the kernel before
+    pdl_trigger();
     extern __shared__ float4 qs[];  // [G][32]: the group's query rows as fp32
     const int bh = blockIdx.y, b = bh / p.Hkv, kvh = bh - b * p.Hkv;
     const int seq_len = p.seq_lens[b];
@@ -142,6 +146,8 @@ __global__ void __launch_bounds__(kSelThreads) block_scores(BlockSelectParams p)
 // are then compacted in block order, the blocks whose key equals T kept from
 // the lowest index up.
 __global__ void __launch_bounds__(kSelThreads) block_topk(BlockSelectParams p) {
+    pdl_wait();  // inputs may come from the kernel before
+    pdl_trigger();
     extern __shared__ uint32_t ukey[];  // [ncomp]
     __shared__ uint32_t hist[256];
     __shared__ uint32_t tmp[32];
@@ -218,6 +224,8 @@ __global__ void __launch_bounds__(kSelThreads) block_topk(BlockSelectParams p) {
 // candidates are a prefix of the row, whose length slot 0 records.
 template <typename T>
 __global__ void __launch_bounds__(128) hisa_scores(HisaScoreParams p) {
+    pdl_wait();  // inputs may come from the kernel before
+    pdl_trigger();
     const int slot = blockIdx.x, row = blockIdx.y, b = row / p.Hq, h = row - b * p.Hq;
     const int seq_len = p.seq_lens[b];
     if (seq_len < 1 || seq_len > p.L_max) return;  // block_topk raised the status
@@ -331,6 +339,8 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
 template <typename T>
 __global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
     block_attn(const __grid_constant__ CUtensorMap kmap, BlockAttnParams p) {
+    pdl_wait();  // inputs may come from the kernel before
+    pdl_trigger();
     extern __shared__ unsigned char smem_raw[];
     __shared__ AttnShared sh;
     constexpr bool kBf16 = sizeof(T) == 2;
@@ -661,11 +671,8 @@ cudaError_t allow_smem(F *kernel, size_t smem) {
 
 cudaError_t launch_block_pool(const BlockPoolParams &p, cudaStream_t stream) {
     const dim3 grid(p.nblk_max, p.B * p.Hkv);
-    if (p.dtype == TKA_BF16)
-        block_pool<__nv_bfloat16><<<grid, 128, 0, stream>>>(p);
-    else
-        block_pool<float><<<grid, 128, 0, stream>>>(p);
-    return cudaGetLastError();
+    if (p.dtype == TKA_BF16) return launch_k(true, block_pool<__nv_bfloat16>, grid, dim3(128), 0, stream, p);
+    return launch_k(true, block_pool<float>, grid, dim3(128), 0, stream, p);
 }
 
 cudaError_t launch_block_select(const BlockSelectParams &p, cudaStream_t stream) {
@@ -674,25 +681,21 @@ cudaError_t launch_block_select(const BlockSelectParams &p, cudaStream_t stream)
     cudaError_t e;
     if (p.dtype == TKA_BF16) {
         if ((e = allow_smem(block_scores<__nv_bfloat16>, qsmem)) != cudaSuccess) return e;
-        block_scores<__nv_bfloat16><<<sgrid, kSelThreads, qsmem, stream>>>(p);
+        e = launch_k(true, block_scores<__nv_bfloat16>, sgrid, dim3(kSelThreads), qsmem, stream, p);
     } else {
         if ((e = allow_smem(block_scores<float>, qsmem)) != cudaSuccess) return e;
-        block_scores<float><<<sgrid, kSelThreads, qsmem, stream>>>(p);
+        e = launch_k(true, block_scores<float>, sgrid, dim3(kSelThreads), qsmem, stream, p);
     }
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (e != cudaSuccess) return e;
     const size_t ksmem = (size_t)p.nblk_max * sizeof(uint32_t);
     if ((e = allow_smem(block_topk, ksmem)) != cudaSuccess) return e;
-    block_topk<<<p.B * p.Hq, kSelThreads, ksmem, stream>>>(p);
-    return cudaGetLastError();
+    return launch_k(true, block_topk, dim3(p.B * p.Hq), dim3(kSelThreads), ksmem, stream, p);
 }
 
 cudaError_t launch_hisa_scores(const HisaScoreParams &p, cudaStream_t stream) {
     const dim3 grid(p.top_blocks, p.B * p.Hq);
-    if (p.dtype == TKA_BF16)
-        hisa_scores<__nv_bfloat16><<<grid, 128, 0, stream>>>(p);
-    else
-        hisa_scores<float><<<grid, 128, 0, stream>>>(p);
-    return cudaGetLastError();
+    if (p.dtype == TKA_BF16) return launch_k(true, hisa_scores<__nv_bfloat16>, grid, dim3(128), 0, stream, p);
+    return launch_k(true, hisa_scores<float>, grid, dim3(128), 0, stream, p);
 }
 
 cudaError_t launch_block_attn(const BlockAttnParams &p0, const void *k_cache, int num_sms, cudaStream_t stream) {
@@ -720,12 +723,10 @@ cudaError_t launch_block_attn(const BlockAttnParams &p0, const void *k_cache, in
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
         if ((e = allow_smem(block_attn<__nv_bfloat16>, smem)) != cudaSuccess) return e;
-        block_attn<__nv_bfloat16><<<grid, kAttnThreads, smem, stream>>>(kmap, p);
-    } else {
-        if ((e = allow_smem(block_attn<float>, smem)) != cudaSuccess) return e;
-        block_attn<float><<<grid, kAttnThreads, smem, stream>>>(kmap, p);
+        return launch_k(true, block_attn<__nv_bfloat16>, dim3(grid), dim3(kAttnThreads), smem, stream, kmap, p);
     }
-    return cudaGetLastError();
+    if ((e = allow_smem(block_attn<float>, smem)) != cudaSuccess) return e;
+    return launch_k(true, block_attn<float>, dim3(grid), dim3(kAttnThreads), smem, stream, kmap, p);
 }
 
 }  // namespace tka

@@ -29,6 +29,8 @@ constexpr int kIdxChunk = 128;  // index keys per CTA iteration
 
 template <typename T, int DI>
 __global__ void __launch_bounds__(128) indexer_scores(IndexerScoreParams p) {
+    pdl_wait();  // inputs may come from the kernel before
+    pdl_trigger();
     extern __shared__ float smem[];
     const int NQ = p.Q * p.H_I;
     float *qs = smem;                 // [NQ][DI]
@@ -101,6 +103,8 @@ __global__ void __launch_bounds__(128) indexer_scores(IndexerScoreParams p) {
 // I = sum_j w_j ReLU(raw_j) from the raw per-head dots the tensor-core scorer
 // wrote ([B*Q*H_I, ld], head-minor rows): grid (key chunks of 256, b * Q).
 __global__ void __launch_bounds__(256) indexer_combine(IndexerScoreParams p, const float *raw) {
+    pdl_wait();  // inputs may come from the kernel before
+    pdl_trigger();
     __shared__ float ws[256];
     const int bq = blockIdx.y, b = bq / p.Q, qpos = bq - b * p.Q;
     const int seq_len = p.seq_lens[b];
@@ -125,6 +129,8 @@ constexpr int kMaxG = 16;  // heads per kv-head held in registers (G <= kMaxG)
 
 template <typename T, int GG>
 __global__ void __launch_bounds__(kAttnWarps * 32) indexer_attn(IndexerAttnParams p) {
+    pdl_wait();  // inputs may come from the kernel before
+    pdl_trigger();
     __shared__ float sm_ml[kAttnWarps][GG][2];
     __shared__ float sm_acc[kAttnWarps][GG][kHeadDim];
     __shared__ unsigned s_ticket;
@@ -254,24 +260,21 @@ cudaError_t launch_scores_di(const IndexerScoreParams &p, int num_sms, cudaStrea
         if (smem > 48 * 1024 && (e = cudaFuncSetAttribute(indexer_scores<__nv_bfloat16, DI>,
                                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
             return e;
-        indexer_scores<__nv_bfloat16, DI><<<grid, 128, smem, stream>>>(p);
+        return launch_k(true, indexer_scores<__nv_bfloat16, DI>, grid, dim3(128), smem, stream, p);
     } else {
         if (smem > 48 * 1024 && (e = cudaFuncSetAttribute(indexer_scores<float, DI>,
                                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
             return e;
-        indexer_scores<float, DI><<<grid, 128, smem, stream>>>(p);
+        return launch_k(true, indexer_scores<float, DI>, grid, dim3(128), smem, stream, p);
     }
-    return cudaGetLastError();
 }
 
 template <int GG>
 cudaError_t launch_attn_g(const IndexerAttnParams &p, cudaStream_t stream) {
     const dim3 grid(p.splits, p.B * p.Q * p.Hkv);
     if (p.dtype == TKA_BF16)
-        indexer_attn<__nv_bfloat16, GG><<<grid, kAttnWarps * 32, 0, stream>>>(p);
-    else
-        indexer_attn<float, GG><<<grid, kAttnWarps * 32, 0, stream>>>(p);
-    return cudaGetLastError();
+        return launch_k(true, indexer_attn<__nv_bfloat16, GG>, grid, dim3(kAttnWarps * 32), 0, stream, p);
+    return launch_k(true, indexer_attn<float, GG>, grid, dim3(kAttnWarps * 32), 0, stream, p);
 }
 
 }  // namespace
@@ -284,8 +287,7 @@ cudaError_t launch_indexer_scores(const IndexerScoreParams &p, int num_sms, cuda
 
 cudaError_t launch_indexer_combine(const IndexerScoreParams &p, const float *raw, cudaStream_t stream) {
     const dim3 grid((p.L_max + 255) / 256, p.B * p.Q);
-    indexer_combine<<<grid, 256, 0, stream>>>(p, raw);
-    return cudaGetLastError();
+    return launch_k(true, indexer_combine, grid, dim3(256), 0, stream, p, raw);
 }
 
 cudaError_t launch_indexer_attn(const IndexerAttnParams &p, cudaStream_t stream) {

@@ -54,6 +54,8 @@ __device__ __forceinline__ size_t global_row(const ScoreParams &p, int b, int kv
 // NT = number of 8-wide query tiles (Q*G <= 8*NT).
 template <int NT>
 __global__ void __launch_bounds__(128) score_bf16_mma(ScoreParams p) {
+    pdl_wait();  // inputs may come from the kernel before
+    pdl_trigger();
     // q fragments, pre-permuted: [nt][step][lane] -> (b0, b1)
     __shared__ uint2 qfrag[NT][8][32];
     const int bh = blockIdx.y, b = bh / p.Hkv, kvh = bh - b * p.Hkv;
@@ -144,6 +146,8 @@ __global__ void __launch_bounds__(128) score_bf16_mma(ScoreParams p) {
 // CUDA-core scorer for any dtype and any number of query rows per kv-head.
 template <typename T>
 __global__ void __launch_bounds__(128) score_generic(ScoreParams p) {
+    pdl_wait();  // inputs may come from the kernel before
+    pdl_trigger();
     extern __shared__ float qs[];  // [NQ][128] fp32
     const int bh = blockIdx.y, b = bh / p.Hkv, kvh = bh - b * p.Hkv;
     const int seq_len = p.seq_lens[b];
@@ -220,27 +224,20 @@ cudaError_t launch_score(const ScoreParams &p, int num_sms, cudaStream_t stream)
     if (gx < 1) gx = 1;
     const dim3 grid(gx, units);
     if (p.dtype == TKA_BF16 && NQ <= 64 && p.pages.table == nullptr) {  // paged caches take score_generic
-        if (NQ <= 8)
-            score_bf16_mma<1><<<grid, 128, 0, stream>>>(p);
-        else if (NQ <= 16)
-            score_bf16_mma<2><<<grid, 128, 0, stream>>>(p);
-        else if (NQ <= 32)
-            score_bf16_mma<4><<<grid, 128, 0, stream>>>(p);
-        else
-            score_bf16_mma<8><<<grid, 128, 0, stream>>>(p);
-        return cudaGetLastError();
+        if (NQ <= 8) return launch_k(true, score_bf16_mma<1>, grid, dim3(128), 0, stream, p);
+        if (NQ <= 16) return launch_k(true, score_bf16_mma<2>, grid, dim3(128), 0, stream, p);
+        if (NQ <= 32) return launch_k(true, score_bf16_mma<4>, grid, dim3(128), 0, stream, p);
+        return launch_k(true, score_bf16_mma<8>, grid, dim3(128), 0, stream, p);
     }
     const size_t smem = (size_t)NQ * kHeadDim * sizeof(float);
     if (p.dtype == TKA_BF16) {
         if (smem > 48 * 1024)
             cudaFuncSetAttribute(score_generic<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        score_generic<__nv_bfloat16><<<grid, 128, smem, stream>>>(p);
-    } else {
-        if (smem > 48 * 1024)
-            cudaFuncSetAttribute(score_generic<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        score_generic<float><<<grid, 128, smem, stream>>>(p);
+        return launch_k(true, score_generic<__nv_bfloat16>, grid, dim3(128), smem, stream, p);
     }
-    return cudaGetLastError();
+    if (smem > 48 * 1024)
+        cudaFuncSetAttribute(score_generic<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    return launch_k(true, score_generic<float>, grid, dim3(128), smem, stream, p);
 }
 
 }  // namespace tka
