@@ -102,6 +102,22 @@ def test_scores_rising_with_position(rise, cuda_device):
     check_token(w, 1024, out, idx, tail, oracle.topk_attn(w, 1024))
 
 
+@pytest.mark.parametrize("B", [1, 5])
+def test_all_scores_equal(B, cuda_device):
+    # one key row repeated along every sequence: every score of a row ties, the
+    # sampled band holds the whole row (more candidates than the per-warp lists
+    # take), and the exact multi-pass route keeps the lowest k positions; B = 5
+    # gives more rows than SMs (512-thread rows), B = 1 the 1024-thread rows
+    L, k = 20000, 1024
+    w = workloads.make_workload(B, 1, 32, 8, L, dtype="bf16", seed=8)
+    w.k_cache[:] = w.k_cache[:, :, :1].expand_as(w.k_cache)
+    out, idx, tail = run_token(w, k)
+    ref = oracle.topk_attn(w, k)
+    assert np.array_equal(idx.cpu().numpy(), ref["idx"])
+    assert (idx.cpu()[..., :] == torch.arange(k, dtype=torch.int32)).all()
+    check_token(w, k, out, idx, tail, ref)
+
+
 def test_repeat_calls_are_bitwise_identical(cuda_device):
     w = workloads.make_workload(2, 1, 32, 8, 3000, dtype="bf16", seed=6)
     q, kc, vc, lens = to_device(w)
