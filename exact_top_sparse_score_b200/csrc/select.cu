@@ -304,8 +304,13 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads) select_topk(SelectP
     auto load_into = [&](auto off_c, auto cnt_c, int n0) {
         constexpr int off = decltype(off_c)::value, cnt = decltype(cnt_c)::value;
         const int p0 = lo + 32 * n0 + lane;
+        if (lo + 32 * (n0 + cnt) <= hi) {  // the whole part lies in the segment (every part but the last)
 #pragma unroll
-        for (int r = 0; r < cnt; r++) x[off + r] = p0 + 32 * r < hi ? __ldcg(s + p0 + 32 * r) : -INFINITY;
+            for (int r = 0; r < cnt; r++) x[off + r] = __ldcg(s + p0 + 32 * r);
+        } else {
+#pragma unroll
+            for (int r = 0; r < cnt; r++) x[off + r] = p0 + 32 * r < hi ? __ldcg(s + p0 + 32 * r) : -INFINITY;
+        }
     };
     using C0 = std::integral_constant<int, 0>;
     using CS = std::integral_constant<int, kStep>;
