@@ -413,6 +413,10 @@ def run_ours(args, world, rank, local):
         h2d = q_host.numel() * q_host.element_size() + lens_host.numel() * 4
         d2h = sum(t.numel() * t.element_size() for t in outs)
         e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+        idx_ready = [torch.cuda.Event() for _ in range(K)]
+        for e in idx_ready:
+            e.record()  # torch creates the CUDA event on its first record
+        side = torch.cuda.Stream(device=dev)
         for i in range(K):
             l2_flush()
             e2e_ev[i][0].record()
@@ -434,9 +438,18 @@ def run_ours(args, world, rank, local):
                 tka.topk_indexer_attn_decode(q_step, kc, vc, i_q, i_w, i_k, lens_step, k, out=out, idx=i_idx,
                                              workspace=ws)
             else:
-                tka.topk_attn_decode(q_step, kc, vc, lens_step, k, out=out, idx=idx, tail_mass=tail, workspace=ws)
-            for h, t in zip(hosts, outs):
-                h.copy_(t, non_blocking=True)
+                # idx is final once the select has run: its read-back (the
+                # largest result) overlaps the gather on a side stream
+                tka.topk_attn_decode(q_step, kc, vc, lens_step, k, out=out, idx=idx, tail_mass=tail, workspace=ws,
+                                     stage_events=[None, None, idx_ready[i], None])
+                side.wait_event(idx_ready[i])
+                with torch.cuda.stream(side):
+                    hosts[1].copy_(idx, non_blocking=True)
+            for j, (h, t) in enumerate(zip(hosts, outs)):
+                if not (staged and j == 1):
+                    h.copy_(t, non_blocking=True)
+            if staged:
+                torch.cuda.current_stream().wait_stream(side)
             e2e_ev[i][1].record()
         torch.cuda.synchronize()
         e2e_ms = sum(e[0].elapsed_time(e[1]) for e in e2e_ev)
@@ -555,6 +568,9 @@ def run_ours(args, world, rank, local):
         e2e_step = e2e_ms_max / K
         res["e2e"] = {"value": world * rows / (e2e_step / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                       "d2h_bytes_per_step": d2h, "ms_per_step": e2e_step}
+        if staged:
+            res["e2e"]["overlap"] = ("idx is read back on a side stream from the event the library records "
+                                     "after the select, while the gather runs")
     if world == 1 and not args.no_cpu_baseline:
         v, cores, sample = time_oracle(w, k, eps=args.certified_eps if certified else None)
         res["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}

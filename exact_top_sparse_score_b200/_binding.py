@@ -177,8 +177,9 @@ def topk_attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tens
                      stream=None, stage_events=None) -> Tuple[torch.Tensor, torch.Tensor, Optional[torch.Tensor]]:
     """Exact Top-k decode attention; returns (out fp32 [B,Q,Hq,d], idx int32 [B,Q,Hq,k], tail fp32 [B,Q,Hq]).
 
-    stage_events: optional four torch.cuda.Event objects recorded before score,
-    before select, before gather and after gather (topk_attn_decode_staged)."""
+    stage_events: optional four torch.cuda.Event objects (or None entries, not
+    recorded) for before score, before select, before gather (idx is final
+    there) and after gather (topk_attn_decode_staged)."""
     lib = load_library()
     shape = make_shape(q, k_cache, scale)
     B, Q, Hq, d = q.shape
@@ -210,7 +211,7 @@ def topk_attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tens
     if stage_events is None:
         rc = lib.topk_attn_decode(*args)
     else:
-        evs = (_vp * 4)(*[e.cuda_event for e in stage_events])
+        evs = (_vp * 4)(*[e.cuda_event if e is not None else None for e in stage_events])
         rc = lib.topk_attn_decode_staged(*args, evs)
     if rc:
         raise TopkAttnError("topk_attn_decode", rc)

@@ -51,6 +51,8 @@ cudaError_t record(const tka_event_t *events, int i, cudaStream_t s) {
     return cudaEventRecord(reinterpret_cast<cudaEvent_t>(events[i]), s);
 }
 
+bool has_event(const tka_event_t *events, int i) { return events && events[i]; }
+
 struct RecordCtx {
     const tka_event_t *events;
     int i;
@@ -315,7 +317,8 @@ tka_status launch_score_part(const DecodeArgs &a, int b0, int b1, cudaStream_t s
         ScoreTcHook hook;
         hook.fn = record_hook;
         hook.ctx = &rc;
-        if (launch_score_tc(tp, q, kc, a.dev->num_sms, s, hook, events == nullptr) != cudaSuccess) return TKA_ERR_CUDA;
+        if (launch_score_tc(tp, q, kc, a.dev->num_sms, s, hook, !has_event(events, 0)) != cudaSuccess)
+            return TKA_ERR_CUDA;
     } else {
         if (record(events, 0, s) != cudaSuccess) return TKA_ERR_CUDA;
         ScoreParams sp;
@@ -357,9 +360,8 @@ tka_status launch_rest_part(const DecodeArgs &a, int b0, int b1, cudaStream_t s,
     se.stats = stats;
     se.tail = tail;
     se.counters = counters;
-    // with no stage events between them, each kernel may start behind the one before
-    const bool pdl = events == nullptr;
-    if (launch_select(se, s, select_threads, pdl) != cudaSuccess) return TKA_ERR_CUDA;
+    // a kernel with no event recorded just before it may start behind the one before
+    if (launch_select(se, s, select_threads, !has_event(events, 1)) != cudaSuccess) return TKA_ERR_CUDA;
     if (a.cert) {
         CertifyParams cp;
         cp.status = a.dev->status;
@@ -373,7 +375,7 @@ tka_status launch_rest_part(const DecodeArgs &a, int b0, int b1, cudaStream_t s,
         cp.stats = stats;
         cp.tail = tail;
         cp.k_used = k_used;
-        if (launch_certify(cp, s, pdl) != cudaSuccess) return TKA_ERR_CUDA;
+        if (launch_certify(cp, s, true) != cudaSuccess) return TKA_ERR_CUDA;
     }
     if (record(events, 2, s) != cudaSuccess) return TKA_ERR_CUDA;
 
@@ -402,7 +404,7 @@ tka_status launch_rest_part(const DecodeArgs &a, int b0, int b1, cudaStream_t s,
     if (splits < 1) splits = 1;
     gp.per_split = (a.k + splits - 1) / splits;
     gp.splits = (a.k + gp.per_split - 1) / gp.per_split;
-    if (launch_gather(gp, s, pdl) != cudaSuccess) return TKA_ERR_CUDA;
+    if (launch_gather(gp, s, !has_event(events, 2)) != cudaSuccess) return TKA_ERR_CUDA;
     return TKA_OK;
 }
 

@@ -101,8 +101,11 @@ tka_status topk_attn_decode(const tka_shape *shape, const void *q, const void *k
 /* Same as topk_attn_decode, and additionally records the caller's CUDA events
  * (cudaEvent_t, created by the caller) on `stream` around the three kernels:
  * events[0] before the score kernel, events[1] between score and select,
- * events[2] between select and gather, events[3] after gather.  Used to time
- * each step inside a benchmark without changing what runs. */
+ * events[2] between select and gather (idx is final there: a caller may start
+ * copying it out while the gather runs), events[3] after gather.  Any entry
+ * may be null (not recorded).  Used to time each step, or to overlap the idx
+ * read-back with the gather, without changing what runs; a kernel that follows
+ * a recorded event does not start early behind the kernel before it. */
 typedef struct CUevent_st *tka_event_t;
 tka_status topk_attn_decode_staged(const tka_shape *shape, const void *q, const void *k_cache,
                                    const void *v_cache, const int32_t *seq_lens, int32_t k, float *out,

@@ -130,6 +130,27 @@ def test_repeat_calls_are_bitwise_identical(cuda_device):
         assert torch.equal(x, y)
 
 
+def test_partial_stage_events(cuda_device):
+    # only the after-select event recorded (the idx read-back overlapping the
+    # gather): same results as the plain call, and idx is final at the event
+    w = workloads.make_workload(4, 1, 32, 8, 6000, dtype="bf16", seed=9)
+    q, kc, vc, lens = to_device(w)
+    a = [t.clone() for t in tka.topk_attn_decode(q, kc, vc, lens, 512)]
+    ev = torch.cuda.Event()
+    ev.record()
+    side = torch.cuda.Stream()
+    out, idx, tail = tka.topk_attn_decode(q, kc, vc, lens, 512, stage_events=[None, None, ev, None])
+    side.wait_event(ev)
+    with torch.cuda.stream(side):
+        idx_copy = idx.clone()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    assert tka.topk_attn_device_status() == 0
+    for x, y in zip(a, (out, idx, tail)):
+        assert torch.equal(x, y)
+    assert torch.equal(idx_copy, a[1])
+
+
 def test_non_default_stream(cuda_device):
     w = workloads.make_workload(1, 1, 8, 2, 1200, dtype="bf16", seed=7)
     q, kc, vc, lens = to_device(w)
