@@ -27,6 +27,7 @@
 // makes the other roles stop, drains the copies and MMAs in flight, frees
 // TMEM and returns.
 #include <cuda.h>
+#include <string.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -90,17 +91,25 @@ struct TileWalk {
     }
 };
 
+// 32 or 64 query columns: the epilogue stages each tile's scores in shared
+// memory and one TMA store writes them (a 3-D box [Q][G][128 keys] of the
+// scores viewed as [B*Q, Hq, ld]); fewer columns store straight from registers
+__host__ __device__ constexpr bool tma_store_for(int N) { return N == 32 || N == 64; }
+
 template <int N>
 __global__ void __launch_bounds__(kThreads, 1)
-    score_tc(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap, ScoreTcParams p) {
+    score_tc(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
+             const __grid_constant__ CUtensorMap smap, ScoreTcParams p) {
     constexpr int S = stages_for(N);
     constexpr uint32_t kCols = tmem_cols_for(N);
     constexpr int kQBuf = N * 256;  // two 64-dim blocks of N rows x 128 B
+    constexpr int kOutBytes = tma_store_for(N) ? N * kTileKeys * 4 : 0;  // one tile of scores, [n][key]
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *stages = base;
     uint8_t *qbuf = stages + S * kTileBytes;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(qbuf + 2 * kQBuf);
+    float *outbuf = reinterpret_cast<float *>(qbuf + 2 * kQBuf);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(qbuf + 2 * kQBuf + kOutBytes);
     uint64_t *full = bars, *empty = bars + S, *qfull = bars + 2 * S, *qempty = qfull + 2, *tfull = qempty + 2,
              *tempty = tfull + 2, *drain = tempty + 2;
     uint32_t *misc = reinterpret_cast<uint32_t *>(drain + 1);
@@ -131,6 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         prefetch_tensormap(&kmap);
         prefetch_tensormap(&qmap);
+        if (tma_store_for(N)) prefetch_tensormap(&smap);
         if (blockIdx.x == 0)
             for (int b = 0; b < p.B; b++)
                 if (!seq_len_ok(p.seq_lens[b], p.Q, p.L_max)) raise_status(p.status, TKA_DEV_BAD_SEQ_LEN);
@@ -221,6 +231,49 @@ __global__ void __launch_bounds__(kThreads, 1)
             int no_abort = 0;
             if (!mbar_wait(drain, 0, reinterpret_cast<volatile int *>(&no_abort))) ok = false;
         }
+    } else if (tma_store_for(N)) {
+        // each tile: TMEM -> registers -> the shared-memory tile (column n at
+        // [n][key]); the 128 epilogue threads decide together whether to go
+        // on (a barrier that ANDs their waits: no thread is left behind at
+        // the barriers below), the accumulator is released as soon as it has
+        // been read, and one thread stores the tile with TMA once the previous
+        // store has finished reading the buffer.  Scores a causal query
+        // position cannot see are stored too: nothing reads them.
+        const int quarter = warp & 3;  // TMEM lanes [32*quarter, +32)
+        const uint32_t tlane = (uint32_t)(quarter * 32) << 16;
+        const int kq = quarter * 32 + lane;
+        const bool issuer = warp == 2 && lane == 0;
+        const float scale = p.scale;
+        for (int i = 0; i < w.count; i++) {
+            const int b = w.bh / p.Hkv, kvh = w.bh - b * p.Hkv;
+            const int buf = i & 1;
+            ok = mbar_wait(&tfull[buf], (i >> 1) & 1, abort);
+            ok = named_bar_and(1, 128, ok);
+            if (!ok) break;
+            tc_fence_after();
+            if (issuer) bulk_wait_read_all();
+            named_bar_sync(1, 128);  // the buffer is free
+#pragma unroll
+            for (int c = 0; c < N / 16; c++) {
+                if (c * 16 >= p.NQ) break;
+                uint32_t r[16];
+                tmem_ld16(tmem + tlane + buf * N + c * 16, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; j++)
+                    if (c * 16 + j < p.NQ) outbuf[(c * 16 + j) * kTileKeys + kq] = __uint_as_float(r[j]) * scale;
+            }
+            tc_fence_before();
+            mbar_arrive(&tempty[buf]);
+            fence_proxy_async_shared();
+            named_bar_sync(1, 128);  // the tile is complete
+            if (issuer) {
+                tma_store_3d(&smap, outbuf, w.t * kTileKeys, kvh * p.G, b * p.Q);
+                bulk_commit_group();
+            }
+            w.next(p);
+        }
+        if (issuer) bulk_wait_all();  // the shared tile outlives every store reading it
     } else {
         const int quarter = warp & 3;      // TMEM lanes [32*quarter, +32)
         const uint32_t tlane = (uint32_t)(quarter * 32) << 16;
@@ -291,12 +344,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int N>
 size_t smem_bytes() {
     constexpr int S = stages_for(N);
-    return 1024 + (size_t)S * kTileBytes + 2 * (size_t)N * 256 + (2 * S + 9) * 8 + 64;
+    return 1024 + (size_t)S * kTileBytes + 2 * (size_t)N * 256 + (tma_store_for(N) ? (size_t)N * kTileKeys * 4 : 0) +
+           (2 * S + 9) * 8 + 64;
 }
 
 template <int N>
-cudaError_t launch_n(const CUtensorMap &km, const CUtensorMap &qm, const ScoreTcParams &p, int num_sms,
-                     cudaStream_t stream, const ScoreTcHook &hook, bool pdl) {
+cudaError_t launch_n(const CUtensorMap &km, const CUtensorMap &qm, const CUtensorMap &sm, const ScoreTcParams &p,
+                     int num_sms, cudaStream_t stream, const ScoreTcHook &hook, bool pdl) {
     const size_t smem = smem_bytes<N>();
     static bool attr_set[64] = {};  // per device: the shared-memory opt-in is a function attribute
     int dev = 0;
@@ -311,7 +365,7 @@ cudaError_t launch_n(const CUtensorMap &km, const CUtensorMap &qm, const ScoreTc
         e = hook.fn(hook.ctx);  // e.g. a timing event, right before the launch
         if (e != cudaSuccess) return e;
     }
-    return launch_k(pdl, score_tc<N>, dim3(num_sms), dim3(kThreads), smem, stream, km, qm, p);
+    return launch_k(pdl, score_tc<N>, dim3(num_sms), dim3(kThreads), smem, stream, km, qm, sm, p);
 }
 
 }  // namespace
@@ -362,10 +416,23 @@ cudaError_t launch_score_tc(const ScoreTcParams &p, const void *q, const void *k
             return cudaErrorInvalidValue;
     }
     const int NQ = p.NQ;
-    if (NQ <= 16) return launch_n<16>(km, qm, p, num_sms, stream, hook, pdl);
-    if (NQ <= 32) return launch_n<32>(km, qm, p, num_sms, stream, hook, pdl);
-    if (NQ <= 64) return launch_n<64>(km, qm, p, num_sms, stream, hook, pdl);
-    return launch_n<128>(km, qm, p, num_sms, stream, hook, pdl);
+    CUtensorMap sm;
+    memset(&sm, 0, sizeof(sm));
+    if (NQ > 16 && NQ <= 64) {
+        // the scores as [B*Q, Hq, ld] fp32; one box = 128 keys of the G heads of a kv-head at all Q positions
+        const cuuint64_t dims[3] = {(cuuint64_t)p.ld, (cuuint64_t)p.Hq, (cuuint64_t)p.B * p.Q};
+        const cuuint64_t strides[2] = {(cuuint64_t)p.ld * 4, (cuuint64_t)p.Hq * p.ld * 4};
+        const cuuint32_t box[3] = {(cuuint32_t)kTileKeys, (cuuint32_t)p.G, (cuuint32_t)p.Q};
+        const cuuint32_t es[3] = {1, 1, 1};
+        if (enc(&sm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, p.scores, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    if (NQ <= 16) return launch_n<16>(km, qm, sm, p, num_sms, stream, hook, pdl);
+    if (NQ <= 32) return launch_n<32>(km, qm, sm, p, num_sms, stream, hook, pdl);
+    if (NQ <= 64) return launch_n<64>(km, qm, sm, p, num_sms, stream, hook, pdl);
+    return launch_n<128>(km, qm, sm, p, num_sms, stream, hook, pdl);
 }
 
 }  // namespace tka
