@@ -239,6 +239,16 @@ __device__ void select_multipass(const SelectParams &p, int row, int vis, const 
     finish_row(p, row, m, zk, zt, base_sel, (uint32_t)k, sm);
 }
 
+// Two 32-bit shared-memory stores, both made only when p holds.
+__device__ __forceinline__ void st_shared_if(bool p, void *a, uint32_t va, void *b, uint32_t vb) {
+    asm volatile(
+        "{\n .reg .pred q;\n setp.ne.u32 q, %0, 0;\n @q st.shared.u32 [%1], %2;\n @q st.shared.u32 [%3], %4;\n}\n" ::"r"(
+            (uint32_t)p),
+        "r"(static_cast<uint32_t>(__cvta_generic_to_shared(a))), "r"(va),
+        "r"(static_cast<uint32_t>(__cvta_generic_to_shared(b))), "r"(vb)
+        : "memory");
+}
+
 __device__ __forceinline__ uint32_t lanemask_lt() {
     uint32_t m;
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
@@ -432,16 +442,14 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads) select_topk(SelectP
             nwin += above;
             const bool plus = xv >= lo_t;
             const uint32_t pb = __ballot_sync(0xffffffffu, plus);
-            if (plus) {
-                const uint32_t slot = nplus + __popc(pb & lt);
-                if (slot < (uint32_t)kPlusCap) {
-                    my_px[slot] = xv;
-                    my_pp[slot] = p0 + 32 * r;
-                }
-                if (!above) {
-                    const uint32_t cs = atomicAdd(&wstat[warp * 8 + 1], 1u);
-                    if (cs < (uint32_t)kWarpCand) my_key[cs] = __float_as_uint(xv);  // converted when ranked
-                }
+            // the ordered list's slot for this lane; the two stores are
+            // predicated (no branch per round)
+            const uint32_t slot = nplus + __popc(pb & lt);
+            st_shared_if(plus && slot < (uint32_t)kPlusCap, my_px + slot, __float_as_uint(xv), my_pp + slot,
+                         (uint32_t)(p0 + 32 * r));
+            if (plus && !above) {
+                const uint32_t cs = atomicAdd(&wstat[warp * 8 + 1], 1u);
+                if (cs < (uint32_t)kWarpCand) my_key[cs] = __float_as_uint(xv);  // converted when ranked
             }
             nplus += __popc(pb);
         }
