@@ -156,6 +156,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         if (lane == 0) {
             const uint64_t evict_first = policy_evict_first();
+            // paged cache: a tile is box_rows-row pieces of one or more pages;
+            // the physical pages of a tile's pieces are read one tile ahead
+            // (independent loads, their latency hidden behind the copies of
+            // the tile before); a piece past the sequence end rereads its last
+            // page (those keys are never stored)
+            constexpr int kMaxPieces = kTileKeys / 16;  // pages hold >= 16 positions
+            const bool paged = p.pages.table != nullptr;
+            const int pshift = p.pages.page_shift;
+            const int box_rows = paged ? min(1 << pshift, kTileKeys) : kTileKeys;
+            const int npieces = kTileKeys / box_rows;
+            int phys_cur[kMaxPieces], phys_nxt[kMaxPieces];
+            auto load_pages = [&](const TileWalk &t, int (&ph)[kMaxPieces]) {
+                const int b = t.bh / p.Hkv;
+                const int lastp = max(p.seq_lens[b] - 1, 0) >> pshift;
+                const int32_t *trow = p.pages.table + (size_t)b * p.pages.max_pages;
+#pragma unroll
+                for (int piece = 0; piece < kMaxPieces; piece++)
+                    if (piece < npieces) ph[piece] = __ldg(trow + min((t.t * kTileKeys + piece * box_rows) >> pshift, lastp));
+            };
+            // pages of a tile or more: one piece, its page read right before its copies
+            const bool ahead = paged && npieces > 1;
+            if (ahead && w.count > 0) load_pages(w, phys_cur);
             int seg = 0;
             for (int i = 0; i < w.count && ok; i++) {
                 const int b = w.bh / p.Hkv, kvh = w.bh - b * p.Hkv;
@@ -178,19 +200,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_load_2d_hint(stages + s * kTileBytes, &kmap, &full[s], 0, row0, evict_first);
                     tma_load_2d_hint(stages + s * kTileBytes + kKBlockBytes, &kmap, &full[s], 64, row0, evict_first);
                 } else {
-                    // paged cache: the tile is box_rows-row pieces of one or
-                    // more pages; a piece past the sequence end rereads its
-                    // last page (those keys are never stored)
-                    const int box_rows = min(1 << p.pages.page_shift, kTileKeys);
-                    const int last = max(p.seq_lens[b] - 1, 0);
-                    for (int piece = 0; piece < kTileKeys / box_rows; piece++) {
-                        int pos = w.t * kTileKeys + piece * box_rows;
-                        if ((pos >> p.pages.page_shift) > (last >> p.pages.page_shift))
-                            pos = ((last >> p.pages.page_shift) << p.pages.page_shift) | (pos & ((1 << p.pages.page_shift) - 1));
-                        const int row0 = (int)paged_row(p.pages, p.status, p.Hkv, b, kvh, pos);
+                    if (!ahead) load_pages(w, phys_cur);
+#pragma unroll
+                    for (int piece = 0; piece < kMaxPieces; piece++) {
+                        if (piece >= npieces) break;
+                        int phys = phys_cur[piece];
+                        if ((unsigned)phys >= (unsigned)p.pages.num_pages) {
+                            raise_status(p.status, TKA_DEV_BAD_PAGE);  // page 0 is read instead
+                            phys = 0;
+                        }
+                        const int pos = w.t * kTileKeys + piece * box_rows;
+                        const int row0 = (int)((((long long)phys * p.Hkv + kvh) << pshift) + (pos & ((1 << pshift) - 1)));
                         uint8_t *dst = stages + s * kTileBytes + piece * box_rows * 128;
                         tma_load_2d_hint(dst, &kmap, &full[s], 0, row0, evict_first);
                         tma_load_2d_hint(dst + kKBlockBytes, &kmap, &full[s], 64, row0, evict_first);
+                    }
+                    // the next tile's pages, read after this tile's copies are out
+                    // (the producer issues in order: a load that waits on another
+                    // load must not hold up the copies)
+                    if (ahead && i + 1 < w.count) {
+                        TileWalk wn = w;
+                        wn.next(p);
+                        load_pages(wn, phys_nxt);
+#pragma unroll
+                        for (int piece = 0; piece < kMaxPieces; piece++) phys_cur[piece] = phys_nxt[piece];
                     }
                 }
                 misc[2] = i + 1;
