@@ -9,26 +9,29 @@
 //
 // One CTA (16 or 32 warps) per row; every warp owns a contiguous segment of
 // the row, lane l holding positions l, l + 32, ... of it, so a warp compacts 32
-// consecutive positions at a time with one ballot.  A segment is streamed in
-// batches of 32 x 32 positions with all loads of a batch in flight together
-// (a segment that fits one batch is read once and kept in registers for all
-// passes); the rows come from L2.  Ranks are taken on order-preserving uint32
-// keys with -0 folded into +0 (canon_key), so key order is float order and
-// the per-position tests below are plain float comparisons:
-//   pass 1  the row maximum and the histogram of the top 11 key bits of a
-//           sample (every eighth group of 32 positions) give a bin range that
-//           holds the k-th key with high probability;
-//   pass 2  scores above the range are counted, keys inside it are collected
-//           (unordered) into per-warp candidate lists;
+// consecutive positions at a time with one ballot.  A segment of up to 32 x 32
+// positions is read once and kept in registers for every pass; a longer one
+// is streamed in double-buffered steps of 16 scores per lane.  Ranks are taken
+// on order-preserving uint32 keys with -0 folded into +0 (canon_key), so key
+// order is float order and the per-position tests below are plain float
+// comparisons:
+//   pass 1  the histogram of the top 11 key bits of a sample (every eighth
+//           group of 32 positions) gives a bin range that holds the k-th key
+//           with high probability;
+//   pass 2  the one pass over the whole row: the row maximum (a running
+//           maximum per lane) and sum_all e^{s-m}; scores above the range are
+//           counted, keys inside it are collected (unordered) into per-warp
+//           candidate lists, and every score at or above the range is
+//           appended with its position to a per-warp list in position order;
 //   exact radix selection over the candidates' keys, in levels of up to 11
 //           bits over the key range the band spans, yields the k-th key T
 //           and how many of the keys equal to T are kept (the lowest
 //           positions); the bins are searched by the whole block;
-//   pass 3  every score is tested against that exact rule and the kept
-//           positions are written straight to their ascending slots (warp
-//           prefix sums plus per-warp offsets), while Z_k = sum_kept e^{s-m}
-//           and Z_tail = sum_dropped e^{s-m} are accumulated; the tail mass
-//           Z_tail / (Z_k + Z_tail) is formed from the dropped terms directly.
+//   pass 3  over the ordered lists only: the kept positions are written
+//           straight to their ascending slots (ballots plus per-warp offsets)
+//           with Z_k = sum_kept e^{s-m}; Z_tail = sum_all - Z_k, and the tail
+//           mass is Z_tail / (Z_k + Z_tail).  A warp whose ordered list
+//           overflowed tests its whole segment again instead.
 // If the sampled range misses the k-th key, or a warp collects more
 // candidates than fit, the row falls back to three exact histogram passes and
 // an ordered compaction pass over the row.
