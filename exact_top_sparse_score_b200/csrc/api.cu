@@ -288,73 +288,59 @@ struct DecodeArgs {
     bool tc;
 };
 
-size_t elem_bytes(const tka_shape *s) { return s->dtype == TKA_BF16 ? 2 : 4; }
-
-// Score of sequences [b0, b1) on s (every per-sequence array offset to b0).
-tka_status launch_score_part(const DecodeArgs &a, int b0, int b1, cudaStream_t s, const tka_event_t *events) {
+// The score kernel of a decode on s.
+tka_status launch_score(const DecodeArgs &a, cudaStream_t s, const tka_event_t *events) {
     const tka_shape *sh = a.shape;
-    const size_t row0 = (size_t)b0 * sh->Q * sh->Hq, eb = elem_bytes(sh);
-    const char *q = static_cast<const char *>(a.q) + row0 * kHeadDim * eb;
-    const char *kc = static_cast<const char *>(a.k_cache);
-    PageTable pt;
-    if (a.pages) {
-        pt = *a.pages;
-        pt.table += (size_t)b0 * pt.max_pages;
-    } else {
-        kc += (size_t)b0 * sh->Hkv * sh->L_max * kHeadDim * eb;
-    }
-    float *scores = reinterpret_cast<float *>(a.ws + a.L.scores) + row0 * a.L.ld;
+    float *scores = reinterpret_cast<float *>(a.ws + a.L.scores);
     if (a.tc) {
         ScoreTcParams tp;
         tp.status = a.dev->status;
-        tp.seq_lens = a.seq_lens + b0;
+        tp.seq_lens = a.seq_lens;
         tp.scores = scores;
-        tp.B = b1 - b0; tp.Q = sh->Q; tp.Hq = sh->Hq; tp.Hkv = sh->Hkv; tp.G = a.G;
+        tp.B = sh->B; tp.Q = sh->Q; tp.Hq = sh->Hq; tp.Hkv = sh->Hkv; tp.G = a.G;
         tp.L_max = sh->L_max; tp.ld = a.L.ld; tp.NQ = sh->Q * a.G;
         tp.scale = resolve_scale(sh);
-        tp.pages = pt;
+        if (a.pages) tp.pages = *a.pages;
         RecordCtx rc{events, 0, s};
         ScoreTcHook hook;
         hook.fn = record_hook;
         hook.ctx = &rc;
-        if (launch_score_tc(tp, q, kc, a.dev->num_sms, s, hook, !has_event(events, 0)) != cudaSuccess)
+        if (launch_score_tc(tp, a.q, a.k_cache, a.dev->num_sms, s, hook, !has_event(events, 0)) != cudaSuccess)
             return TKA_ERR_CUDA;
     } else {
         if (record(events, 0, s) != cudaSuccess) return TKA_ERR_CUDA;
         ScoreParams sp;
         sp.status = a.dev->status;
-        sp.q = q;
-        sp.k = kc;
-        sp.seq_lens = a.seq_lens + b0;
+        sp.q = a.q;
+        sp.k = a.k_cache;
+        sp.seq_lens = a.seq_lens;
         sp.scores = scores;
-        sp.B = b1 - b0; sp.Q = sh->Q; sp.Hq = sh->Hq; sp.Hkv = sh->Hkv; sp.G = a.G;
+        sp.B = sh->B; sp.Q = sh->Q; sp.Hq = sh->Hq; sp.Hkv = sh->Hkv; sp.G = a.G;
         sp.L_max = sh->L_max; sp.ld = a.L.ld; sp.dtype = sh->dtype;
         sp.scale = resolve_scale(sh);
-        sp.pages = pt;
-        if (launch_score(sp, a.dev->num_sms, s) != cudaSuccess) return TKA_ERR_CUDA;
+        if (a.pages) sp.pages = *a.pages;
+        if (tka::launch_score(sp, a.dev->num_sms, s) != cudaSuccess) return TKA_ERR_CUDA;
     }
     return TKA_OK;
 }
 
-// Select (k) -> [certify] -> gather of sequences [b0, b1) on s.
-tka_status launch_rest_part(const DecodeArgs &a, int b0, int b1, cudaStream_t s, int select_threads,
-                            const tka_event_t *events) {
+// Select (k) -> [certify] -> gather of a decode on s.
+tka_status launch_rest(const DecodeArgs &a, cudaStream_t s, int select_threads, const tka_event_t *events) {
     const tka_shape *sh = a.shape;
-    const size_t row0 = (size_t)b0 * sh->Q * sh->Hq, eb = elem_bytes(sh);
-    const int rows = (b1 - b0) * sh->Q * sh->Hq;
-    const float *scores = reinterpret_cast<const float *>(a.ws + a.L.scores) + row0 * a.L.ld;
-    int32_t *idx = a.idx + row0 * a.k;
-    float *w = reinterpret_cast<float *>(a.ws + a.L.weights) + row0 * a.k;
-    float4 *stats = reinterpret_cast<float4 *>(a.ws + a.L.stats) + row0;
-    unsigned *counters = reinterpret_cast<unsigned *>(a.ws + a.L.counters) + row0;
-    float *tail = a.tail ? a.tail + row0 : nullptr;
-    int32_t *k_used = a.cert ? a.cert->k_used + row0 : nullptr;
+    const int rows = sh->B * sh->Q * sh->Hq;
+    const float *scores = reinterpret_cast<const float *>(a.ws + a.L.scores);
+    int32_t *idx = a.idx;
+    float *w = reinterpret_cast<float *>(a.ws + a.L.weights);
+    float4 *stats = reinterpret_cast<float4 *>(a.ws + a.L.stats);
+    unsigned *counters = reinterpret_cast<unsigned *>(a.ws + a.L.counters);
+    float *tail = a.tail;
+    int32_t *k_used = a.cert ? a.cert->k_used : nullptr;
 
     SelectParams se;
     se.status = a.dev->status;
     se.scores = scores;
-    se.seq_lens = a.seq_lens + b0;
-    se.B = b1 - b0; se.Q = sh->Q; se.Hq = sh->Hq; se.L_max = sh->L_max; se.ld = a.L.ld; se.k = a.k;
+    se.seq_lens = a.seq_lens;
+    se.B = sh->B; se.Q = sh->Q; se.Hq = sh->Hq; se.L_max = sh->L_max; se.ld = a.L.ld; se.k = a.k;
     se.idx = idx;
     se.w = w;
     se.stats = stats;
@@ -366,8 +352,8 @@ tka_status launch_rest_part(const DecodeArgs &a, int b0, int b1, cudaStream_t s,
         CertifyParams cp;
         cp.status = a.dev->status;
         cp.scores = scores;
-        cp.seq_lens = a.seq_lens + b0;
-        cp.B = b1 - b0; cp.Q = sh->Q; cp.Hq = sh->Hq; cp.L_max = sh->L_max; cp.ld = a.L.ld;
+        cp.seq_lens = a.seq_lens;
+        cp.B = sh->B; cp.Q = sh->Q; cp.Hq = sh->Hq; cp.L_max = sh->L_max; cp.ld = a.L.ld;
         cp.k_max = a.k;
         cp.eps = a.cert->eps;
         cp.idx = idx;
@@ -381,22 +367,18 @@ tka_status launch_rest_part(const DecodeArgs &a, int b0, int b1, cudaStream_t s,
 
     GatherParams gp;
     gp.status = a.dev->status;
-    gp.v = a.pages ? a.v_cache
-                   : static_cast<const char *>(a.v_cache) + (size_t)b0 * sh->Hkv * sh->L_max * kHeadDim * eb;
-    gp.seq_lens = a.seq_lens + b0;
-    gp.B = b1 - b0; gp.Q = sh->Q; gp.Hq = sh->Hq; gp.Hkv = sh->Hkv; gp.G = a.G;
+    gp.v = a.v_cache;
+    gp.seq_lens = a.seq_lens;
+    gp.B = sh->B; gp.Q = sh->Q; gp.Hq = sh->Hq; gp.Hkv = sh->Hkv; gp.G = a.G;
     gp.L_max = sh->L_max; gp.k = a.k; gp.dtype = sh->dtype;
     gp.idx = idx;
     gp.w = w;
     gp.stats = stats;
-    gp.partial = reinterpret_cast<float *>(a.ws + a.L.partial) + row0 * a.L.max_splits * kHeadDim;
+    gp.partial = reinterpret_cast<float *>(a.ws + a.L.partial);
     gp.counters = counters;
-    gp.out = a.out + row0 * kHeadDim;
+    gp.out = a.out;
     gp.kcount = k_used;
-    if (a.pages) {
-        gp.pages = *a.pages;
-        gp.pages.table += (size_t)b0 * gp.pages.max_pages;
-    }
+    if (a.pages) gp.pages = *a.pages;
     // one wave of eight CTAs per SM (splits = floor(8 x SMs / rows), at least 1),
     // never fewer than kMinKeysPerSplit keys per CTA
     int splits = (a.dev->num_sms * 8) / rows;
@@ -443,14 +425,14 @@ tka_status decode_impl(const tka_shape *shape, const void *q, const void *k_cach
     a.tc = score_tc_supported(shape->dtype, shape->Q * a.G) &&
            (pages || (long long)shape->B * shape->Hkv * shape->L_max < (1LL << 31));
 
-    st = launch_score_part(a, 0, shape->B, s, events);
+    st = launch_score(a, s, events);
     if (st != TKA_OK) return st;
     if (record(events, 1, s) != cudaSuccess) return TKA_ERR_CUDA;
     // more rows than SMs: 512-thread select CTAs, two rows per SM at a time
     // (a 1024-thread CTA takes a whole SM's registers, and the rows would run
     // in waves of one per SM); otherwise 1024 threads per row
     const int rows = shape->B * shape->Q * shape->Hq;
-    st = launch_rest_part(a, 0, shape->B, s, rows > a.dev->num_sms ? 512 : 1024, events);
+    st = launch_rest(a, s, rows > a.dev->num_sms ? 512 : 1024, events);
     if (st != TKA_OK) return st;
     if (record(events, 3, s) != cudaSuccess) return TKA_ERR_CUDA;
     return TKA_OK;
