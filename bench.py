@@ -9,14 +9,20 @@ Llama-3-8B-shaped GQA decode layer: B=8, 32 query / 8 KV heads, d=128,
 L=32768, k=2048, bf16 cache.
 
 Prints ONE JSON line (rank 0).  Timing: W untimed warm-up steps, then exactly
-K timed steps, each bracketed by CUDA events on the launching stream, with an
-L2 flush between steps outside the events (a 256 MiB write, then a 256 MiB
-read, so that no dirty line of the flush buffer is left in L2 to be written
-back inside the timed region); the sum of the
-K step times, max over ranks.  Multi-GPU (torchrun) runs one independent
-replica per GPU (the path shards by sequence with no exchange): weak scaling.
+K timed steps of plain API calls, each bracketed by CUDA events on the
+launching stream, with an L2 flush between steps outside the events (a 256 MiB
+write, then a 256 MiB read, so that no dirty line of the flush buffer is left
+in L2 to be written back inside the timed region); the sum of the K step
+times, max over ranks, gives `value`.  The token variant then times a second
+pass of K steps with events between its three kernels (`stage_us`, and the
+score kernel's roofline).  `e2e` repeats the K steps through the public API
+with the step's inputs copied from pinned host memory and its results copied
+back inside the events (idx on a side stream while the gather runs).
+Multi-GPU (torchrun) runs one independent replica per GPU (the path shards by
+sequence with no exchange): weak scaling.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1..5] [--impl ours|reference]
+                  [--certified-eps E | --paged P | --hisa BS,TOP | --indexer H_I,D_I]
 """
 from __future__ import annotations
 
