@@ -100,6 +100,24 @@ def alg_bytes_token(w, k, kept=None):
     return k_bytes(w) + kept * 2 * row + rows * w.d * (elem_bytes(w) + 4) + rows * (k * 4 + 4)
 
 
+def unique_kept_rows(idx, w):
+    """Kept positions counted once per (sequence, kv-head): the union over the
+    G heads and Q positions of the group (what the gather must read at least
+    once; -1 padding excluded).  idx [B, Q, Hq, k] on the device."""
+    k = idx.shape[-1]
+    g = idx.view(w.B, w.Q, w.Hkv, w.Hq // w.Hkv, k).permute(0, 2, 1, 3, 4).reshape(w.B * w.Hkv, -1)
+    srt = torch.sort(g, dim=1).values
+    new = torch.ones_like(srt, dtype=torch.bool)
+    new[:, 1:] = srt[:, 1:] != srt[:, :-1]
+    return int((new & (srt >= 0)).sum())
+
+
+def alg_bytes_unique(w, k, uniq_rows):
+    """The stricter algorithmic bytes: K once + every unique kept V row once + q, out, idx and tail."""
+    rows = w.B * w.Q * w.Hq
+    return k_bytes(w) + uniq_rows * w.d * elem_bytes(w) + rows * w.d * (elem_bytes(w) + 4) + rows * (k * 4 + 4)
+
+
 def alg_bytes_block(w):
     """Block keys (fp32) of every competing block + the kept blocks' K and V rows + q/out/block_idx."""
     bs, top = w.block_size, w.top_blocks
@@ -480,6 +498,10 @@ def run_ours(args, world, rank, local):
     total_ms, e2e_ms_max = float(vals[0]), float(vals[1])
     stage_tot = [float(x) for x in vals[2:]]
 
+    # unique kept rows from this rank's last result (token variant): the
+    # stricter bytes, counted on the device after the timing
+    alg_u = alg_bytes_unique(w, k, unique_kept_rows(idx, w)) if (staged or paged) else None
+
     if rank != 0:
         return None
     ms = total_ms / K
@@ -514,6 +536,8 @@ def run_ours(args, world, rank, local):
         "alg_gbs": alg / (ms / 1e3) / 1e9,
         "alg_frac_of_spec_8tbs": alg / (ms / 1e3) / 1e9 / SPEC_HBM_GBS,
         "alg_frac_of_measured_hbm": alg / (ms / 1e3) / 1e9 / peak,
+        **({"alg_bytes_unique_rows": alg_u, "unique_gbs": alg_u / (ms / 1e3) / 1e9,
+            "unique_frac_of_measured_hbm": alg_u / (ms / 1e3) / 1e9 / peak} if alg_u else {}),
         "gpu_launches": launches_per_step * K,
         "clocks": clocks.summary(),
     }
