@@ -97,18 +97,8 @@ __device__ __forceinline__ float warp_max(float v) {
     return v;
 }
 
-// Block-wide sum/max of one value per thread (blockDim.x multiple of 32,
-// <= 1024).  `red` is >= 32 floats of shared memory; contains a barrier.
-__device__ __forceinline__ float block_sum(float v, float *red) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    v = warp_sum(v);
-    __syncthreads();
-    if (lane == 0) red[warp] = v;
-    __syncthreads();
-    float t = lane < nw ? red[lane] : 0.f;
-    return warp_sum(t);
-}
-
+// Block-wide max of one value per thread (blockDim.x multiple of 32, <= 1024).
+// `red` is >= 32 floats of shared memory; contains two barriers.
 __device__ __forceinline__ float block_max(float v, float *red) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     v = warp_max(v);

@@ -60,35 +60,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     return false;
 }
 
-// try_wait that may suspend the thread for up to `ns` nanoseconds while the
-// phase is incomplete (the thread resumes as soon as it completes), so that a
-// waiting warp takes no issue slots from the warps doing work.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t ns) {
-    uint32_t ok;
-    asm volatile(
-        "{\n"
-        ".reg .pred p;\n"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
-        "selp.b32 %0, 1, 0, p;\n"
-        "}\n"
-        : "=r"(ok)
-        : "r"(smem_addr(bar)), "r"(parity), "r"(ns)
-        : "memory");
-    return ok != 0;
-}
-
-// mbar_wait with suspending polls of at most `ns` each; gives up after
-// kMaxSleepPolls polls or once *abort is set.
-constexpr uint32_t kMaxSleepPolls = 1u << 16;
-
-__device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity, volatile int *abort, uint32_t ns) {
-    for (uint32_t i = 0; i < kMaxSleepPolls; i++) {
-        if (mbar_try_wait_sleep(bar, parity, ns)) return true;
-        if (*abort) return false;
-    }
-    return false;
-}
-
 // ---------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int x, int y) {
