@@ -27,3 +27,42 @@ def test_unique_bytes_never_exceed_the_formula_bytes():
     u = bench.unique_kept_rows(idx, w)
     assert u == 10
     assert bench.alg_bytes_unique(w, 8, u) < bench.alg_bytes_token(w, 8, kept=4 * 8)
+
+
+def _run_bench(*args, env_extra=None):
+    import json
+    import os
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, **(env_extra or {}))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), *args], capture_output=True, text=True,
+                       cwd=root, env=env, timeout=300)
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    return r.returncode, [json.loads(l) for l in lines]
+
+
+def test_reference_arm_prints_one_contract_line():
+    rc, out = _run_bench("--impl", "reference", "--config", "1", "--steps", "3", "--warmup", "3")
+    assert rc == 0 and len(out) == 1
+    r = out[0]
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+                "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert key in r, key
+    assert r["impl"] == "reference" and r["steps"] == 3 and r["warmup"] == 3 and r["value"] > 0
+    assert r["config"]["workload"]
+    assert {"value", "unit", "cores", "kind", "sample"} <= set(r["cpu_baseline"])
+    assert r["cpu_baseline"]["kind"] == "oracle" and r["cpu_baseline"]["value"] == r["value"]
+    assert r["e2e"] == {"value": r["value"], "unit": r["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_do_no_work():
+    rc, out = _run_bench("--impl", "reference", "--config", "1", "--steps", "3", "--warmup", "3",
+                         env_extra={"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
+    assert rc == 0 and out == []
+
+
+def test_too_few_warmup_steps_are_refused():
+    rc, out = _run_bench("--impl", "reference", "--config", "1", "--steps", "3", "--warmup", "2")
+    assert rc != 0 and out == []
