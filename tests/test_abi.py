@@ -124,3 +124,34 @@ def test_binding_rejects_mismatched_output_buffers(lib):
         tka.topk_attn_decode(q, kc, kc, lens, 8, tail_mass=torch.zeros(1, 1, 3, dtype=torch.float32))
     with pytest.raises(ValueError):  # host tensors: there is no CPU path
         tka.topk_attn_decode(q, kc, kc, lens, 8)
+
+
+def test_every_entry_point_refuses_host_tensors(lib):
+    # there is no CPU path anywhere: each public call raises on host memory
+    # (before any launch) instead of computing something on the CPU
+    import torch
+    import exact_top_sparse_score_b200 as tka
+    B, Hq, Hkv, L, d = 1, 4, 2, 64, 128
+    q = torch.zeros(B, 1, Hq, d, dtype=torch.bfloat16)
+    kc = torch.zeros(B, Hkv, L, d, dtype=torch.bfloat16)
+    lens = torch.full((B,), L, dtype=torch.int32)
+    bk = torch.zeros(B, Hkv, L // 16, d, dtype=torch.float32)
+    pages = torch.zeros(L // 16 * B, Hkv, 16, d, dtype=torch.bfloat16)
+    table = torch.arange(L // 16, dtype=torch.int32).view(B, L // 16)
+    qi = torch.zeros(B, 1, 4, 64, dtype=torch.bfloat16)
+    wi = torch.zeros(B, 1, 4, dtype=torch.float32)
+    ki = torch.zeros(B, L, 64, dtype=torch.bfloat16)
+    calls = {
+        "decode": lambda: tka.topk_attn_decode(q, kc, kc, lens, 8),
+        "paged": lambda: tka.topk_attn_decode_paged(q, pages, pages, table, lens, 8),
+        "certified": lambda: tka.topk_attn_decode_certified(q, kc, kc, lens, 0.1, 8),
+        "static": lambda: tka.topk_attn_decode_static(q, kc, kc, lens, 8, out=torch.zeros(B, 1, Hq, d),
+                                                      idx=torch.zeros(B, 1, Hq, 8, dtype=torch.int32)),
+        "pool": lambda: tka.topk_block_pool_keys(kc, lens, 16),
+        "block": lambda: tka.topk_block_attn_decode(q, kc, kc, bk, lens, 16, 2),
+        "hisa": lambda: tka.topk_hisa_attn_decode(q, kc, kc, bk, lens, 16, 2, 8),
+        "indexer": lambda: tka.topk_indexer_attn_decode(q, kc, kc, qi, wi, ki, lens, 8),
+    }
+    for name, call in calls.items():
+        with pytest.raises(ValueError, match="CUDA tensor"):
+            call()
