@@ -342,7 +342,9 @@ def run_ours(args, world, rank, local):
             i_idx = torch.empty((w.B, w.Q, k), dtype=torch.int32, device=dev)
             ws = torch.empty(tka._binding.load_library().topk_indexer_attn_workspace_size(
                 make_shape(q, kc), i_h, i_d, k), dtype=torch.uint8, device=dev)
-            launches_per_step = 3  # indexer_scores, select, indexer_attn
+            # 128-dim bf16 index keys: the tensor-core scorer + the weighted ReLU combine;
+            # otherwise indexer_scores on CUDA cores; then select and indexer_attn
+            launches_per_step = 4 if (i_d == 128 and w.dtype == "bf16" and w.Q * i_h <= 128) else 3
 
             def step(events=None, qq=q):
                 if events:
