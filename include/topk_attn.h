@@ -26,6 +26,12 @@
  *   - Every data pointer is DEVICE memory owned by the caller.  The library
  *     never allocates, frees or synchronises inside a compute call; it only
  *     enqueues kernels on `stream` (a cudaStream_t; NULL = legacy default).
+ *     The kernels are launched with programmatic stream serialization (they
+ *     may be scheduled while the kernel before them on the stream finishes)
+ *     and wait for all earlier work on the stream before reading anything,
+ *     so results are ordered exactly as with plain launches.  A caller that
+ *     launches its own next kernel with that attribute must likewise wait
+ *     (griddepcontrol.wait) before reading this library's outputs.
  *   - Layouts are row-major and contiguous:
  *       q         [B, Q, Hq, d]        dtype of the cache
  *       k_cache   [B, Hkv, L_max, d]   bf16 or fp32
