@@ -97,6 +97,12 @@ __device__ __forceinline__ float warp_max(float v) {
     return v;
 }
 
+__device__ __forceinline__ float warp_min(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
 // Block-wide max of one value per thread (blockDim.x multiple of 32, <= 1024).
 // `red` is >= 32 floats of shared memory; contains two barriers.
 __device__ __forceinline__ float block_max(float v, float *red) {

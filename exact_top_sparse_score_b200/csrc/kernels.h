@@ -189,9 +189,9 @@ struct ScoreTcHook {
 };
 cudaError_t launch_score_tc(const ScoreTcParams &p, const void *q, const void *k_cache, int num_sms,
                             cudaStream_t stream, const ScoreTcHook &hook, bool pdl = false);
-// threads: 1024 (one CTA per SM) or 512 (shares an SM with a scorer CTA)
+// threads: 1024 (one row per SM) or 512 (two rows per SM)
 cudaError_t launch_select(const SelectParams &p, cudaStream_t stream, int threads = 1024, bool pdl = false);
-size_t select_smem_bytes(int threads);
+size_t select_smem_bytes(int threads, int k);
 cudaError_t launch_gather(const GatherParams &p, cudaStream_t stream, bool pdl = false);
 cudaError_t launch_certify(const CertifyParams &p, cudaStream_t stream, bool pdl = false);
 bool indexer_supported(int G, int d_I);

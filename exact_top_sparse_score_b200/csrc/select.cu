@@ -8,35 +8,31 @@
 // Top-k Sparse Attention via Total Variation Distance" (abstract).
 //
 // One CTA (16 or 32 warps) per row; every warp owns a contiguous segment of
-// the row, lane l holding positions l, l + 32, ... of it, so a warp compacts 32
-// consecutive positions at a time with one ballot.  A segment of up to 32 x 32
-// positions is read once and kept in registers for every pass; a longer one
-// is streamed in double-buffered steps of 16 scores per lane.  Ranks are taken
-// on order-preserving uint32 keys with -0 folded into +0 (canon_key), so key
-// order is float order and the per-position tests below are plain float
-// comparisons:
-//   pass 1  the histogram of the top 11 key bits of a sample (every eighth
-//           group of 32 positions) gives a bin range that holds the k-th key
-//           with high probability;
-//   pass 2  the one pass over the whole row: the row maximum (a running
-//           maximum per lane) and sum_all e^{s-m}; scores above the range are
-//           counted, keys inside it are collected (unordered) into per-warp
-//           candidate lists, and every score at or above the range is
-//           appended with its position to a per-warp list in position order;
-//   exact radix selection over the candidates' keys, in levels of up to 11
-//           bits over the key range the band spans, yields the k-th key T
-//           and how many of the keys equal to T are kept (the lowest
-//           positions); the bins are searched by the whole block;
-//   pass 3  over the ordered lists only: the kept positions are written
-//           straight to their ascending slots (ballots plus per-warp offsets)
-//           with Z_k = sum_kept e^{s-m}; Z_tail = sum_all - Z_k, and the tail
-//           mass is Z_tail / (Z_k + Z_tail).  A warp whose ordered list
-//           overflowed tests its whole segment again instead.
-// If the sampled range misses the k-th key, or a warp collects more
-// candidates than fit, the row falls back to three exact histogram passes and
-// an ordered compaction pass over the row.
-#include <type_traits>
-
+// the row, lane l reading positions l, l + 32, ... of it, so a warp compacts
+// 32 consecutive positions at a time with one ballot.  Ranks are taken on
+// order-preserving uint32 keys with -0 folded into +0 (canon_key), so key
+// order is float order and a key threshold is also a float threshold.  The
+// row is read from L2 (the scores were just written) once, after a sample:
+//   sample  the maximum and the histogram of the top 11 key bits of every
+//           eighth group of 32 positions (every position of a short row);
+//           with the next 11 key bits of the sample keys inside the coarse
+//           bin, this gives lo_t, the sample key of the k-th key's sample
+//           rank pushed down by 5 binomial standard deviations (to 2^10
+//           keys): below the k-th score with high probability;
+//   pass    the row maximum m, sum_all e^{s - m_s} against the sample maximum
+//           m_s (rescaled to m afterwards), and every score >= lo_t appended
+//           with its position to a per-warp list in position order (one
+//           ballot per 32 positions) -- a little more than k entries;
+//   the exact k-th key T among the list entries by radix levels of up to 11
+//           bits over the keys between lo_t and m, and how many of the keys
+//           equal to T are kept (the lowest positions);
+//   emit    from the lists only: every kept entry (s > T, or s = T among the
+//           first ties) to its final ascending slot, with Z_k over the kept
+//           terms; Z_tail = sum_all - Z_k, the tail mass Z_tail / (Z_k + Z_tail).
+// If fewer than k scores reach lo_t, a warp's list overflows, or the sample
+// maximum lies too far below the row maximum for the sum against it, the row
+// falls back to three exact histogram passes and an ordered compaction pass
+// over the row.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -44,16 +40,11 @@ namespace tka {
 
 namespace {
 
-// A row is taken by one CTA of kThreads threads: 1024 when the select runs
-// alone (one CTA per SM), 512 when it shares the SMs with the scorer of the
-// next batch chunk (a 512-thread CTA and a scorer CTA fit one SM's registers
-// and shared memory together).  Up to 32 warps: per-warp words are reduced by
-// one warp, lane w reading warp w's.
-constexpr int kCandWords = 8192;  // candidate keys held in shared memory per row, split evenly over the warps
-constexpr int kPlusWords = 6144;  // (score, position) pairs of the scores at or above the band, split likewise
-constexpr int kHeld = 32;  // scores per lane held in registers (a resident segment: 32 x 32 positions)
-constexpr int kStep = 16;  // scores per lane per step of a streamed segment (half the registers)
-constexpr int kSampleMinLen = 16384;            // rows this long histogram a 1/8 sample in pass 1
+// A row is taken by one CTA: 1024 threads when there are no more rows than
+// SMs (one row per SM), else 512 threads so that two rows share an SM.  Up to
+// 32 warps: per-warp words are reduced by one warp, lane w reading warp w's.
+constexpr int kU = 8;                // scores per lane per streamed chunk (two chunks in flight)
+constexpr int kS = 8;                // sampled groups of 32 positions per warp (held in registers)
 
 constexpr int kBatch = 8;  // float4 loads in flight per thread
 
@@ -242,43 +233,90 @@ __device__ void select_multipass(const SelectParams &p, int row, int vis, const 
     finish_row(p, row, m, zk, zt, base_sel, (uint32_t)k, sm);
 }
 
-// Two 32-bit shared-memory stores, both made only when p holds.
-__device__ __forceinline__ void st_shared_if(bool p, void *a, uint32_t va, void *b, uint32_t vb) {
-    asm volatile(
-        "{\n .reg .pred q;\n setp.ne.u32 q, %0, 0;\n @q st.shared.u32 [%1], %2;\n @q st.shared.u32 [%3], %4;\n}\n" ::"r"(
-            (uint32_t)p),
-        "r"(static_cast<uint32_t>(__cvta_generic_to_shared(a))), "r"(va),
-        "r"(static_cast<uint32_t>(__cvta_generic_to_shared(b))), "r"(vb)
-        : "memory");
-}
-
 __device__ __forceinline__ uint32_t lanemask_lt() {
     uint32_t m;
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
     return m;
 }
 
-__host__ __device__ constexpr size_t smem_words(int warps) {
-    return 2048 + 104 + warps * 8 + kCandWords + 2048 + 2 * kPlusWords;
+// Entries of a warp's ordered list (score, position) -- enough for twice the
+// kept positions of an evenly spread row, at least 64 -- plus one slot that
+// absorbs the writes past a full list.
+__host__ __device__ constexpr int list_cap_for(int k, int warps) {
+    const int c = (2 * k + 1024 + warps - 1) / warps;
+    return ((c < 64 ? 64 : c) + 31) & ~31;
+}
+
+__host__ __device__ constexpr size_t smem_words_for(int k, int warps) {
+    return 2048 + 104 + (size_t)warps * 8 + 2 * (size_t)warps * (list_cap_for(k, warps) + 1);
+}
+
+// A position known to lie inside the streamed range (a compile-time true).
+struct InRange {
+    __device__ __forceinline__ constexpr operator bool() const { return true; }
+};
+
+// Streams positions [lo, hi) of s through f(x, pos, valid) in chunks of
+// 32 kU positions (lane l: pos = chunk start + 32 u + l), the next chunk's
+// loads in flight while the current one is processed.  valid is the
+// compile-time constant InRange{} for every chunk that lies wholly inside the
+// range; past the range x is -inf.
+template <typename F>
+__device__ __forceinline__ void stream_range(const float *s, int lo, int hi, int lane, F &&f) {
+    const int nch = (hi - lo + 32 * kU - 1) / (32 * kU);
+    float a[kU], b[kU];
+    auto load = [&](float(&x)[kU], int c) {
+        const int p0 = lo + c * 32 * kU + lane;
+        if (lo + (c + 1) * 32 * kU <= hi) {
+#pragma unroll
+            for (int u = 0; u < kU; u++) x[u] = __ldcg(s + p0 + 32 * u);
+        } else {
+#pragma unroll
+            for (int u = 0; u < kU; u++) x[u] = p0 + 32 * u < hi ? __ldcg(s + p0 + 32 * u) : -INFINITY;
+        }
+    };
+    auto run = [&](float(&x)[kU], int c) {
+        const int p0 = lo + c * 32 * kU + lane;
+        if (lo + (c + 1) * 32 * kU <= hi) {
+#pragma unroll
+            for (int u = 0; u < kU; u++) f(x[u], p0 + 32 * u, InRange{});
+        } else {
+#pragma unroll
+            for (int u = 0; u < kU; u++) f(x[u], p0 + 32 * u, p0 + 32 * u < hi);
+        }
+    };
+    if (nch > 0) load(a, 0);
+    for (int c = 0; c < nch; c += 2) {
+        if (c + 1 < nch) load(b, c + 1);
+        run(a, c);
+        if (c + 1 < nch) {
+            if (c + 2 < nch) load(a, c + 2);
+            run(b, c + 1);
+        }
+    }
+}
+
+// A 64-bit shared-memory store {x, y} made only when p holds.
+__device__ __forceinline__ void st_shared_v2_if(bool p, void *a, uint32_t x, uint32_t y) {
+    asm volatile("{\n .reg .pred q;\n setp.ne.u32 q, %0, 0;\n @q st.shared.v2.u32 [%1], {%2, %3};\n}\n" ::"r"(
+                     (uint32_t)p),
+                 "r"(static_cast<uint32_t>(__cvta_generic_to_shared(a))), "r"(x), "r"(y)
+                 : "memory");
 }
 
 template <int kThreads>
 __global__ void __launch_bounds__(kThreads, 1024 / kThreads) select_topk(SelectParams p) {
     constexpr int kWarps = kThreads / 32;
     static_assert(kWarps <= 32 && kThreads % 32 == 0, "at most 32 whole warps");
-    constexpr int kWarpCand = kCandWords / kWarps;  // a warp's candidate list
     extern __shared__ __align__(16) uint32_t dyn[];
     SelectSmem sm;
-    sm.hist = dyn;                                                   // [2048]
-    sm.tmp = dyn + 2048;                                             // [32]
-    sm.red = reinterpret_cast<float *>(dyn + 2048 + 32);             // [64]
-    sm.scal = dyn + 2048 + 96;                                       // [8]
-    uint32_t *wstat = dyn + 2048 + 104;                              // [kWarps][8]
-    uint32_t *wc_key = wstat + kWarps * 8;                           // [kWarps][kWarpCand]
-    uint32_t *hist2 = wc_key + kWarps * kWarpCand;                   // [2048] second radix histogram
-    constexpr int kPlusCap = kPlusWords / kWarps;                    // a warp's list of scores >= the band
-    float *plus_x = reinterpret_cast<float *>(hist2 + 2048);         // [kWarps][kPlusCap]
-    int32_t *plus_pos = reinterpret_cast<int32_t *>(plus_x + kPlusWords);  // [kWarps][kPlusCap]
+    sm.hist = dyn;                                        // [2048]
+    sm.tmp = dyn + 2048;                                  // [32]
+    sm.red = reinterpret_cast<float *>(dyn + 2048 + 32);  // [64]
+    sm.scal = dyn + 2048 + 96;                            // [8]
+    uint32_t *wstat = dyn + 2048 + 104;                   // [kWarps][8]
+    const int cap = list_cap_for(p.k, kWarps);
+    uint2 *lists = reinterpret_cast<uint2 *>(wstat + kWarps * 8);  // [kWarps][cap + 1] {score bits, position}
 
     const int row = blockIdx.x;
     pdl_wait();  // the scores come from the kernel before
@@ -301,351 +339,285 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads) select_topk(SelectP
     }
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint32_t lt = lanemask_lt();
-    // this warp's contiguous segment; lane l holds positions lo + 32 r + l of
-    // it, -inf past the segment's end (so the passes below need no bounds
-    // tests: -inf is never kept and weighs 0).  A segment of up to 32 kHeld
-    // positions is loaded once and kept in registers for every pass; a longer
-    // one is streamed in steps of 32 kStep positions through the two halves
-    // of the same registers, the loads of the next step in flight while the
-    // current one is processed.
+    // this warp's contiguous segment [lo, hi) of the row
     const int seg = (((vis + kWarps - 1) / kWarps) + 31) & ~31;
     const int lo = min(vis, warp * seg), hi = min(vis, lo + seg);
-    const bool resident = hi - lo <= 32 * kHeld;
-    const int nstep = (hi - lo + 32 * kStep - 1) / (32 * kStep);
-    float x[kHeld];
-    // positions lo + 32 (n0 + r) + lane into x[off + r], r < cnt
-    auto load_into = [&](auto off_c, auto cnt_c, int n0) {
-        constexpr int off = decltype(off_c)::value, cnt = decltype(cnt_c)::value;
-        const int p0 = lo + 32 * n0 + lane;
-        if (lo + 32 * (n0 + cnt) <= hi) {  // the whole part lies in the segment (every part but the last)
-#pragma unroll
-            for (int r = 0; r < cnt; r++) x[off + r] = __ldcg(s + p0 + 32 * r);
-        } else {
-#pragma unroll
-            for (int r = 0; r < cnt; r++) x[off + r] = p0 + 32 * r < hi ? __ldcg(s + p0 + 32 * r) : -INFINITY;
-        }
-    };
-    using C0 = std::integral_constant<int, 0>;
-    using CS = std::integral_constant<int, kStep>;
-    using CH = std::integral_constant<int, kHeld>;
-    // calls f(off_c, cnt_c, p0) on every part of the segment held in x
-    auto for_segment = [&](auto &&f) {
-        if (resident) {
-            f(C0{}, CH{}, lo + lane);
-            return;
-        }
-        load_into(C0{}, CS{}, 0);
-        for (int st = 0; st < nstep; st += 2) {
-            if (st + 1 < nstep) load_into(CS{}, CS{}, (st + 1) * kStep);
-            f(C0{}, CS{}, lo + 32 * st * kStep + lane);
-            if (st + 1 < nstep) {
-                if (st + 2 < nstep) load_into(C0{}, CS{}, (st + 2) * kStep);
-                f(CS{}, CS{}, lo + 32 * (st + 1) * kStep + lane);
-            }
-        }
-    };
-    if (resident) load_into(C0{}, CH{}, 0);
-
-    // pass 1: the histogram of the top 11 key bits of a sample: every eighth
-    // group of 32 consecutive positions (every position on short rows) -- the
-    // threshold is looked for there.  A streamed segment reads just its
-    // sample here.
-    for (int i = threadIdx.x; i < 2048; i += kThreads) sm.hist[i] = 0u;
-    __syncthreads();
-    const bool sampled = vis >= kSampleMinLen;  // always so for a streamed segment
-    uint32_t nsample = 0u;
-    if (resident) {
-        if (sampled) {
-#pragma unroll
-            for (int r = 0; r < kHeld; r += 8) {
-                if (lo + lane + 32 * r < hi) {
-                    atomicAdd(&sm.hist[canon_key(x[r]) >> 21], 1u);
-                    nsample++;
-                }
-            }
-        } else {
-#pragma unroll
-            for (int r = 0; r < kHeld; r++) {
-                if (lo + lane + 32 * r < hi) {
-                    atomicAdd(&sm.hist[canon_key(x[r]) >> 21], 1u);
-                    nsample++;
-                }
-            }
-        }
-    } else {
-        // groups 0, 8, 16, ... of the segment, four loads in flight
-        for (int g0 = 0; lo + 32 * g0 < hi; g0 += 32) {
-            float v[4];
-#pragma unroll
-            for (int u = 0; u < 4; u++) {
-                const int pos = lo + 32 * (g0 + 8 * u) + lane;
-                v[u] = pos < hi ? __ldcg(s + pos) : 0.f;
-            }
-#pragma unroll
-            for (int u = 0; u < 4; u++) {
-                if (lo + 32 * (g0 + 8 * u) + lane < hi) {
-                    atomicAdd(&sm.hist[canon_key(v[u]) >> 21], 1u);
-                    nsample++;
-                }
-            }
-        }
-    }
-    if (lane == 0) wstat[warp * 8 + 1] = 0u;  // this warp's candidate count, for pass 2
-    nsample = warp_sum(nsample);
-    if (lane == 0) wstat[warp * 8 + 6] = nsample;
-    __syncthreads();  // the histogram and the sample counts are complete
     // word f of the lane-th warp (0 past the last warp), for warp-wide reductions
     auto wword = [&](int f) { return lane < kWarps ? wstat[lane * 8 + f] : 0u; };
-    const uint32_t total_sample = warp_sum(wword(6));
-    // bins above b_hi are kept; bins [b_lo, b_hi] hold the candidates.  On the
-    // sample the k-th key has rank about k * nsample / vis; the range is
-    // widened by 4 binomial standard deviations each way and checked exactly
-    // below.  As floats: x >= hi_t is above, lo_t <= x < hi_t a candidate.
-    float hi_t, lo_t;
-    uint32_t b_hi, b_lo;
+
+    // ---- sample: up to kS groups of 32 positions per warp, evenly spaced over
+    // its segment (every group of a segment of at most kS groups), kept in
+    // registers; their minimum, maximum and a histogram in 2048 bins of equal
+    // width between the two give lo_t, a value at or below the sample's
+    // rank-(k * nsample / vis) score pushed down by 5 binomial standard
+    // deviations (on an unsampled row, at or below the k-th score itself)
+    const int gstep = max(1, ((seg >> 5) + kS - 1) / kS);
+    const bool sampled = gstep > 1;
+    float sv[kS];
+    float smin = INFINITY, smax = -INFINITY;
+    uint32_t nsample = 0u;
+#pragma unroll
+    for (int j = 0; j < kS; j++) {
+        const int pos = lo + 32 * j * gstep + lane;
+        sv[j] = pos < hi ? __ldcg(s + pos) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < kS; j++) {
+        if (lo + 32 * j * gstep + lane < hi) {
+            smin = fminf(smin, sv[j]);
+            smax = fmaxf(smax, sv[j]);
+            nsample++;
+        }
+    }
+    nsample = warp_sum(nsample);
+    smin = warp_min(smin);
+    smax = warp_max(smax);
+    if (lane == 0) {
+        wstat[warp * 8 + 0] = nsample;
+        wstat[warp * 8 + 1] = __float_as_uint(smin);
+        wstat[warp * 8 + 2] = __float_as_uint(smax);
+    }
+    for (int i = threadIdx.x; i < 2048; i += kThreads) sm.hist[i] = 0u;
+    __syncthreads();
+    const uint32_t total_sample = warp_sum(wword(0));
+    const float min_s = warp_min(lane < kWarps ? __uint_as_float(wstat[lane * 8 + 1]) : INFINITY);
+    const float m_s = warp_max(lane < kWarps ? __uint_as_float(wstat[lane * 8 + 2]) : -INFINITY);
+    const float scale_s = m_s > min_s ? 2048.f / (m_s - min_s) : 0.f;
+#pragma unroll
+    for (int j = 0; j < kS; j++)
+        if (lo + 32 * j * gstep + lane < hi)
+            atomicAdd(&sm.hist[min(2047, (int)((sv[j] - min_s) * scale_s))], 1u);
+    __syncthreads();
+    float lo_t;
     {
         const float ks = (float)k * (float)total_sample / (float)vis;
-        const float margin = sampled ? 4.f * sqrtf(ks) + 4.f : 0.f;
-        const uint32_t need_hi = (uint32_t)fmaxf(1.f, floorf(ks - margin));
-        const uint32_t need_lo = (uint32_t)fminf((float)total_sample, ceilf(ks + margin));
-        block_find_bins<2048>(sm.hist, need_hi, max(need_lo, need_hi), sm.tmp, sm.scal);
-        b_hi = sm.scal[0];
-        b_lo = sm.scal[2];
-        // a NaN threshold compares false: nothing above bin 2044 (+inf) or below bin 4 (-FLT_MAX)
-        hi_t = b_hi >= 2044u ? __uint_as_float(0x7fc00000u) : key_float((b_hi + 1u) << 21);
-        lo_t = key_float(b_lo << 21);
+        const float margin = sampled ? 5.f * sqrtf(ks) + 4.f : 0.f;
+        const uint32_t need = (uint32_t)fminf((float)total_sample, fmaxf(1.f, ceilf(ks + margin)));
+        block_find_bins<2048>(sm.hist, need, need, sm.tmp, sm.scal);
+        const uint32_t b_lo = sm.scal[0];
+        // one bin lower than the bin's bottom edge: below every sample score in it
+        lo_t = b_lo > 0u ? min_s + (float)(b_lo - 1u) / scale_s : -INFINITY;
     }
+    for (int i = threadIdx.x; i < 2048; i += kThreads) sm.hist[i] = 0u;  // for the list histogram
 
-    // pass 2: the row maximum; count the positions above the range; collect
-    // the keys inside it (in any order: only their values matter) into this
-    // warp's candidate list; append every score at or above the range, with
-    // its position, to this warp's ordered list (one ballot per round keeps
-    // position order); sum e^{s - m_lane} over this lane's positions against
-    // a running lane maximum m_lane (rescaled when it grows)
-    uint32_t nwin = 0u, nplus = 0u;
-    uint32_t *my_key = wc_key + warp * kWarpCand;
-    float *my_px = plus_x + warp * kPlusCap;
-    int32_t *my_pp = plus_pos + warp * kPlusCap;
+    // ---- the one pass over the row: its maximum, sum e^{s - m_s} against the
+    // sample maximum, and every score >= lo_t appended with its position to
+    // this warp's list in position order (one ballot per 32 positions; a full
+    // list keeps counting, its extra writes go to the spare slot)
+    uint2 *my_list = lists + warp * (cap + 1);
+    const float ms_l2e = m_s * kLog2e;
     float m_lane = -INFINITY, zall = 0.f;
-    for_segment([&](auto off_c, auto cnt_c, int p0) {
-        constexpr int off = decltype(off_c)::value, cnt = decltype(cnt_c)::value;
-        float bm = x[off];
-#pragma unroll
-        for (int r = 1; r < cnt; r++) bm = fmaxf(bm, x[off + r]);
-        if (bm > m_lane) {  // never true for a part with no position (all -inf)
-            zall *= exp2_approx((m_lane - bm) * kLog2e);
-            m_lane = bm;
-        }
-        const float ml = m_lane == -INFINITY ? 0.f : m_lane * kLog2e;
-#pragma unroll
-        for (int r = 0; r < cnt; r++) {
-            const float xv = x[off + r];
-            zall += exp2_approx(fmaf(xv, kLog2e, -ml));
-            const bool above = xv >= hi_t;
-            nwin += above;
-            const bool plus = xv >= lo_t;
-            const uint32_t pb = __ballot_sync(0xffffffffu, plus);
-            // the ordered list's slot for this lane; the two stores are
-            // predicated (no branch per round)
-            const uint32_t slot = nplus + __popc(pb & lt);
-            st_shared_if(plus && slot < (uint32_t)kPlusCap, my_px + slot, __float_as_uint(xv), my_pp + slot,
-                         (uint32_t)(p0 + 32 * r));
-            if (plus && !above) {
-                const uint32_t cs = atomicAdd(&wstat[warp * 8 + 1], 1u);
-                if (cs < (uint32_t)kWarpCand) my_key[cs] = __float_as_uint(xv);  // converted when ranked
-            }
-            nplus += __popc(pb);
-        }
+    uint32_t nl = 0u;
+    stream_range(s, lo, hi, lane, [&](float x, int pos, auto valid) {
+        m_lane = fmaxf(m_lane, x);
+        zall += exp2_approx(fmaf(x, kLog2e, -ms_l2e));
+        const bool sel = valid && x >= lo_t;
+        const uint32_t bal = __ballot_sync(0xffffffffu, sel);
+        const uint32_t slot = min(nl + __popc(bal & lt), (uint32_t)cap);
+        st_shared_v2_if(sel, my_list + slot, __float_as_uint(x), (uint32_t)pos);
+        nl += __popc(bal);
     });
-    float m = warp_max(m_lane);
-    if (lane == 0) wstat[warp * 8 + 5] = __float_as_uint(m);
-    nwin = warp_sum(nwin);
-    if (lane == 0) wstat[warp * 8 + 0] = nwin;
+    {
+        const float mw = warp_max(m_lane);
+        const float zw = warp_sum(zall);
+        if (lane == 0) {
+            wstat[warp * 8 + 3] = nl;
+            wstat[warp * 8 + 4] = __float_as_uint(mw);
+            wstat[warp * 8 + 5] = __float_as_uint(zw);
+        }
+    }
     __syncthreads();
-    m = warp_max(lane < kWarps ? __uint_as_float(wstat[lane * 8 + 5]) : -INFINITY);  // the row maximum
-    const float m_l2e = m * kLog2e;
-    // this lane's sum against the row maximum
-    zall = m_lane == -INFINITY ? 0.f : zall * exp2_approx((m_lane - m) * kLog2e);
-    // block totals, every warp reducing the per-warp words (lane w reads warp w's)
-    const uint32_t above = warp_sum(wword(0));
-    const uint32_t ncand = warp_sum(wword(1));
-    const bool overflow = __any_sync(0xffffffffu, wword(1) > (uint32_t)kWarpCand);
-    if (overflow || above >= (uint32_t)k || above + ncand < (uint32_t)k) {
-        // the sampled range missed the k-th key or a warp's list overflowed:
-        // take the exact multi-pass route
+    const float m = warp_max(lane < kWarps ? __uint_as_float(wstat[lane * 8 + 4]) : -INFINITY);  // row maximum
+    const uint32_t total = warp_sum(wword(3));
+    const bool overflow = __any_sync(0xffffffffu, wword(3) > (uint32_t)cap);
+    if (overflow || total < (uint32_t)k || (m - m_s) * kLog2e > 96.f) {
+        // a warp's list is full, the sample misled, or the sum against the
+        // sample maximum could overflow: take the exact multi-pass route
         __syncthreads();
         select_multipass(p, row, vis, sm);
         return;
     }
+    // sum_all e^{s - m}
+    const float z_all =
+        warp_sum(lane < kWarps ? __uint_as_float(wstat[lane * 8 + 5]) : 0.f) * exp2_approx((m_s - m) * kLog2e);
 
-    // exact radix selection over the candidates' keys.  They lie in the
-    // band's key range [base, base + 2^rem) (bins b_lo..b_hi of 2^21 keys;
-    // with no upper threshold, everything up to the top key), so every level
-    // splits the current range into at most 2048 bins and the candidates
-    // spread over the bins instead of piling into the few bins of the band
-    // (few conflicting atomics); two levels reach a single key unless the
-    // band spans more than two bins.
-    const uint32_t need = (uint32_t)k - above;
-    uint32_t gt = 0u, base = b_lo << 21;
-    int rem;
-    {
-        const uint32_t nb = (b_hi >= 2044u ? 2047u : b_hi) - b_lo + 1u;  // >= 1
-        rem = 21 + (nb > 1u ? 32 - __clz(nb - 1u) : 0);                // <= 32
-    }
-    // two histograms: level L counts into sm.hist (L even) or hist2 (L odd)
-    // while the other one is cleared for level L + 1; warp 0 searches between
-    // two barriers
-    for (int i = threadIdx.x; i < 2048; i += kThreads) {
-        sm.hist[i] = 0u;
-        hist2[i] = 0u;
-    }
-    __syncthreads();
-    const uint32_t my_cand = wstat[warp * 8 + 1];
-    for (int level = 0; rem > 0; level++) {
-        const int sh = rem > 11 ? rem - 11 : 0;
-        uint32_t *h = (level & 1) ? hist2 : sm.hist;
-        const unsigned long long span = 1ull << rem;
-        for (uint32_t i = lane; i < my_cand; i += 32) {  // this warp's own list
-            const uint32_t key = canon_key(__uint_as_float(my_key[i]));
-            if (key >= base && (unsigned long long)(key - base) < span) atomicAdd(&h[(key - base) >> sh], 1u);
+    // ---- which list entries are kept.  Either every entry whose bin (2048
+    // bins of equal width between lo_t and m) is at or above the bin b* that
+    // holds the k-th score, when b* is kept whole; or the rule s > T, or
+    // s == T among the first r_eq ties, with T the exact k-th score.
+    bool by_bin = false;
+    uint32_t bstar = 0u;
+    const float scale1 = m > lo_t && lo_t > -INFINITY ? 2048.f / (m - lo_t) : 0.f;
+    auto bin1 = [&](float x) { return min(2047u, (uint32_t)((x - lo_t) * scale1)); };
+    uint32_t T_key = 0u, r_eq = 0u;
+    bool resolved = false;
+    if (scale1 > 0.f) {
+        for (uint32_t i = lane; i < nl; i += 32) atomicAdd(&sm.hist[bin1(__uint_as_float(my_list[i].x))], 1u);
+        if (threadIdx.x == 0) sm.scal[4] = 0u;  // entries of b* collected below
+        __syncthreads();
+        block_find_bins<2048>(sm.hist, (uint32_t)k, (uint32_t)k, sm.tmp, sm.scal);
+        bstar = sm.scal[0];
+        const uint32_t c_star = sm.hist[bstar], r = (uint32_t)k - sm.scal[1];  // 1 <= r <= c_star
+        if (r == c_star) {
+            by_bin = true;
+            resolved = true;
+        } else if (c_star <= 32u) {
+            uint32_t *cand = sm.tmp;  // [32]: the tmp words are free until the next block search
+            for (uint32_t i = lane; i < nl; i += 32) {
+                const float xv = __uint_as_float(my_list[i].x);
+                if (bin1(xv) == bstar) cand[atomicAdd(&sm.scal[4], 1u)] = canon_key(xv);
+            }
+            __syncthreads();
+            if (warp == 0) {
+                const uint32_t mine = lane < (int)c_star ? cand[lane] : 0u;
+                uint32_t g = 0u, e = 0u;
+                for (uint32_t j = 0; j < c_star; j++) {
+                    const uint32_t o = cand[j];
+                    g += o > mine;
+                    e += o == mine;
+                }
+                const uint32_t hit = __ballot_sync(0xffffffffu, lane < (int)c_star && g < r && r <= g + e);
+                const int L = hit ? __ffs(hit) - 1 : 0;
+                const uint32_t tk = __shfl_sync(0xffffffffu, mine, L), tg = __shfl_sync(0xffffffffu, g, L);
+                if (lane == 0) {
+                    sm.scal[5] = tk;
+                    sm.scal[6] = r - tg;
+                    if (!hit) raise_status(p.status, TKA_DEV_INTERNAL);
+                }
+            }
+            __syncthreads();
+            T_key = sm.scal[5];
+            r_eq = sm.scal[6];
+            resolved = true;
         }
-        if (level >= 1) {  // the previous level's histogram, for the next level
-            uint32_t *hn = (level & 1) ? sm.hist : hist2;
-            for (int i = threadIdx.x; i < 2048; i += kThreads) hn[i] = 0u;
-        }
-        __syncthreads();  // the histogram is complete
-        block_find_bins<2048>(h, need - gt, need - gt, sm.tmp, sm.scal);
-        gt += sm.scal[1];
-        base += sm.scal[0] << sh;
-        rem = sh;
     }
-    const uint32_t T = base;
-    // keys equal to T: the first r_eq of them (by position) are kept
-    const uint32_t r_eq = need - gt;
+    if (!resolved) {
+        // many scores share b*, or no bins could be formed: radix levels of
+        // up to 11 bits over the keys of the list entries, from the smallest
+        // possible to that of m
+        __syncthreads();  // every thread has read the words of the pass above
+        uint32_t base = lo_t > -INFINITY ? canon_key(lo_t) : 0u, gt = 0u;
+        const uint32_t span_m1 = canon_key(m) - base;
+        int rem = span_m1 ? 32 - __clz(span_m1) : 0;
+        while (rem > 0) {
+            const int sh = rem > 11 ? rem - 11 : 0;
+            __syncthreads();
+            for (int i = threadIdx.x; i < 2048; i += kThreads) sm.hist[i] = 0u;
+            __syncthreads();
+            for (uint32_t i = lane; i < nl; i += 32) {
+                const uint32_t d = canon_key(__uint_as_float(my_list[i].x)) - base;
+                if ((rem >= 32 || d < (1u << rem)) && (d >> sh) < 2048u) atomicAdd(&sm.hist[d >> sh], 1u);
+            }
+            __syncthreads();
+            block_find_bins<2048>(sm.hist, (uint32_t)k - gt, (uint32_t)k - gt, sm.tmp, sm.scal);
+            gt += sm.scal[1];
+            base += sm.scal[0] << sh;
+            rem = sh;
+        }
+        T_key = base;
+        r_eq = (uint32_t)k - gt;
+    }
+    const float T_f = key_float(T_key);
+    const float m_l2e = m * kLog2e;
+    auto above = [&](float x) { return by_bin ? bin1(x) >= bstar : x > T_f; };
+    auto tie = [&](float x) { return !by_bin && x == T_f; };
 
-    // per warp: candidates above T and ties at T, then output offsets
+    // ---- per warp: kept entries above T and ties at T, then output offsets
     {
         uint32_t g = 0u, t = 0u;
-        for (uint32_t i = lane; i < wstat[warp * 8 + 1]; i += 32) {
-            const uint32_t key = canon_key(__uint_as_float(my_key[i]));
-            g += key > T;
-            t += key == T;
+        for (uint32_t i = lane; i < nl; i += 32) {
+            const float xv = __uint_as_float(my_list[i].x);
+            g += above(xv);
+            t += tie(xv);
         }
         g = warp_sum(g);
         t = warp_sum(t);
         if (lane == 0) {
-            wstat[warp * 8 + 2] = g;
-            wstat[warp * 8 + 3] = t;
+            wstat[warp * 8 + 5] = g;
+            wstat[warp * 8 + 6] = t;
         }
     }
     __syncthreads();
-    // output offsets: warp w keeps its scores above the range, its candidates
-    // above T and the ties at T that fall among the first r_eq of the row
     uint32_t out_run, tie_run, n_eq;
     {
-        const uint32_t tie_l = wword(3);
+        const uint32_t tie_l = wword(6);
         const uint32_t tie_incl = warp_incl_scan(tie_l), tie_excl = tie_incl - tie_l;
-        const uint32_t kept_l = wword(0) + wword(2) +
-                                (r_eq > tie_excl ? min(tie_l, r_eq - tie_excl) : 0u);
+        const uint32_t kept_l = wword(5) + (r_eq > tie_excl ? min(tie_l, r_eq - tie_excl) : 0u);
         const uint32_t out_incl = warp_incl_scan(kept_l);
         out_run = __shfl_sync(0xffffffffu, out_incl - kept_l, warp);
         tie_run = __shfl_sync(0xffffffffu, tie_excl, warp);
         n_eq = __shfl_sync(0xffffffffu, tie_incl, 31);
     }
-    const bool rank_ties = n_eq != r_eq;
+    const bool rank_ties = r_eq < n_eq;
     const uint32_t out_begin = out_run;
 
-    // pass 3: the exact rule -- s > T, or s == T among the first r_eq ties
-    // (s >= T when every tie is kept) -- written straight to the final
-    // ascending positions, with the softmax sums of kept and dropped scores.
-    // As float comparisons: canon_key order is float order.  A warp whose
-    // ordered list is complete takes its kept positions from the list (every
-    // kept score is at or above the range) and its dropped mass as the total
-    // less the kept; a warp whose list overflowed streams its segment again.
-    const float T_f = key_float(T);
+    // ---- emit every kept entry straight to its final ascending slot
     int32_t *idx = p.idx + (size_t)row * k;
     float *wv = p.w + (size_t)row * k;
-    float zk = 0.f, zt = 0.f;
-    auto emit = [&](bool sel, float e, int pos) {
+    float zk = 0.f;
+    for (uint32_t i0 = 0; i0 < nl; i0 += 32) {
+        const uint32_t i = i0 + lane;
+        const uint2 e = i < nl ? my_list[i] : make_uint2(__float_as_uint(-INFINITY), 0u);
+        const float xv = __uint_as_float(e.x);
+        const bool in = i < nl;
+        bool sel = in && above(xv);
+        if (rank_ties) {
+            const bool t = in && tie(xv);
+            const uint32_t tb = __ballot_sync(0xffffffffu, t);
+            sel = sel || (t && tie_run + __popc(tb & lt) < r_eq);
+            tie_run += __popc(tb);
+        } else {
+            sel = sel || (in && tie(xv));
+        }
         const uint32_t sb = __ballot_sync(0xffffffffu, sel);
         if (sel) {
+            const float ew = exp2_approx(fmaf(xv, kLog2e, -m_l2e));
             const uint32_t o = out_run + __popc(sb & lt);
             if (o < (uint32_t)k) {  // always true unless the counts above are wrong
-                idx[o] = pos;
-                wv[o] = e;
+                idx[o] = (int32_t)e.y;
+                wv[o] = ew;
             }
-            zk += e;
-        } else {
-            zt += e;
+            zk += ew;
         }
         out_run += __popc(sb);
-    };
-    if (nplus <= (uint32_t)kPlusCap) {
-        for (uint32_t i0 = 0; i0 < nplus; i0 += 32) {
-            const uint32_t i = i0 + lane;
-            const float xv = i < nplus ? my_px[i] : -INFINITY;
-            bool sel;
-            if (rank_ties) {
-                const bool tie = xv == T_f;
-                const uint32_t tb = __ballot_sync(0xffffffffu, tie);
-                sel = xv > T_f || (tie && tie_run + __popc(tb & lt) < r_eq);
-                tie_run += __popc(tb);
-            } else {
-                sel = xv >= T_f;
-            }
-            const uint32_t sb = __ballot_sync(0xffffffffu, sel);
-            if (sel) {
-                const float e = exp2_approx(fmaf(xv, kLog2e, -m_l2e));
-                const uint32_t o = out_run + __popc(sb & lt);
-                if (o < (uint32_t)k) {  // always true unless the counts above are wrong
-                    idx[o] = my_pp[i];
-                    wv[o] = e;
-                }
-                zk += e;
-            }
-            out_run += __popc(sb);
-        }
-        // dropped = all - kept, per warp (the warp's lanes sum to its totals)
-        zt = zall - zk;
-    } else {
-        for_segment([&](auto off_c, auto cnt_c, int p0) {
-            constexpr int off = decltype(off_c)::value, cnt = decltype(cnt_c)::value;
-#pragma unroll
-            for (int r = 0; r < cnt; r++) {
-                const float xv = x[off + r];
-                bool sel = xv >= T_f;
-                if (rank_ties) {
-                    const bool tie = xv == T_f;
-                    const uint32_t tb = __ballot_sync(0xffffffffu, tie);
-                    sel = xv > T_f || (tie && tie_run + __popc(tb & lt) < r_eq);
-                    tie_run += __popc(tb);
-                }
-                emit(sel, exp2_approx(fmaf(xv, kLog2e, -m_l2e)), p0 + 32 * r);
-            }
-        });
     }
-    if (lane == 0) wstat[warp * 8 + 4] = out_run - out_begin;
+    zk = warp_sum(zk);
+    if (lane == 0) {
+        wstat[warp * 8 + 6] = __float_as_uint(zk);
+        wstat[warp * 8 + 7] = out_run - out_begin;
+    }
     __syncthreads();
-    const uint32_t written = warp_sum(wword(4));
-    finish_row(p, row, m, zk, zt, written, (uint32_t)k, sm);
+    if (warp == 0) {
+        const float zk_row = warp_sum(lane < kWarps ? __uint_as_float(wstat[lane * 8 + 6]) : 0.f);
+        const uint32_t written = warp_sum(wword(7));
+        if (lane == 0) {
+            const float zt = fmaxf(z_all - zk_row, 0.f);  // formed as total - kept: >= 0
+            if (written != (uint32_t)k) raise_status(p.status, TKA_DEV_INTERNAL);
+            p.stats[row] = make_float4(m, zk_row, zt, 0.f);
+            if (p.tail) p.tail[row] = zt / (zk_row + zt);
+            p.counters[row] = 0u;
+        }
+    }
 }
 
 }  // namespace
 
-size_t select_smem_bytes(int threads) { return smem_words(threads / 32) * 4; }
+size_t select_smem_bytes(int threads, int k) { return smem_words_for(k, threads / 32) * 4; }
 
 namespace {
 
 template <int kThreads>
 cudaError_t launch_n(const SelectParams &p, cudaStream_t stream, bool pdl) {
     const int rows = p.B * p.Q * p.Hq;
-    const size_t smem = select_smem_bytes(kThreads);
+    const size_t smem = select_smem_bytes(kThreads, p.k);
     static bool attr_set[64] = {};  // per device: the shared-memory opt-in is a function attribute
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (smem > 48 * 1024 && (dev < 0 || dev >= 64 || !attr_set[dev])) {
-        e = cudaFuncSetAttribute(select_topk<kThreads>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+        // the largest size any k takes, so that one setting serves every call
+        e = cudaFuncSetAttribute(select_topk<kThreads>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)select_smem_bytes(kThreads, kMaxK));
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
