@@ -212,25 +212,52 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- CPU oracle
 
-def time_oracle(w, k, budget_s=10.0, max_reps=50, eps=None):
-    """The oracle as it stands on this host's cores, whole workload repeated
-    until `budget_s` has elapsed.  Returns (queries/s, cores, sample text)."""
+def time_oracle(w, k, budget_s=10.0, max_reps=50, eps=None, nthreads=0):
+    """The oracle as it stands on this host's cores (nthreads = 0: all of
+    them), whole workload repeated until `budget_s` has elapsed (at least
+    once).  Returns (queries/s, threads used, sample text)."""
     import oracle
     rows = w.B * w.Q * w.Hq
     reps, t0 = 0, time.perf_counter()
     while True:
         if w.variant == "block":
-            oracle.block_attn(w, w.block_size, w.top_blocks)
+            oracle.block_attn(w, w.block_size, w.top_blocks, nthreads=nthreads)
         elif eps is not None:
-            oracle.certified_attn(w, eps, k)
+            oracle.certified_attn(w, eps, k, nthreads=nthreads)
         else:
-            oracle.topk_attn(w, k)
+            oracle.topk_attn(w, k, nthreads=nthreads)
         reps += 1
         dt = time.perf_counter() - t0
         if dt >= budget_s or reps >= max_reps:
             break
     sample = f"whole workload ({rows} query rows) x {reps} repetitions, {dt:.1f} s"
-    return rows * reps / dt, oracle.max_threads(), sample
+    return rows * reps / dt, (nthreads or oracle.max_threads()), sample
+
+
+def workload_config(w, k, world, args):
+    """The `config` object of the JSON line: the same for both arms."""
+    certified = args.certified_eps is not None and w.variant != "block"
+    paged = args.paged is not None and w.variant != "block" and not certified
+    hisa = args.hisa is not None and w.variant != "block" and not certified and not paged
+    indexer = args.indexer is not None and w.variant != "block" and not certified and not paged and not hisa
+    cfg = {
+        "workload": w.name, "B": w.B, "Q": w.Q, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "L_max": w.L_max,
+        "k": k, "block_size": w.block_size, "top_blocks": w.top_blocks,
+        "seq_lens": "full" if int(w.seq_lens.min()) == w.L_max else [int(x) for x in w.seq_lens],
+        "accumulate": "fp32", "parallelism": f"replica x{world} (independent sequences per GPU)",
+        "l2": "flushed between timed steps (256 MiB write + 256 MiB read, outside the timed events)",
+    }
+    if certified:
+        cfg.update({"certified_eps": args.certified_eps, "k_max": k})
+    if paged:
+        cfg.update({"page_size": args.paged, "pages": "shuffled pool, block tables"})
+    if hisa:
+        h_bs, h_top = (int(x) for x in args.hisa.split(","))
+        cfg.update({"hisa_block_size": h_bs, "hisa_top_blocks": h_top})
+    if indexer:
+        i_h, i_d = (int(x) for x in args.indexer.split(","))
+        cfg.update({"indexer_heads": i_h, "indexer_dims": i_d, "indexer_inputs": "synthetic"})
+    return cfg
 
 
 # ----------------------------------------------------------------------------- runs
@@ -521,17 +548,7 @@ def run_ours(args, world, rank, local):
         "vs_baseline": None,
         "dtype": w.dtype,
         "data": "synthetic (seeded numpy PCG64, rounded once to the cache dtype)",
-        "config": {
-            "workload": w.name, "B": w.B, "Q": w.Q, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "L_max": w.L_max,
-            "k": k, "block_size": w.block_size, "top_blocks": w.top_blocks,
-            "seq_lens": "full" if int(w.seq_lens.min()) == w.L_max else [int(x) for x in w.seq_lens],
-            "accumulate": "fp32", "parallelism": f"replica x{world} (independent sequences per GPU)",
-            "l2": "flushed between timed steps (256 MiB write + 256 MiB read, outside the timed events)",
-            **({"certified_eps": args.certified_eps, "k_max": k} if certified else {}),
-            **({"page_size": args.paged, "pages": "shuffled pool, block tables"} if paged else {}),
-            **({"hisa_block_size": h_bs, "hisa_top_blocks": h_top} if hisa else {}),
-            **({"indexer_heads": i_h, "indexer_dims": i_d, "indexer_inputs": "synthetic"} if indexer else {}),
-        },
+        "config": workload_config(w, k, world, args),
         "us_per_step": ms * 1e3,
         "tokens_per_s": world * w.B * w.Q / (ms / 1e3),
         "alg_bytes_per_step": alg,
@@ -615,8 +632,11 @@ def run_ours(args, world, rank, local):
             res["e2e"]["overlap"] = ("idx is read back on a side stream from the event the library records "
                                      "after the select, while the gather runs")
     if world == 1 and not args.no_cpu_baseline:
-        v, cores, sample = time_oracle(w, k, eps=args.certified_eps if certified else None)
-        res["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+        eps = args.certified_eps if certified else None
+        v, cores, sample = time_oracle(w, k, eps=eps)
+        v1, _, sample1 = time_oracle(w, k, budget_s=5.0, eps=eps, nthreads=1)
+        res["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+                               "value_1thread": v1, "sample_1thread": sample1}
     return res
 
 
@@ -650,8 +670,7 @@ def run_reference(args, rank):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded numpy PCG64)",
-        "config": {"workload": w.name, "B": w.B, "Q": w.Q, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "L_max": w.L_max,
-                   "k": k, "block_size": w.block_size, "top_blocks": w.top_blocks},
+        "config": workload_config(w, k, args.gpus, args),
         "impl": "reference",
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

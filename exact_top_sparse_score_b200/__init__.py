@@ -23,7 +23,9 @@ from ._binding import (  # noqa: F401
     topk_attn_decode_paged,
     topk_attn_decode_static,
     topk_attn_static_workspace_capacity,
+    topk_attn_debug_set_wait_limit,
     topk_attn_device_status,
+    topk_attn_last_device_status,
     topk_attn_workspace_size,
     topk_block_attn_decode,
     topk_block_pool_keys,

@@ -13,7 +13,7 @@ _LIB_NAME = "libtopk_attn.so"
 TKA_F32, TKA_BF16 = 0, 1
 DEV_BAD_SEQ_LEN, DEV_INTERNAL, DEV_TIMEOUT, DEV_BAD_PAGE = 0x1, 0x2, 0x4, 0x8
 _STATUS = {0: "TKA_OK", 1: "TKA_ERR_INVALID_ARG", 2: "TKA_ERR_UNSUPPORTED", 3: "TKA_ERR_WORKSPACE",
-           4: "TKA_ERR_CUDA"}
+           4: "TKA_ERR_CUDA", 5: "TKA_ERR_TIMEOUT"}
 
 
 class TopkAttnError(RuntimeError):
@@ -82,6 +82,10 @@ def load_library() -> ctypes.CDLL:
         lib.topk_block_attn_decode.restype = ctypes.c_int
         lib.topk_attn_device_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_uint32)]
         lib.topk_attn_device_status.restype = ctypes.c_int
+        lib.topk_attn_last_device_status.argtypes = [_vp]
+        lib.topk_attn_last_device_status.restype = ctypes.c_int
+        lib.topk_attn_debug_set_wait_limit.argtypes = [ctypes.c_uint32]
+        lib.topk_attn_debug_set_wait_limit.restype = None
         lib.topk_attn_status_string.argtypes = [ctypes.c_int]
         lib.topk_attn_status_string.restype = ctypes.c_char_p
         _lib = lib
@@ -101,6 +105,9 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
 
 
 def _check_cuda(**tensors):
+    """Every tensor must be a contiguous CUDA tensor, all on one device (the
+    library launches on the current device, which the wrappers set to it)."""
+    dev = None
     for name, t in tensors.items():
         if t is None:
             continue
@@ -108,6 +115,26 @@ def _check_cuda(**tensors):
             raise ValueError(f"{name} must be a CUDA tensor")
         if not t.is_contiguous():
             raise ValueError(f"{name} must be contiguous")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, the other tensors on {dev}")
+
+
+def _on_device(fn):
+    """Runs a wrapper with the device of its first tensor argument current, so
+    that the library's kernels, its per-device state and the default stream
+    all belong to the device the tensors live on."""
+    import functools
+
+    @functools.wraps(fn)
+    def run(*args, **kwargs):
+        first = args[0] if args else None
+        if isinstance(first, torch.Tensor) and first.is_cuda:
+            with torch.cuda.device(first.device):
+                return fn(*args, **kwargs)
+        return fn(*args, **kwargs)
+    return run
 
 
 def _check_out(name: str, t: Optional[torch.Tensor], dtype: torch.dtype, shape: tuple):
@@ -170,6 +197,7 @@ def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor], stream_ha
     return ws
 
 
+@_on_device
 def topk_attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, seq_lens: torch.Tensor,
                      k: int, *, scale: float = 0.0, out: Optional[torch.Tensor] = None,
                      idx: Optional[torch.Tensor] = None, tail_mass: Optional[torch.Tensor] = None,
@@ -218,6 +246,7 @@ def topk_attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tens
     return out, idx, tail_mass
 
 
+@_on_device
 def topk_attn_decode_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,
                            block_table: torch.Tensor, seq_lens: torch.Tensor, k: int, *, scale: float = 0.0,
                            out: Optional[torch.Tensor] = None, idx: Optional[torch.Tensor] = None,
@@ -267,6 +296,7 @@ def topk_attn_decode_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torc
     return out, idx, tail_mass
 
 
+@_on_device
 def topk_attn_decode_certified(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                                seq_lens: torch.Tensor, eps: float, k_max: int, *, scale: float = 0.0,
                                out: Optional[torch.Tensor] = None, idx: Optional[torch.Tensor] = None,
@@ -313,6 +343,7 @@ def topk_attn_decode_certified(q: torch.Tensor, k_cache: torch.Tensor, v_cache: 
     return out, idx, tail_mass, k_used
 
 
+@_on_device
 def topk_attn_decode_static(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, seq_lens: torch.Tensor,
                             k: int, *, out: torch.Tensor, idx: torch.Tensor, tail_mass: Optional[torch.Tensor] = None,
                             scale: float = 0.0, stream=None) -> None:
@@ -325,6 +356,8 @@ def topk_attn_decode_static(q: torch.Tensor, k_cache: torch.Tensor, v_cache: tor
     B, Q, Hq, d = q.shape
     if seq_lens.dtype != torch.int32 or tuple(seq_lens.shape) != (B,):
         raise TypeError("seq_lens must be int32 [B]")
+    if v_cache.dtype != k_cache.dtype or v_cache.shape != k_cache.shape:
+        raise TypeError("v_cache must match k_cache in dtype and shape")
     _check_out("out", out, torch.float32, (B, Q, Hq, d))
     _check_out("idx", idx, torch.int32, (B, Q, Hq, k))
     _check_out("tail_mass", tail_mass, torch.float32, (B, Q, Hq))
@@ -340,6 +373,7 @@ def topk_attn_static_workspace_capacity() -> int:
     return int(load_library().topk_attn_static_workspace_capacity())
 
 
+@_on_device
 def topk_block_pool_keys(k_cache: torch.Tensor, seq_lens: torch.Tensor, block_size: int, *,
                          block_keys: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """Mean-pooled block keys fp32 [B, Hkv, ceil(L_max/block_size), d]."""
@@ -360,6 +394,7 @@ def topk_block_pool_keys(k_cache: torch.Tensor, seq_lens: torch.Tensor, block_si
     return block_keys
 
 
+@_on_device
 def topk_block_attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                            block_keys: torch.Tensor, seq_lens: torch.Tensor, block_size: int, top_blocks: int, *,
                            scale: float = 0.0, out: Optional[torch.Tensor] = None,
@@ -397,6 +432,18 @@ def topk_block_attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torc
     return out, block_idx
 
 
+def topk_attn_last_device_status(stream=None) -> int:
+    """Synchronises the stream and returns the device status word read as a
+    status code (5 = TKA_ERR_TIMEOUT when a bounded wait gave up), clearing it."""
+    return int(load_library().topk_attn_last_device_status(_stream(stream)))
+
+
+def topk_attn_debug_set_wait_limit(polls: int) -> None:
+    """Diagnostics: polls before a pipeline wait inside the tensor-core score
+    and block-attention kernels gives up (0 restores the default bound)."""
+    load_library().topk_attn_debug_set_wait_limit(int(polls))
+
+
 def topk_attn_device_status(stream=None) -> int:
     """Synchronises the stream and returns (and clears) the device status bits."""
     bits = ctypes.c_uint32(0)
@@ -406,6 +453,7 @@ def topk_attn_device_status(stream=None) -> int:
     return int(bits.value)
 
 
+@_on_device
 def topk_hisa_attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_keys: torch.Tensor,
                           seq_lens: torch.Tensor, block_size: int, top_blocks: int, k: int, *, scale: float = 0.0,
                           out: Optional[torch.Tensor] = None, idx: Optional[torch.Tensor] = None,
@@ -454,6 +502,7 @@ def topk_hisa_attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch
     return out, idx, tail_mass, block_idx
 
 
+@_on_device
 def topk_indexer_attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, q_idx: torch.Tensor,
                              w_idx: torch.Tensor, k_idx: torch.Tensor, seq_lens: torch.Tensor, k: int, *,
                              scale: float = 0.0, out: Optional[torch.Tensor] = None,

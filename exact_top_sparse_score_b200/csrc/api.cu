@@ -4,6 +4,9 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -12,6 +15,10 @@ namespace {
 
 __device__ unsigned int g_status = 0u;
 
+// Polls before a pipeline wait inside a kernel gives up (0: the kernels'
+// default bound); set only through topk_attn_debug_set_wait_limit.
+std::atomic<uint32_t> g_wait_polls{0u};
+
 constexpr int kMaxDevices = 64;
 constexpr int kMaxQ = 64;
 constexpr int kMaxRowsPerKvHead = 256;  // Q * G
@@ -19,25 +26,30 @@ constexpr int kMaxLen = 1 << 24;
 constexpr int kMinKeysPerSplit = 64;
 
 struct DeviceInfo {
-    bool ready = false;
+    std::atomic<bool> ready{false};  // published (release) once the fields below are set
     int num_sms = 0;
     unsigned *status = nullptr;  // device address of g_status
 };
 DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;  // serialises the first lookup on a device
 
-// SM count and status-word address of the current device (looked up once).
+// SM count and status-word address of the current device (looked up once;
+// concurrent first calls from several host threads wait for one lookup).
 cudaError_t device_info(DeviceInfo **out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     DeviceInfo &d = g_dev[dev];
-    if (!d.ready) {
-        e = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
-        if (e != cudaSuccess) return e;
-        e = cudaGetSymbolAddress(reinterpret_cast<void **>(&d.status), g_status);
-        if (e != cudaSuccess) return e;
-        d.ready = true;
+    if (!d.ready.load(std::memory_order_acquire)) {
+        std::lock_guard<std::mutex> lock(g_dev_mu);
+        if (!d.ready.load(std::memory_order_relaxed)) {
+            e = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
+            if (e != cudaSuccess) return e;
+            e = cudaGetSymbolAddress(reinterpret_cast<void **>(&d.status), g_status);
+            if (e != cudaSuccess) return e;
+            d.ready.store(true, std::memory_order_release);
+        }
     }
     *out = &d;
     return cudaSuccess;
@@ -301,6 +313,7 @@ tka_status launch_score(const DecodeArgs &a, cudaStream_t s, const tka_event_t *
         tp.L_max = sh->L_max; tp.ld = a.L.ld; tp.NQ = sh->Q * a.G;
         tp.scale = resolve_scale(sh);
         if (a.pages) tp.pages = *a.pages;
+        tp.max_polls = g_wait_polls.load(std::memory_order_relaxed);
         RecordCtx rc{events, 0, s};
         ScoreTcHook hook;
         hook.fn = record_hook;
@@ -421,7 +434,8 @@ tka_status decode_impl(const tka_shape *shape, const void *q, const void *k_cach
     a.ws = static_cast<char *>(workspace);
     if (device_info(&a.dev) != cudaSuccess) return TKA_ERR_CUDA;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // the tensor map addresses cache rows with int32 coordinates
+    // the tensor map addresses cache rows with int32 coordinates (a K cache of
+    // 2^31 rows, 512 GB, does not fit one GPU; the CUDA-core scorer takes it)
     a.tc = score_tc_supported(shape->dtype, shape->Q * a.G) &&
            (pages || (long long)shape->B * shape->Hkv * shape->L_max < (1LL << 31));
 
@@ -562,6 +576,7 @@ tka_status topk_block_attn_decode(const tka_shape *shape, const void *q, const v
     ap.part_acc = reinterpret_cast<float *>(ws + L.part_acc);
     ap.counters = counters;
     ap.out = out;
+    ap.max_polls = g_wait_polls.load(std::memory_order_relaxed);
     if (launch_block_attn(ap, k_cache, dev->num_sms, s) != cudaSuccess) return TKA_ERR_CUDA;
     return TKA_OK;
 }
@@ -708,6 +723,7 @@ tka_status topk_indexer_attn_decode(const tka_shape *shape, const void *q, const
         tp.B = shape->B; tp.Q = shape->Q; tp.Hq = H_I; tp.Hkv = 1; tp.G = H_I;
         tp.L_max = shape->L_max; tp.ld = L.ld; tp.NQ = shape->Q * H_I;
         tp.scale = 1.f;
+        tp.max_polls = g_wait_polls.load(std::memory_order_relaxed);
         if (launch_score_tc(tp, q_idx, k_idx, dev->num_sms, s, ScoreTcHook{}) != cudaSuccess) return TKA_ERR_CUDA;
         if (launch_indexer_combine(ip, tp.scores, s) != cudaSuccess) return TKA_ERR_CUDA;
     } else if (launch_indexer_scores(ip, dev->num_sms, s) != cudaSuccess) {
@@ -762,6 +778,18 @@ tka_status topk_attn_device_status(tka_stream_t stream, uint32_t *bits) {
     return TKA_OK;
 }
 
+tka_status topk_attn_last_device_status(tka_stream_t stream) {
+    uint32_t bits = 0u;
+    const tka_status st = topk_attn_device_status(stream, &bits);
+    if (st != TKA_OK) return st;
+    if (bits & TKA_DEV_TIMEOUT) return TKA_ERR_TIMEOUT;
+    if (bits & (TKA_DEV_BAD_SEQ_LEN | TKA_DEV_BAD_PAGE)) return TKA_ERR_INVALID_ARG;
+    if (bits & TKA_DEV_INTERNAL) return TKA_ERR_CUDA;
+    return TKA_OK;
+}
+
+void topk_attn_debug_set_wait_limit(uint32_t polls) { g_wait_polls.store(polls, std::memory_order_relaxed); }
+
 const char *topk_attn_status_string(tka_status status) {
     switch (status) {
         case TKA_OK: return "TKA_OK";
@@ -769,6 +797,7 @@ const char *topk_attn_status_string(tka_status status) {
         case TKA_ERR_UNSUPPORTED: return "TKA_ERR_UNSUPPORTED";
         case TKA_ERR_WORKSPACE: return "TKA_ERR_WORKSPACE";
         case TKA_ERR_CUDA: return "TKA_ERR_CUDA";
+        case TKA_ERR_TIMEOUT: return "TKA_ERR_TIMEOUT";
     }
     return "unknown tka_status";
 }

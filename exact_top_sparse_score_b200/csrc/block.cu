@@ -336,7 +336,9 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-template <typename T>
+// kProbe: the pipeline waits are diagnostic probes bounded by p.max_polls
+// (the instantiation launched only when a test has lowered the limit)
+template <typename T, bool kProbe>
 __global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
     block_attn(const __grid_constant__ CUtensorMap kmap, BlockAttnParams p) {
     pdl_wait();  // inputs may come from the kernel before
@@ -372,6 +374,7 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
     }
     __syncthreads();
     volatile int *abort = &sh.abort;
+    const uint32_t polls = p.max_polls;  // diagnostic probes (kProbe only)
 
     if (warp == kProducerWarp) {
         // ------------------------------------------------ producer warp
@@ -399,7 +402,8 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
                 if (lane == 0) {
                     const long long k = i0 + u - beg;
                     const int s = (int)(k % S);
-                    const bool ok = k < S || sm100::mbar_wait(&sh.empty[s], (uint32_t)((k / S - 1) & 1), abort);
+                    const bool ok =
+                        k < S || sm100::pipe_wait<kProbe>(&sh.empty[s], (uint32_t)((k / S - 1) & 1), abort, polls);
                     if (ok) {
                         const int rows = v & 255;
                         sh.n[s] = rows;
@@ -451,7 +455,7 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
         if (first_shared) erow[ne++] = r_first;
         if (beg < end && r_last != r_first && row_shared(r_last)) erow[ne++] = r_last;
         for (int e = 0; e < ne; e++) {
-            if (!sm100::mbar_wait(&sh.piece_ready[e], 0, abort)) break;
+            if (!sm100::pipe_wait<kProbe>(&sh.piece_ready[e], 0, abort, polls)) break;
             const int row = erow[e];
             const int seq_len = p.seq_lens[row / p.Hq];
             if (seq_len < 1 || seq_len > p.L_max) continue;  // block_topk raised the status
@@ -548,7 +552,7 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
             const int sl = p.seq_lens[row / p.Hq];
             cur_valid = sl >= 1 && sl <= p.L_max;
         }
-        const bool landed = sm100::mbar_wait(&sh.full[s], (uint32_t)((k / S) & 1), abort);
+        const bool landed = sm100::pipe_wait<kProbe>(&sh.full[s], (uint32_t)((k / S) & 1), abort, polls);
         if (!consumers_all(landed)) {
             if (threadIdx.x == 0) {
                 if (!*abort) raise_status(p.status, TKA_DEV_TIMEOUT);
@@ -722,11 +726,17 @@ cudaError_t launch_block_attn(const BlockAttnParams &p0, const void *k_cache, in
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
-        if ((e = allow_smem(block_attn<__nv_bfloat16>, smem)) != cudaSuccess) return e;
-        return launch_k(true, block_attn<__nv_bfloat16>, dim3(grid), dim3(kAttnThreads), smem, stream, kmap, p);
+        if ((e = allow_smem(block_attn<__nv_bfloat16, false>, smem)) != cudaSuccess) return e;
+        if ((e = allow_smem(block_attn<__nv_bfloat16, true>, smem)) != cudaSuccess) return e;
+        if (p.max_polls)
+            return launch_k(true, block_attn<__nv_bfloat16, true>, dim3(grid), dim3(kAttnThreads), smem, stream, kmap, p);
+        return launch_k(true, block_attn<__nv_bfloat16, false>, dim3(grid), dim3(kAttnThreads), smem, stream, kmap, p);
     }
-    if ((e = allow_smem(block_attn<float>, smem)) != cudaSuccess) return e;
-    return launch_k(true, block_attn<float>, dim3(grid), dim3(kAttnThreads), smem, stream, kmap, p);
+    if ((e = allow_smem(block_attn<float, false>, smem)) != cudaSuccess) return e;
+    if ((e = allow_smem(block_attn<float, true>, smem)) != cudaSuccess) return e;
+    if (p.max_polls)
+        return launch_k(true, block_attn<float, true>, dim3(grid), dim3(kAttnThreads), smem, stream, kmap, p);
+    return launch_k(true, block_attn<float, false>, dim3(grid), dim3(kAttnThreads), smem, stream, kmap, p);
 }
 
 }  // namespace tka

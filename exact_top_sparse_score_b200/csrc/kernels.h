@@ -29,6 +29,7 @@ struct ScoreTcParams {
     int B, Q, Hq, Hkv, G, L_max, ld, NQ;
     float scale;
     PageTable pages;          // paged cache: the K tensor map covers [num_pages*Hkv*page, 128]
+    uint32_t max_polls = 0;   // polls before a pipeline wait gives up (0: the default bound)
 };
 
 struct SelectParams {
@@ -152,6 +153,7 @@ struct BlockAttnParams {
     float *out;               // [rows, 128]
     int stages;               // set by the launcher
     uint32_t stage_bytes;
+    uint32_t max_polls = 0;   // polls before a pipeline wait gives up (0: the default bound)
 };
 
 // Launches kernel<<<grid, block, smem, stream>>>(args...), allowed to start

@@ -29,6 +29,8 @@
 #include <cuda.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -96,7 +98,9 @@ struct TileWalk {
 // scores viewed as [B*Q, Hq, ld]); fewer columns store straight from registers
 __host__ __device__ constexpr bool tma_store_for(int N) { return N == 32 || N == 64; }
 
-template <int N>
+// kProbe: the pipeline waits are diagnostic probes bounded by p.max_polls
+// (the instantiation launched only when a test has lowered the limit)
+template <int N, bool kProbe>
 __global__ void __launch_bounds__(kThreads, 1)
     score_tc(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
              const __grid_constant__ CUtensorMap smap, ScoreTcParams p) {
@@ -152,6 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     TileWalk w;
     w.init(p);
     bool ok = true;
+    const uint32_t polls = p.max_polls;  // diagnostic probes (kProbe only)
 
     if (warp == 0) {
         if (lane == 0) {
@@ -183,7 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int b = w.bh / p.Hkv, kvh = w.bh - b * p.Hkv;
                 if (w.seg_first(i)) {
                     const int qb = seg & 1;
-                    if (seg >= 2) ok = mbar_wait(&qempty[qb], ((seg >> 1) - 1) & 1, abort);
+                    if (seg >= 2) ok = pipe_wait<kProbe>(&qempty[qb], ((seg >> 1) - 1) & 1, abort, polls);
                     if (!ok) break;
                     uint8_t *dst = qbuf + qb * kQBuf;
                     mbar_arrive_expect_tx(&qfull[qb], 2u * 128u * p.NQ);
@@ -192,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     misc[3] = seg + 1;
                 }
                 const int s = i % S;
-                if (i >= S) ok = mbar_wait(&empty[s], ((i / S) - 1) & 1, abort);
+                if (i >= S) ok = pipe_wait<kProbe>(&empty[s], ((i / S) - 1) & 1, abort, polls);
                 if (!ok) break;
                 mbar_arrive_expect_tx(&full[s], kTileBytes);
                 if (p.pages.table == nullptr) {
@@ -237,10 +242,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             int seg = 0;
             for (int i = 0; i < w.count && ok; i++) {
                 const int qb = seg & 1;
-                if (w.seg_first(i)) ok = mbar_wait(&qfull[qb], (seg >> 1) & 1, abort);
+                if (w.seg_first(i)) ok = pipe_wait<kProbe>(&qfull[qb], (seg >> 1) & 1, abort, polls);
                 const int s = i % S, buf = i & 1;
-                if (ok) ok = mbar_wait(&full[s], (i / S) & 1, abort);
-                if (ok && i >= 2) ok = mbar_wait(&tempty[buf], ((i >> 1) - 1) & 1, abort);
+                if (ok) ok = pipe_wait<kProbe>(&full[s], (i / S) & 1, abort, polls);
+                if (ok && i >= 2) ok = pipe_wait<kProbe>(&tempty[buf], ((i >> 1) - 1) & 1, abort, polls);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t a0 = smem_addr(stages + s * kTileBytes), b0 = smem_addr(qbuf + qb * kQBuf);
@@ -280,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < w.count; i++) {
             const int b = w.bh / p.Hkv, kvh = w.bh - b * p.Hkv;
             const int buf = i & 1;
-            ok = mbar_wait(&tfull[buf], (i >> 1) & 1, abort);
+            ok = pipe_wait<kProbe>(&tfull[buf], (i >> 1) & 1, abort, polls);
             ok = named_bar_and(1, 128, ok);
             if (!ok) break;
             tc_fence_after();
@@ -315,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int b = w.bh / p.Hkv, kvh = w.bh - b * p.Hkv;
             const int seq_len = p.seq_lens[b];
             const int buf = i & 1;
-            ok = mbar_wait(&tfull[buf], (i >> 1) & 1, abort);
+            ok = pipe_wait<kProbe>(&tfull[buf], (i >> 1) & 1, abort, polls);
             if (!ok) break;
             tc_fence_after();
             const int key = w.t * kTileKeys + quarter * 32 + lane;
@@ -385,20 +390,24 @@ template <int N>
 cudaError_t launch_n(const CUtensorMap &km, const CUtensorMap &qm, const CUtensorMap &sm, const ScoreTcParams &p,
                      int num_sms, cudaStream_t stream, const ScoreTcHook &hook, bool pdl) {
     const size_t smem = smem_bytes<N>();
-    static bool attr_set[64] = {};  // per device: the shared-memory opt-in is a function attribute
+    static std::atomic<bool> attr_set[64] = {};  // per device: the shared-memory opt-in is a function attribute
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-        e = cudaFuncSetAttribute(score_tc<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (dev < 0 || dev >= 64 || !attr_set[dev].load(std::memory_order_acquire)) {
+        e = cudaFuncSetAttribute(score_tc<N, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(score_tc<N, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) attr_set[dev] = true;
+        if (dev >= 0 && dev < 64) attr_set[dev].store(true, std::memory_order_release);
     }
     if (hook.fn) {
         e = hook.fn(hook.ctx);  // e.g. a timing event, right before the launch
         if (e != cudaSuccess) return e;
     }
-    return launch_k(pdl, score_tc<N>, dim3(num_sms), dim3(kThreads), smem, stream, km, qm, sm, p);
+    if (p.max_polls)
+        return launch_k(pdl, score_tc<N, true>, dim3(num_sms), dim3(kThreads), smem, stream, km, qm, sm, p);
+    return launch_k(pdl, score_tc<N, false>, dim3(num_sms), dim3(kThreads), smem, stream, km, qm, sm, p);
 }
 
 }  // namespace
@@ -424,7 +433,8 @@ cudaError_t launch_score_tc(const ScoreTcParams &p, const void *q, const void *k
     CUtensorMap km, qm;
     {
         // K cache as rows of 128 bf16: [B*Hkv*L_max, 128] (paged: [num_pages*Hkv*page, 128]);
-        // boxes of 128 rows (paged: min(page, 128) rows) x 64 dims
+        // boxes of 128 rows (paged: min(page, 128) rows) x 64 dims.  (A 3-D map
+        // [B*Hkv][L_max][128] with boxes one kv-head deep streamed 5 % slower.)
         const bool paged = p.pages.table != nullptr;
         const cuuint64_t nrows = paged ? (cuuint64_t)p.pages.num_pages * p.Hkv << p.pages.page_shift
                                        : (cuuint64_t)p.B * p.Hkv * p.L_max;

@@ -33,6 +33,8 @@
 // maximum lies too far below the row maximum for the sum against it, the row
 // falls back to three exact histogram passes and an ordered compaction pass
 // over the row.
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -610,16 +612,16 @@ template <int kThreads>
 cudaError_t launch_n(const SelectParams &p, cudaStream_t stream, bool pdl) {
     const int rows = p.B * p.Q * p.Hq;
     const size_t smem = select_smem_bytes(kThreads, p.k);
-    static bool attr_set[64] = {};  // per device: the shared-memory opt-in is a function attribute
+    static std::atomic<bool> attr_set[64] = {};  // per device: the shared-memory opt-in is a function attribute
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    if (dev < 0 || dev >= 64 || !attr_set[dev].load(std::memory_order_acquire)) {
         // the largest size any k takes, so that one setting serves every call
         e = cudaFuncSetAttribute(select_topk<kThreads>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)select_smem_bytes(kThreads, kMaxK));
         if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) attr_set[dev] = true;
+        if (dev >= 0 && dev < 64) attr_set[dev].store(true, std::memory_order_release);
     }
     return launch_k(pdl, select_topk<kThreads>, dim3(rows), dim3(kThreads), smem, stream, p);
 }

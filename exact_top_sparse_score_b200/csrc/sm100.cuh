@@ -33,6 +33,21 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                  : "memory");
 }
 
+// Non-blocking probe of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n"
+        ".reg .pred p;\n"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        "selp.b32 %0, 1, 0, p;\n"
+        "}\n"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -58,6 +73,25 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
         if ((i & 63u) == 63u && *abort) return false;
     }
     return false;
+}
+
+// The diagnostic form of a pipeline wait: at most `polls` non-blocking probes,
+// so that a small limit really makes the wait give up.  Kernels use it only
+// in a separate instantiation, launched when a test has lowered the limit;
+// the instantiation that normally runs keeps mbar_wait.
+__device__ __forceinline__ bool mbar_wait_probes(uint64_t *bar, uint32_t parity, uint32_t polls) {
+    for (uint32_t i = 0; i < polls; i++)
+        if (mbar_test_wait(bar, parity)) return true;
+    return false;
+}
+
+// A pipeline wait of a kernel instantiated with or without diagnostic waits.
+template <bool kProbe>
+__device__ __forceinline__ bool pipe_wait(uint64_t *bar, uint32_t parity, volatile int *abort, uint32_t polls) {
+    if constexpr (kProbe)
+        return mbar_wait_probes(bar, parity, polls);
+    else
+        return mbar_wait(bar, parity, abort);
 }
 
 // ---------------------------------------------------------------- TMA

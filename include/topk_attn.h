@@ -42,7 +42,11 @@
  *       tail_mass fp32 [B, Q, Hq]
  *     q, k_cache, v_cache and out must be 16-byte aligned, the workspace
  *     256-byte aligned.
- *     Cache rows at positions >= seq_lens[b] are never read.
+ *     Cache rows at positions >= seq_lens[b] never affect a result.  V rows
+ *     there are never read; K rows are read in tiles of 128 positions, so the
+ *     last tile below seq_lens[b] may read up to 127 rows past it (inside
+ *     [0, L_max) of the same kv-head, or of the page pool for a paged cache),
+ *     and those scores are discarded.
  *   - Arguments are checked on the host before anything is launched; a bad
  *     argument returns an error code and launches nothing.  seq_lens lives on
  *     the device, so its values are checked by the kernels: a sequence whose
@@ -67,7 +71,8 @@ typedef enum {
     TKA_ERR_INVALID_ARG = 1, /* null pointer, misaligned pointer, non-positive size */
     TKA_ERR_UNSUPPORTED = 2, /* valid but outside the supported set above */
     TKA_ERR_WORKSPACE = 3,   /* workspace pointer missing or smaller than required */
-    TKA_ERR_CUDA = 4         /* a launch or CUDA runtime call failed */
+    TKA_ERR_CUDA = 4,        /* a launch or CUDA runtime call failed */
+    TKA_ERR_TIMEOUT = 5      /* topk_attn_last_device_status only: a bounded wait inside a kernel gave up */
 } tka_status;
 
 typedef enum { TKA_F32 = 0, TKA_BF16 = 1 } tka_dtype;
@@ -171,9 +176,9 @@ tka_status topk_attn_decode_certified(const tka_shape *shape, const void *q, con
  * device current) looks up the array's device address; make that first call
  * before any stream capture.  Every call on a device shares the array: calls
  * whose work overlaps on the GPU race, so order them (one stream, or events).
- * Shapes whose topk_attn_workspace_size() exceeds the capacity return
- * TKA_ERR_WORKSPACE; other arguments are checked as in topk_attn_decode.
- * Allocates nothing. */
+ * Arguments are checked first, as topk_attn_decode checks them (an invalid
+ * argument returns that error); a valid call whose topk_attn_workspace_size()
+ * exceeds the capacity returns TKA_ERR_WORKSPACE.  Allocates nothing. */
 size_t topk_attn_static_workspace_capacity(void);
 tka_status topk_attn_decode_static(const tka_shape *shape, const void *q, const void *k_cache,
                                    const void *v_cache, const int32_t *seq_lens, int32_t k, float *out,
@@ -251,6 +256,25 @@ tka_status topk_hisa_attn_decode(const tka_shape *shape, const void *q, const vo
 /* Synchronises `stream`, returns the device status word of the current device
  * (TKA_DEV_* bits raised by kernels since the last read) in *bits and clears it. */
 tka_status topk_attn_device_status(tka_stream_t stream, uint32_t *bits);
+
+/* The same read as a status code: synchronises `stream`, reads and clears the
+ * device status word of the current device, and returns TKA_ERR_TIMEOUT if a
+ * bounded wait inside a kernel gave up (TKA_DEV_TIMEOUT), else
+ * TKA_ERR_INVALID_ARG for a bad sequence length or page (TKA_DEV_BAD_SEQ_LEN,
+ * TKA_DEV_BAD_PAGE), else TKA_ERR_CUDA for a failed internal check
+ * (TKA_DEV_INTERNAL), else TKA_OK.  Errors of the read itself are returned as
+ * topk_attn_device_status returns them. */
+tka_status topk_attn_last_device_status(tka_stream_t stream);
+
+/* Diagnostics: the number of polls after which a pipeline wait inside the
+ * tensor-core score kernel and the block-attention kernel gives up (0, the
+ * default, restores the kernels' own bound of about 4 million polls).  A
+ * wait that gives up raises TKA_DEV_TIMEOUT; the kernel then stops, lets the
+ * copies and tensor-core operations it has issued complete, frees what it
+ * holds and returns, leaving that call's results incomplete.  Meant for tests
+ * of that path (a limit of a few polls makes the first wait give up); it
+ * applies to the calls made after it, process-wide. */
+void topk_attn_debug_set_wait_limit(uint32_t polls);
 
 /* Human-readable name of a status code. */
 const char *topk_attn_status_string(tka_status status);

@@ -46,6 +46,16 @@ def test_library_exports_every_declared_symbol(lib):
 def test_status_strings(lib):
     assert lib.topk_attn_status_string(0) == b"TKA_OK"
     assert lib.topk_attn_status_string(3) == b"TKA_ERR_WORKSPACE"
+    assert lib.topk_attn_status_string(5) == b"TKA_ERR_TIMEOUT"
+
+
+def test_device_status_calls_are_declared_and_exported(lib):
+    names = declared_functions()
+    for n in ["topk_attn_device_status", "topk_attn_last_device_status", "topk_attn_debug_set_wait_limit"]:
+        assert n in names and hasattr(lib, n)
+    # the wait limit is a plain host-side setting: setting and clearing it launches nothing
+    bd.topk_attn_debug_set_wait_limit(8)
+    bd.topk_attn_debug_set_wait_limit(0)
 
 
 def shape(B=2, Q=1, Hq=8, Hkv=2, d=128, L=1000, dtype=1, scale=0.0):
@@ -124,6 +134,49 @@ def test_binding_rejects_mismatched_output_buffers(lib):
         tka.topk_attn_decode(q, kc, kc, lens, 8, tail_mass=torch.zeros(1, 1, 3, dtype=torch.float32))
     with pytest.raises(ValueError):  # host tensors: there is no CPU path
         tka.topk_attn_decode(q, kc, kc, lens, 8)
+
+
+def test_static_call_checks_arguments_before_its_capacity(lib):
+    # a null pointer is an argument error even on a shape too large for the array
+    big = shape(B=8, Q=1, Hq=32, Hkv=8, L=65536)
+    assert bd.topk_attn_workspace_size(big, 2048) > lib.topk_attn_static_workspace_capacity()
+    assert lib.topk_attn_decode_static(ctypes.byref(big), None, FAKE, FAKE, FAKE, 2048, FAKE, FAKE, FAKE,
+                                       None) == INVALID
+    assert lib.topk_attn_decode_static(ctypes.byref(big), FAKE + 8, FAKE, FAKE, FAKE, 2048, FAKE, FAKE, FAKE,
+                                       None) == INVALID
+    assert lib.topk_attn_decode_static(ctypes.byref(big), FAKE, FAKE, FAKE, FAKE, 2048, FAKE, FAKE, FAKE,
+                                       None) == WORKSPACE
+
+
+def test_static_binding_checks_v_cache_before_any_launch(lib):
+    import torch
+    import exact_top_sparse_score_b200 as tka
+    q = torch.zeros(1, 1, 4, 128, dtype=torch.bfloat16)
+    kc = torch.zeros(1, 2, 64, 128, dtype=torch.bfloat16)
+    lens = torch.full((1,), 64, dtype=torch.int32)
+    out = torch.zeros(1, 1, 4, 128)
+    idx = torch.zeros(1, 1, 4, 8, dtype=torch.int32)
+    for vc in (torch.zeros(1, 2, 32, 128, dtype=torch.bfloat16), torch.zeros(1, 2, 64, 128)):
+        with pytest.raises(TypeError, match="v_cache"):
+            tka.topk_attn_decode_static(q, kc, vc, lens, 8, out=out, idx=idx)
+
+
+class _FakeCuda:
+    """Stands in for a CUDA tensor in the binding's host-side checks (no GPU here)."""
+
+    def __init__(self, index):
+        import torch
+        self.is_cuda = True
+        self.device = torch.device("cuda", index)
+
+    def is_contiguous(self):
+        return True
+
+
+def test_binding_requires_every_tensor_on_one_device():
+    bd._check_cuda(q=_FakeCuda(0), k_cache=_FakeCuda(0), out=None)
+    with pytest.raises(ValueError, match="k_cache is on cuda:1"):
+        bd._check_cuda(q=_FakeCuda(0), k_cache=_FakeCuda(1))
 
 
 def test_every_entry_point_refuses_host_tensors(lib):

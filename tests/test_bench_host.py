@@ -66,3 +66,14 @@ def test_reference_arm_other_ranks_do_no_work():
 def test_too_few_warmup_steps_are_refused():
     rc, out = _run_bench("--impl", "reference", "--config", "1", "--steps", "3", "--warmup", "2")
     assert rc != 0 and out == []
+
+
+def test_both_arms_describe_the_workload_with_one_config_object():
+    # the reference arm prints exactly the config object the CUDA arm builds
+    import argparse
+    import workloads
+    rc, out = _run_bench("--impl", "reference", "--config", "1", "--steps", "3", "--warmup", "3")
+    assert rc == 0 and len(out) == 1
+    w = workloads.config_workload(1, seed=1001)
+    args = argparse.Namespace(certified_eps=None, paged=None, hisa=None, indexer=None)
+    assert out[0]["config"] == bench.workload_config(w, w.k, 1, args)

@@ -48,6 +48,8 @@ def test_static_workspace_matches_regular_entry_point_twice(cuda_device):
         (workloads.make_workload(2, 1, 32, 8, 20000, dtype="bf16", seq_lens=[20000, 13001], k_mean_std=0.5,
                                  seed=901), 512),
         (workloads.make_workload(3, 2, 16, 4, 9000, dtype="bf16", seq_lens=[9000, 4444, 77], seed=902), 300),
+        # fp32 cache: the CUDA-core scorer's scores in the shared array, with another k
+        (workloads.make_workload(2, 1, 8, 4, 6000, dtype="f32", seq_lens=[6000, 2500], seed=903), 77),
     ]
     for w, k in cases:
         q, kc, vc, lens = to_device(w)
@@ -60,6 +62,29 @@ def test_static_workspace_matches_regular_entry_point_twice(cuda_device):
         np.testing.assert_allclose(got[0].cpu().numpy(), ref[0].cpu().numpy(), atol=atol, rtol=rtol)
         assert torch.equal(got[1], ref[1])
         assert (got[2] - ref[2]).abs().max().item() <= TAIL_TOL
+
+
+@pytest.mark.gpu
+def test_static_call_allocates_nothing(cuda_device):
+    """The binding-level call with every output preallocated leaves the torch
+    allocator's count of allocated bytes unchanged (and the library itself
+    never calls a device allocator)."""
+    w = workloads.make_workload(2, 1, 32, 8, 12000, dtype="bf16", seed=904)
+    q, kc, vc, lens = to_device(w)
+    k = 400
+    out = torch.empty((2, 1, 32, 128), dtype=torch.float32, device=q.device)
+    idx = torch.empty((2, 1, 32, k), dtype=torch.int32, device=q.device)
+    tail = torch.empty((2, 1, 32), dtype=torch.float32, device=q.device)
+    tka.topk_attn_decode_static(q, kc, vc, lens, k, out=out, idx=idx, tail_mass=tail)  # first call: address lookup
+    torch.cuda.synchronize()
+    before = torch.cuda.memory_allocated()
+    for _ in range(3):
+        tka.topk_attn_decode_static(q, kc, vc, lens, k, out=out, idx=idx, tail_mass=tail)
+    torch.cuda.synchronize()
+    assert torch.cuda.memory_allocated() == before
+    assert tka.topk_attn_device_status() == 0
+    ref = tka.topk_attn_decode(q, kc, vc, lens, k)
+    assert torch.equal(idx, ref[1])
 
 
 def test_static_workspace_rejects_shapes_beyond_its_capacity():
