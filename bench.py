@@ -133,6 +133,15 @@ def alg_bytes_block(w):
     return total + rows * w.d * (elem_bytes(w) + 4) + rows * (top + 1) * 4
 
 
+def block_select_launches(G, nblk_max):
+    """Kernels the block selection takes: one on a cluster of 8 CTAs per
+    (sequence, kv-head) when a kv-head's block scores fit its shared memory
+    (96 KB: queries, G chunks of scores, one head's gathered scores and keys),
+    else block scores + one top-k CTA per row."""
+    chmax = -(-nblk_max // 8)
+    return 1 if G * 32 * 16 + G * chmax * 4 + nblk_max * 8 <= 96 * 1024 else 2
+
+
 def measured_hbm_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -337,7 +346,7 @@ def run_ours(args, world, rank, local):
                          dtype=torch.uint8, device=dev)
         out = torch.empty((w.B, w.Q, w.Hq, w.d), dtype=torch.float32, device=dev)
         bidx = torch.empty((w.B, w.Q, w.Hq, w.top_blocks + 1), dtype=torch.int32, device=dev)
-        launches_per_step = 3  # block_scores, block_topk, block_attn
+        launches_per_step = block_select_launches(w.G, -(-w.L_max // w.block_size)) + 1  # + block_attn
 
         def step(events=None, qq=q):
             if events:
@@ -384,7 +393,8 @@ def run_ours(args, world, rank, local):
             h_bidx = torch.empty((w.B, 1, w.Hq, h_top), dtype=torch.int32, device=dev)
             ws = torch.empty(tka._binding.load_library().topk_hisa_attn_workspace_size(
                 make_shape(q, kc), h_bs, h_top, k), dtype=torch.uint8, device=dev)
-            launches_per_step = 5  # block_scores, block_topk, hisa_scores, select, gather
+            # block selection, hisa_scores, select, gather
+            launches_per_step = block_select_launches(w.G, -(-w.L_max // h_bs)) + 3
 
             def step(events=None, qq=q):
                 if events:

@@ -23,6 +23,8 @@
 //                 order.
 #include <string.h>
 
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -88,6 +90,8 @@ __global__ void __launch_bounds__(128) block_pool(BlockPoolParams p) {
 
 constexpr int kScoreBlocks = 64;  // blocks per CTA of block_scores
 constexpr int kSelThreads = 256;
+constexpr int kClusterCtas = 8;   // CTAs of block_select_cluster per (b, kv-head)
+constexpr size_t kClusterSmem = 96 * 1024;  // shared memory block_select_cluster may take
 
 // bscore[row, j] = scale * <q_row, block_keys[b, kvh, j, :]> for the competing
 // blocks j < nblk - 1 of every query row of kv-head kvh.  Eight lanes share a
@@ -139,41 +143,15 @@ __global__ void __launch_bounds__(kSelThreads) block_scores(BlockSelectParams p)
     }
 }
 
-// Keeps, per query row, the top_blocks competing blocks with the highest
-// scores (ties to the lower block) plus the current block, ascending.  The
-// threshold key T (the top_blocks-th largest) comes from a radix selection
-// over the scores' order-preserving keys, 8 bits at a time; the kept blocks
-// are then compacted in block order, the blocks whose key equals T kept from
-// the lowest index up.
-__global__ void __launch_bounds__(kSelThreads) block_topk(BlockSelectParams p) {
-    pdl_wait();  // inputs may come from the kernel before
-    pdl_trigger();
-    extern __shared__ uint32_t ukey[];  // [ncomp]
-    __shared__ uint32_t hist[256];
-    __shared__ uint32_t tmp[32];
-    __shared__ uint32_t s_bin, s_above;
-    const int row = blockIdx.x, b = row / p.Hq;
-    const int seq_len = p.seq_lens[b];
-    if (seq_len < 1 || seq_len > p.L_max) {
-        if (threadIdx.x == 0) raise_status(p.status, TKA_DEV_BAD_SEQ_LEN);
-        return;
-    }
-    if (threadIdx.x == 0 && p.counters) p.counters[row] = 0u;
-    const int nblk = (seq_len + p.block_size - 1) / p.block_size;
-    const int ncomp = nblk - p.force_last;  // blocks competing for the top_blocks slots
-    const int top = p.top_blocks;
-    const int width = top + p.force_last;
-    int32_t *out = p.block_idx + (size_t)row * width;
-    if (ncomp <= top) {  // every block is kept: nothing to rank
-        for (int i = threadIdx.x; i < width; i += kSelThreads) out[i] = i < nblk ? i : -1;
-        return;
-    }
-    if (top == 0) {  // only the current block
-        if (threadIdx.x == 0) out[0] = nblk - 1;
-        return;
-    }
-    const float *sc = p.bscore + (size_t)row * p.nblk_max;
-    for (int j = threadIdx.x; j < ncomp; j += kSelThreads) ukey[j] = order_key(sc[j]);
+// Keeps the `top` largest of the ncomp keys ukey[0..ncomp) (ties to the lower
+// block) and, when force_last is set, the current block nblk - 1; writes them
+// ascending to out[0..top + force_last).  Requires 0 < top < ncomp.  The
+// threshold key T (the top-th largest) comes from a radix selection over the
+// keys, 8 bits at a time; the kept blocks are then compacted in block order,
+// the blocks whose key equals T kept from the lowest index up.  Called by the
+// whole block (kSelThreads threads).
+__device__ void keep_top_blocks(const uint32_t *ukey, int ncomp, int nblk, int top, int force_last, int32_t *out,
+                                unsigned *status, uint32_t *hist, uint32_t *tmp, uint32_t *s_bin, uint32_t *s_above) {
     uint32_t prefix = 0u, mask = 0u, need = (uint32_t)top;
     for (int shift = 24; shift >= 0; shift -= 8) {
         for (int i = threadIdx.x; i < 256; i += kSelThreads) hist[i] = 0u;
@@ -183,10 +161,10 @@ __global__ void __launch_bounds__(kSelThreads) block_topk(BlockSelectParams p) {
             if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
         }
         __syncthreads();
-        find_bin(hist, 256, need, tmp, &s_bin, &s_above);
-        prefix |= s_bin << shift;
+        find_bin(hist, 256, need, tmp, s_bin, s_above);
+        prefix |= *s_bin << shift;
         mask |= 255u << shift;
-        need -= s_above;
+        need -= *s_above;
     }
     const uint32_t T = prefix;  // keys above T are kept, and the first `need` keys equal to T
     const int per = (ncomp + kSelThreads - 1) / kSelThreads;
@@ -201,7 +179,7 @@ __global__ void __launch_bounds__(kSelThreads) block_topk(BlockSelectParams p) {
     const uint32_t take_eq = need > eq_before ? min(eq, need - eq_before) : 0u;
     uint32_t pos = block_excl_scan(gt + take_eq, tmp, &total);
     if (total != (uint32_t)top) {  // never true unless the selection above is wrong
-        if (threadIdx.x == 0) raise_status(p.status, TKA_DEV_INTERNAL);
+        if (threadIdx.x == 0) raise_status(status, TKA_DEV_INTERNAL);
         return;
     }
     uint32_t eqr = eq_before;
@@ -211,7 +189,245 @@ __global__ void __launch_bounds__(kSelThreads) block_topk(BlockSelectParams p) {
         if (u == T) keep = eqr++ < need;
         if (keep) out[pos++] = j;
     }
-    if (threadIdx.x == 0 && p.force_last) out[top] = nblk - 1;  // the current block has the highest index
+    if (threadIdx.x == 0 && force_last) out[top] = nblk - 1;  // the current block has the highest index
+}
+
+// keep_top_blocks with one histogram level instead of radix levels: the
+// scores' minimum and maximum, a histogram in 2048 bins of equal width between
+// them, the bin b* that holds the top-th score; when b* is kept whole, every
+// block whose bin is at or above b* is kept, else the exact top-th key T is
+// ranked among the (at most 32) blocks of b* by one warp, ties at T kept from
+// the lowest block up.  One block-wide scan then writes the kept blocks in
+// ascending order.  Returns false, having written nothing, when more than 32
+// blocks share b* or the scores are all equal (the caller takes the radix
+// route).  x holds the ncomp competing blocks' scores; ukey receives their
+// order keys.
+__device__ bool keep_top_blocks_hist(const float *x, uint32_t *ukey, int ncomp, int nblk, int top, int force_last,
+                                     int32_t *out, unsigned *status, uint32_t *hist, uint32_t *tmp, uint32_t *scal,
+                                     float *red) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    constexpr int kWarps = kSelThreads / 32;
+    float lo = INFINITY, hi = -INFINITY;
+    for (int j = threadIdx.x; j < ncomp; j += kSelThreads) {
+        const float v = x[j];
+        ukey[j] = order_key(v);
+        lo = fminf(lo, v);
+        hi = fmaxf(hi, v);
+    }
+    for (int i = threadIdx.x; i < 2048; i += kSelThreads) hist[i] = 0u;
+    lo = warp_min(lo);
+    hi = warp_max(hi);
+    if (lane == 0) {
+        red[warp] = lo;
+        red[kWarps + warp] = hi;
+    }
+    if (threadIdx.x == 0) scal[4] = 0u;
+    __syncthreads();
+    lo = warp_min(lane < kWarps ? red[lane] : INFINITY);
+    hi = warp_max(lane < kWarps ? red[kWarps + lane] : -INFINITY);
+    if (!(hi > lo) || !(hi - lo < INFINITY)) return false;  // all equal (or not finite): radix route
+    const float scale = 2048.f / (hi - lo);
+    auto bin = [&](float v) { return min(2047u, (uint32_t)((v - lo) * scale)); };
+    for (int j = threadIdx.x; j < ncomp; j += kSelThreads) atomicAdd(&hist[bin(x[j])], 1u);
+    __syncthreads();
+    block_find_bins<2048>(hist, (uint32_t)top, (uint32_t)top, tmp, scal);
+    const uint32_t bstar = scal[0];
+    const uint32_t c_star = hist[bstar], r = (uint32_t)top - scal[1];  // 1 <= r <= c_star
+    if (c_star > 32u) return false;  // uniform: every thread read the same words
+    uint32_t T = 0u, r_eq = 0u;
+    const bool by_bin = r == c_star;
+    if (!by_bin) {
+        uint64_t *cand = reinterpret_cast<uint64_t *>(hist);  // [32] (key, block): the bins are no longer read
+        __syncthreads();
+        for (int j = threadIdx.x; j < ncomp; j += kSelThreads)
+            if (bin(x[j]) == bstar) cand[atomicAdd(&scal[4], 1u)] = ((uint64_t)ukey[j] << 32) | (uint32_t)j;
+        __syncthreads();
+        if (warp == 0) {
+            const uint32_t mine = lane < (int)c_star ? (uint32_t)(cand[lane] >> 32) : 0u;
+            uint32_t g = 0u, e = 0u;
+            for (uint32_t i = 0; i < c_star; i++) {
+                const uint32_t o = (uint32_t)(cand[i] >> 32);
+                g += o > mine;
+                e += o == mine;
+            }
+            const uint32_t hit = __ballot_sync(0xffffffffu, lane < (int)c_star && g < r && r <= g + e);
+            const int L = hit ? __ffs(hit) - 1 : 0;
+            const uint32_t tk = __shfl_sync(0xffffffffu, mine, L), tg = __shfl_sync(0xffffffffu, g, L);
+            if (lane == 0) {
+                scal[5] = tk;
+                scal[6] = r - tg;
+                if (!hit) raise_status(status, TKA_DEV_INTERNAL);
+            }
+        }
+        __syncthreads();
+        T = scal[5];
+        r_eq = scal[6];
+    }
+    // kept: a bin above b*, all of b* when it is kept whole, else a key above
+    // T or one of the first r_eq keys equal to T (in block order)
+    const int per = (ncomp + kSelThreads - 1) / kSelThreads;
+    const int j0 = threadIdx.x * per, j1 = min(j0 + per, ncomp);
+    uint32_t kept = 0u, ties = 0u;
+    for (int j = j0; j < j1; j++) {
+        const uint32_t bj = bin(x[j]);
+        if (by_bin) {
+            kept += bj >= bstar;
+        } else {
+            kept += bj > bstar || (bj == bstar && ukey[j] > T);
+            ties += bj == bstar && ukey[j] == T;
+        }
+    }
+    uint32_t total;
+    const uint32_t before = block_excl_scan(kept | (ties << 16), tmp, &total);  // both counts < 2^16
+    uint32_t pos = before & 0xffffu, tie_rank = before >> 16;
+    const uint32_t written = (total & 0xffffu) + min(total >> 16, r_eq);
+    if (written != (uint32_t)top) {  // never true unless the selection above is wrong
+        if (threadIdx.x == 0) raise_status(status, TKA_DEV_INTERNAL);
+        return true;
+    }
+    pos += min(tie_rank, r_eq);  // the ties before this thread's that are kept
+    for (int j = j0; j < j1; j++) {
+        const uint32_t bj = bin(x[j]);
+        bool keep;
+        if (by_bin) {
+            keep = bj >= bstar;
+        } else {
+            keep = bj > bstar || (bj == bstar && ukey[j] > T);
+            if (bj == bstar && ukey[j] == T) keep = tie_rank++ < r_eq;
+        }
+        if (keep) out[pos++] = j;
+    }
+    if (threadIdx.x == 0 && force_last) out[top] = nblk - 1;  // the current block has the highest index
+    return true;
+}
+
+// The easy cases of a row's block list: every competing block kept, or only
+// the current block.  Returns false when the row needs a selection.
+__device__ __forceinline__ bool trivial_blocks(int ncomp, int nblk, int top, int width, int32_t *out) {
+    if (ncomp <= top) {  // every block is kept: nothing to rank
+        for (int i = threadIdx.x; i < width; i += kSelThreads) out[i] = i < nblk ? i : -1;
+        return true;
+    }
+    if (top == 0) {  // only the current block
+        if (threadIdx.x == 0) out[0] = nblk - 1;
+        return true;
+    }
+    return false;
+}
+
+// One CTA per query row: the row's competing blocks' scores (from
+// block_scores), then keep_top_blocks.
+__global__ void __launch_bounds__(kSelThreads) block_topk(BlockSelectParams p) {
+    pdl_wait();  // inputs may come from the kernel before
+    pdl_trigger();
+    extern __shared__ uint32_t ukey[];  // [ncomp]
+    __shared__ __align__(16) uint32_t hist[2048];
+    __shared__ uint32_t tmp[32];
+    __shared__ uint32_t scal[8];
+    __shared__ float red[16];
+    const int row = blockIdx.x, b = row / p.Hq;
+    const int seq_len = p.seq_lens[b];
+    if (seq_len < 1 || seq_len > p.L_max) {
+        if (threadIdx.x == 0) raise_status(p.status, TKA_DEV_BAD_SEQ_LEN);
+        return;
+    }
+    if (threadIdx.x == 0 && p.counters) p.counters[row] = 0u;
+    const int nblk = (seq_len + p.block_size - 1) / p.block_size;
+    const int ncomp = nblk - p.force_last;  // blocks competing for the top_blocks slots
+    const int top = p.top_blocks, width = top + p.force_last;
+    int32_t *out = p.block_idx + (size_t)row * width;
+    if (trivial_blocks(ncomp, nblk, top, width, out)) return;
+    const float *sc = p.bscore + (size_t)row * p.nblk_max;
+    if (keep_top_blocks_hist(sc, ukey, ncomp, nblk, top, p.force_last, out, p.status, hist, tmp, scal, red)) return;
+    __syncthreads();
+    keep_top_blocks(ukey, ncomp, nblk, top, p.force_last, out, p.status, hist, tmp, &scal[0], &scal[1]);
+}
+
+// block_scores and block_topk in one launch, for a kv-head's block scores that
+// fit in shared memory: a cluster of kClusterCtas CTAs per (b, kv-head).  CTA
+// r of the cluster scores the r-th contiguous chunk of the competing blocks
+// against all G query heads of the kv-head (each block key read once) into
+// its own shared memory; after a cluster barrier, CTA g mod kClusterCtas
+// gathers head g's scores of every chunk from the other CTAs' shared memory
+// (distributed shared memory) and keeps its top blocks.  A last cluster
+// barrier keeps every CTA's scores in place until all gathers are done.
+template <typename T>
+__global__ void __launch_bounds__(kSelThreads) block_select_cluster(BlockSelectParams p) {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    pdl_wait();  // inputs may come from the kernel before
+    pdl_trigger();
+    extern __shared__ float4 dyn4[];
+    __shared__ __align__(16) uint32_t hist[2048];
+    __shared__ uint32_t tmp[32];
+    __shared__ uint32_t scal[8];
+    __shared__ float red[16];
+    const int G = p.G;
+    const int chmax = (p.nblk_max + kClusterCtas - 1) / kClusterCtas;
+    float4 *qs = dyn4;                                          // [G][32]
+    float *sc = reinterpret_cast<float *>(dyn4 + G * 32);       // [G][chmax]
+    uint32_t *ukey = reinterpret_cast<uint32_t *>(sc + (size_t)G * chmax);  // [nblk_max]
+    float *xs = reinterpret_cast<float *>(ukey + p.nblk_max);               // [nblk_max] one head's scores
+    const int rank = (int)cluster.block_rank();
+    const int bh = blockIdx.y, b = bh / p.Hkv, kvh = bh - b * p.Hkv;
+    const int seq_len = p.seq_lens[b];
+    const bool valid = seq_len >= 1 && seq_len <= p.L_max;
+    const int nblk = valid ? (seq_len + p.block_size - 1) / p.block_size : 0;
+    const int ncomp = nblk - p.force_last;
+    const int top = p.top_blocks, width = top + p.force_last;
+    const bool rank_rows = valid && ncomp > top && top > 0;
+    const int ch = (max(ncomp, 1) + kClusterCtas - 1) / kClusterCtas;  // <= chmax
+    if (rank_rows) {
+        const T *q = reinterpret_cast<const T *>(p.q) + ((size_t)b * p.Hq + (size_t)kvh * G) * kHeadDim;
+        for (int e = threadIdx.x; e < G * 32; e += kSelThreads) qs[e] = load4(q + 4 * e);
+        __syncthreads();
+        // eight lanes per block, lane c holding float4 columns c, c + 8, c + 16, c + 24
+        const int c = threadIdx.x & 7;
+        const float4 *bk = reinterpret_cast<const float4 *>(p.block_keys + (size_t)bh * p.nblk_max * kHeadDim);
+        const int j_lo = rank * ch, j_hi = min(ncomp, j_lo + ch);
+        for (int j0 = j_lo; j0 < j_hi; j0 += kSelThreads / 8) {
+            const int j = j0 + (threadIdx.x >> 3);
+            float4 kv[4];
+#pragma unroll
+            for (int u = 0; u < 4; u++)
+                kv[u] = j < j_hi ? __ldg(bk + (size_t)j * 32 + c + 8 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int g = 0; g < G; g++) {
+                float s = 0.f;
+#pragma unroll
+                for (int u = 0; u < 4; u++) {
+                    const float4 qv = qs[g * 32 + c + 8 * u];
+                    s += qv.x * kv[u].x + qv.y * kv[u].y + qv.z * kv[u].z + qv.w * kv[u].w;
+                }
+                s += __shfl_xor_sync(0xffffffffu, s, 1);
+                s += __shfl_xor_sync(0xffffffffu, s, 2);
+                s += __shfl_xor_sync(0xffffffffu, s, 4);
+                if (c == 0 && j < j_hi) sc[(size_t)g * chmax + (j - j_lo)] = s * p.scale;
+            }
+        }
+    }
+    cluster.sync();  // every chunk's scores are in place
+    for (int g = rank; g < G; g += kClusterCtas) {
+        const int row = b * p.Hq + kvh * G + g;
+        if (!valid) {
+            if (threadIdx.x == 0) raise_status(p.status, TKA_DEV_BAD_SEQ_LEN);
+            continue;
+        }
+        if (threadIdx.x == 0 && p.counters) p.counters[row] = 0u;
+        int32_t *out = p.block_idx + (size_t)row * width;
+        if (trivial_blocks(ncomp, nblk, top, width, out)) continue;
+        for (int j = threadIdx.x; j < ncomp; j += kSelThreads) {
+            const int owner = j / ch;
+            const float *remote = cluster.map_shared_rank(sc, owner);
+            xs[j] = remote[(size_t)g * chmax + (j - owner * ch)];
+        }
+        __syncthreads();
+        if (!keep_top_blocks_hist(xs, ukey, ncomp, nblk, top, p.force_last, out, p.status, hist, tmp, scal, red)) {
+            __syncthreads();
+            keep_top_blocks(ukey, ncomp, nblk, top, p.force_last, out, p.status, hist, tmp, &scal[0], &scal[1]);
+        }
+        __syncthreads();  // xs and ukey are rewritten for the next head
+    }
+    cluster.sync();  // no CTA's scores go away while another CTA still reads them
 }
 
 // ---------------------------------------------------------------- hisa_scores
@@ -665,9 +881,14 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
 }
 
 
+// Opts a kernel in to `smem` bytes of dynamic shared memory when that, with
+// the kernel's static shared memory, passes the 48 KB available without it.
 template <typename F>
 cudaError_t allow_smem(F *kernel, size_t smem) {
-    if (smem <= 48 * 1024) return cudaSuccess;
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
+    if (e != cudaSuccess) return e;
+    if (smem + fa.sharedSizeBytes <= 48 * 1024) return cudaSuccess;
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
 }
 
@@ -680,9 +901,37 @@ cudaError_t launch_block_pool(const BlockPoolParams &p, cudaStream_t stream) {
 }
 
 cudaError_t launch_block_select(const BlockSelectParams &p, cudaStream_t stream) {
+    cudaError_t e;
+    // one launch on a cluster per (b, kv-head) when the kv-head's scores fit
+    // in shared memory: query rows, G chunks of scores and the gathered keys
+    const size_t chmax = (p.nblk_max + kClusterCtas - 1) / kClusterCtas;
+    const size_t csmem = (size_t)p.G * 32 * sizeof(float4) + (size_t)p.G * chmax * sizeof(float) +
+                         (size_t)p.nblk_max * (sizeof(uint32_t) + sizeof(float));
+    if (csmem <= kClusterSmem) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(kClusterCtas, p.B * p.Hkv);
+        cfg.blockDim = dim3(kSelThreads);
+        cfg.dynamicSmemBytes = csmem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = kClusterCtas;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 2;
+        if (p.dtype == TKA_BF16) {
+            if ((e = allow_smem(block_select_cluster<__nv_bfloat16>, csmem)) != cudaSuccess) return e;
+            return cudaLaunchKernelEx(&cfg, block_select_cluster<__nv_bfloat16>, p);
+        }
+        if ((e = allow_smem(block_select_cluster<float>, csmem)) != cudaSuccess) return e;
+        return cudaLaunchKernelEx(&cfg, block_select_cluster<float>, p);
+    }
+    // otherwise: scores to the workspace, then one CTA per row
     const dim3 sgrid((p.nblk_max + kScoreBlocks - 1) / kScoreBlocks, p.B * p.Hkv);
     const size_t qsmem = (size_t)p.G * kHeadDim * sizeof(float);
-    cudaError_t e;
     if (p.dtype == TKA_BF16) {
         if ((e = allow_smem(block_scores<__nv_bfloat16>, qsmem)) != cudaSuccess) return e;
         e = launch_k(true, block_scores<__nv_bfloat16>, sgrid, dim3(kSelThreads), qsmem, stream, p);
@@ -692,7 +941,7 @@ cudaError_t launch_block_select(const BlockSelectParams &p, cudaStream_t stream)
     }
     if (e != cudaSuccess) return e;
     const size_t ksmem = (size_t)p.nblk_max * sizeof(uint32_t);
-    if ((e = allow_smem(block_topk, ksmem)) != cudaSuccess) return e;
+    if ((e = allow_smem(block_topk, ksmem)) != cudaSuccess) return e;  // + 8.3 KB of static shared memory
     return launch_k(true, block_topk, dim3(p.B * p.Hq), dim3(kSelThreads), ksmem, stream, p);
 }
 

@@ -190,7 +190,9 @@ BLOCK_CASES = [
     ("bf16", 1, 8, 2, 256, [1], 64, 4),                 # one-key sequence
     ("bf16", 2, 8, 2, 3000, [3000, 2500], 32, 0),       # only the current block
     ("bf16", 1, 8, 2, 65536, [65521], 16, 255),         # 4095 blocks, the largest top_blocks
-    ("bf16", 2, 8, 2, 32768, [32768, 20000], 16, 40),   # 2048 blocks: a warp per row, 64 keys per lane
+    ("bf16", 2, 8, 2, 32768, [32768, 20000], 16, 40),   # 2048 blocks
+    ("bf16", 1, 64, 2, 131072, [131000], 16, 8),        # G = 32 x 8192 blocks: the kv-head's scores exceed the
+                                                        # cluster's shared memory -> two launches via the workspace
 ]
 
 
