@@ -133,6 +133,14 @@ def alg_bytes_block(w):
     return total + rows * w.d * (elem_bytes(w) + 4) + rows * (top + 1) * 4
 
 
+def one_launch(w, num_sms):
+    """Whether the library decodes this token workload in one launch (a small
+    cache: at most 65536 rows in all, no more query rows or kv-heads than SMs,
+    at most 64 query rows per kv-head)."""
+    rows, units = w.B * w.Q * w.Hq, w.B * w.Hkv
+    return w.B * w.Hkv * w.L_max <= 65536 and rows <= num_sms and units <= num_sms and w.Q * (w.Hq // w.Hkv) <= 64
+
+
 def block_select_launches(G, nblk_max):
     """Kernels the block selection takes: one on a cluster of 8 CTAs per
     (sequence, kv-head) when a kv-head's block scores fit its shared memory
@@ -362,7 +370,7 @@ def run_ours(args, world, rank, local):
         out = torch.empty((w.B, w.Q, w.Hq, w.d), dtype=torch.float32, device=dev)
         idx = torch.empty((w.B, w.Q, w.Hq, k), dtype=torch.int32, device=dev)
         tail = torch.empty((w.B, w.Q, w.Hq), dtype=torch.float32, device=dev)
-        launches_per_step = 3
+        launches_per_step = 1 if one_launch(w, torch.cuda.get_device_properties(dev).multi_processor_count) else 3
         if certified:
             k_used = torch.empty((w.B, w.Q, w.Hq), dtype=torch.int32, device=dev)
             launches_per_step = 4  # + certify

@@ -403,6 +403,43 @@ tka_status launch_rest(const DecodeArgs &a, cudaStream_t s, int select_threads, 
     return TKA_OK;
 }
 
+// Whether a decode is small enough for the one-launch path: at most kTinyKeys
+// cache rows in all, no more query rows and kv-heads than SMs (one CTA per
+// query row after the grid barrier, every CTA resident at once), and at most
+// 64 query rows per kv-head (their query vectors sit in shared memory).
+constexpr long long kTinyKeys = 1 << 16;
+
+bool use_tiny(const tka_shape *sh, int num_sms) {
+    const long long rows = (long long)sh->B * sh->Q * sh->Hq, units = (long long)sh->B * sh->Hkv;
+    return (long long)sh->B * sh->Hkv * sh->L_max <= kTinyKeys && rows <= num_sms && units <= num_sms &&
+           sh->Q * (sh->Hq / sh->Hkv) <= 64;
+}
+
+tka_status launch_tiny_decode(const DecodeArgs &a, cudaStream_t s) {
+    const tka_shape *sh = a.shape;
+    TinyParams tp;
+    SelectParams &se = tp.sel;
+    se.status = a.dev->status;
+    se.scores = reinterpret_cast<const float *>(a.ws + a.L.scores);
+    se.seq_lens = a.seq_lens;
+    se.B = sh->B; se.Q = sh->Q; se.Hq = sh->Hq; se.L_max = sh->L_max; se.ld = a.L.ld; se.k = a.k;
+    se.idx = a.idx;
+    se.w = reinterpret_cast<float *>(a.ws + a.L.weights);
+    se.stats = reinterpret_cast<float4 *>(a.ws + a.L.stats);
+    se.tail = a.tail;
+    se.counters = reinterpret_cast<unsigned *>(a.ws + a.L.counters);
+    tp.scores = reinterpret_cast<float *>(a.ws + a.L.scores);
+    tp.q = a.q; tp.k = a.k_cache; tp.v = a.v_cache;
+    tp.Hkv = sh->Hkv; tp.G = a.G; tp.dtype = sh->dtype;
+    tp.scale = resolve_scale(sh);
+    tp.out = a.out;
+    const int units = sh->B * sh->Hkv, rows = sh->B * sh->Q * sh->Hq;
+    const int chunks = (sh->L_max + 127) / 128;
+    tp.cpb = max(1, min(a.dev->num_sms / units, chunks));
+    const int grid = max(units * tp.cpb, rows);
+    return launch_tiny(tp, grid, s) == cudaSuccess ? TKA_OK : TKA_ERR_CUDA;
+}
+
 // Score -> select (k) -> [certify] -> gather on `stream`.
 tka_status decode_impl(const tka_shape *shape, const void *q, const void *k_cache, const void *v_cache,
                        const int32_t *seq_lens, int32_t k, float *out, int32_t *idx, float *tail_mass,
@@ -438,6 +475,10 @@ tka_status decode_impl(const tka_shape *shape, const void *q, const void *k_cach
     // 2^31 rows, 512 GB, does not fit one GPU; the CUDA-core scorer takes it)
     a.tc = score_tc_supported(shape->dtype, shape->Q * a.G) &&
            (pages || (long long)shape->B * shape->Hkv * shape->L_max < (1LL << 31));
+
+    // a small problem (no events to record between steps): one launch does
+    // all three steps
+    if (!events && !cert && !pages && use_tiny(shape, a.dev->num_sms)) return launch_tiny_decode(a, s);
 
     st = launch_score(a, s, events);
     if (st != TKA_OK) return st;

@@ -156,6 +156,19 @@ struct BlockAttnParams {
     uint32_t max_polls = 0;   // polls before a pipeline wait gives up (0: the default bound)
 };
 
+// The one-launch decode of a small problem (tiny.cu): the select step's
+// parameters (scores, idx, w, stats, tail, counters, shape and k) plus what
+// scoring and the attention step need.
+struct TinyParams {
+    SelectParams sel;
+    float *scores;            // the same buffer as sel.scores, written by the scoring phase
+    const void *q, *k, *v;    // q [B, Q, Hq, 128]; caches [B, Hkv, L_max, 128]
+    int Hkv, G, dtype;
+    float scale;
+    float *out;               // [B*Q*Hq, 128]
+    int cpb;                  // CTAs scoring each kv-head
+};
+
 // Launches kernel<<<grid, block, smem, stream>>>(args...), allowed to start
 // early behind the previous kernel on the stream when pdl is set (the kernel
 // calls pdl_wait() before reading earlier results).
@@ -196,6 +209,9 @@ cudaError_t launch_select(const SelectParams &p, cudaStream_t stream, int thread
 size_t select_smem_bytes(int threads, int k);
 cudaError_t launch_gather(const GatherParams &p, cudaStream_t stream, bool pdl = false);
 cudaError_t launch_certify(const CertifyParams &p, cudaStream_t stream, bool pdl = false);
+size_t tiny_smem_bytes(int NQ, int k);
+// One cooperative grid of `grid` CTAs (all resident at once)
+cudaError_t launch_tiny(const TinyParams &p, int grid, cudaStream_t stream);
 bool indexer_supported(int G, int d_I);
 cudaError_t launch_indexer_scores(const IndexerScoreParams &p, int num_sms, cudaStream_t stream);
 cudaError_t launch_indexer_attn(const IndexerAttnParams &p, cudaStream_t stream);

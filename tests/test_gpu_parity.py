@@ -257,3 +257,21 @@ def test_block_bad_seq_len_raises_status_and_skips_sequence(cuda_device):
     ref = oracle.block_attn(w0, 32, 6)
     _, bidx0 = tka.topk_block_attn_decode(q[:1], kc[:1], vc[:1], bk[:1], lens[:1], 32, 6)
     check_block(w0, 32, 6, out[:1], bidx0, ref)
+
+
+def test_one_launch_path_matches_three_launches(cuda_device):
+    """Small problems take one cooperative launch (score, grid barrier, select
+    and attention per row); the staged call records events between its steps,
+    so it takes the three-kernel path.  With an fp32 cache both score on the
+    CUDA cores in the same order: identical kept sets, outputs to rounding."""
+    w = workloads.make_workload(2, 2, 8, 4, 4096, dtype="f32", seq_lens=[4096, 1777], seed=77)
+    q, kc, vc, lens = to_device(w)
+    k = 96
+    out1, idx1, tail1 = tka.topk_attn_decode(q, kc, vc, lens, k)
+    ev = [torch.cuda.Event(), None, None, None]
+    out3, idx3, tail3 = tka.topk_attn_decode(q, kc, vc, lens, k, stage_events=ev)
+    torch.cuda.synchronize()
+    assert tka.topk_attn_device_status() == 0
+    assert torch.equal(idx1, idx3)
+    assert (out1 - out3).abs().max().item() <= 1e-5 and (tail1 - tail3).abs().max().item() <= 1e-6
+    check_token(w, k, out1, idx1, tail1, oracle.topk_attn(w, k))
