@@ -67,6 +67,21 @@ __device__ __forceinline__ uint32_t canon_key(float f) { return order_key(__fadd
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
 
+// An L2 policy for data read once: the lines it brings in are evicted first,
+// so that streaming it does not push out lines still to be read.
+__device__ __forceinline__ uint64_t l2_evict_first() {
+    uint64_t pol;
+    asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+// A 4-byte load that bypasses L1 and allocates in L2 under policy `pol`.
+__device__ __forceinline__ float ld_l2_hint(const float *a, uint64_t pol) {
+    float v;
+    asm("ld.global.L1::no_allocate.L2::cache_hint.f32 %0, [%1], %2;" : "=f"(v) : "l"(a), "l"(pol));
+    return v;
+}
+
 // 2^t by the hardware approximation (PTX ex2.approx.ftz.f32).
 __device__ __forceinline__ float exp2_approx(float t) {
     float r;

@@ -266,18 +266,31 @@ struct InRange {
 // loads in flight while the current one is processed.  valid is the
 // compile-time constant InRange{} for every chunk that lies wholly inside the
 // range; past the range x is -inf.
-template <typename F>
+// kEvictFirst: the scores of all rows exceed L2, so part of them was pushed
+// out by the ones written after; evict-first loads keep the lines still
+// resident from being pushed out by the ones this read brings back.
+template <bool kEvictFirst>
+__device__ __forceinline__ float ld_score(const float *a, uint64_t pol) {
+    if constexpr (kEvictFirst)
+        return ld_l2_hint(a, pol);
+    else
+        return __ldcg(a);
+}
+
+template <bool kEvictFirst, typename F>
 __device__ __forceinline__ void stream_range(const float *s, int lo, int hi, int lane, F &&f) {
     const int nch = (hi - lo + 32 * kU - 1) / (32 * kU);
     float a[kU], b[kU];
+    const uint64_t pol = kEvictFirst ? l2_evict_first() : 0ull;
     auto load = [&](float(&x)[kU], int c) {
         const int p0 = lo + c * 32 * kU + lane;
         if (lo + (c + 1) * 32 * kU <= hi) {
 #pragma unroll
-            for (int u = 0; u < kU; u++) x[u] = __ldcg(s + p0 + 32 * u);
+            for (int u = 0; u < kU; u++) x[u] = ld_score<kEvictFirst>(s + p0 + 32 * u, pol);
         } else {
 #pragma unroll
-            for (int u = 0; u < kU; u++) x[u] = p0 + 32 * u < hi ? __ldcg(s + p0 + 32 * u) : -INFINITY;
+            for (int u = 0; u < kU; u++)
+                x[u] = p0 + 32 * u < hi ? ld_score<kEvictFirst>(s + p0 + 32 * u, pol) : -INFINITY;
         }
     };
     auto run = [&](float(&x)[kU], int c) {
@@ -310,8 +323,9 @@ __device__ __forceinline__ void st_shared_v2_if(bool p, void *a, uint32_t x, uin
 }
 
 // The select step of one row by the whole CTA (kThreads threads, the dynamic
-// shared memory select_smem_bytes(kThreads, p.k)).
-template <int kThreads>
+// shared memory select_smem_bytes(kThreads, p.k)); kEvictFirst as for
+// ld_score.
+template <int kThreads, bool kEvictFirst = false>
 __device__ void select_row(const SelectParams &p, int row) {
     constexpr int kWarps = kThreads / 32;
     static_assert(kWarps <= 32 && kThreads % 32 == 0, "at most 32 whole warps");
@@ -363,7 +377,7 @@ __device__ void select_row(const SelectParams &p, int row) {
 #pragma unroll
     for (int j = 0; j < kS; j++) {
         const int pos = lo + 32 * j * gstep + lane;
-        sv[j] = pos < hi ? __ldcg(s + pos) : 0.f;
+        sv[j] = pos < hi ? ld_score<kEvictFirst>(s + pos, kEvictFirst ? l2_evict_first() : 0ull) : 0.f;
     }
 #pragma unroll
     for (int j = 0; j < kS; j++) {
@@ -412,7 +426,7 @@ __device__ void select_row(const SelectParams &p, int row) {
     const float ms_l2e = m_s * kLog2e;
     float m_lane = -INFINITY, zall = 0.f;
     uint32_t nl = 0u;
-    stream_range(s, lo, hi, lane, [&](float x, int pos, auto valid) {
+    stream_range<kEvictFirst>(s, lo, hi, lane, [&](float x, int pos, auto valid) {
         m_lane = fmaxf(m_lane, x);
         zall += exp2_approx(fmaf(x, kLog2e, -ms_l2e));
         const bool sel = valid && x >= lo_t;
