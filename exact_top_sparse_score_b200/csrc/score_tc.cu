@@ -94,8 +94,10 @@ struct TileWalk {
 };
 
 // 32 or 64 query columns: the epilogue stages each tile's scores in shared
-// memory and one TMA store writes them (a 3-D box [Q][G][128 keys] of the
-// scores viewed as [B*Q, Hq, ld]); fewer columns store straight from registers
+// memory (two staging tiles, 64 KB with 64 columns: the 4 K stages, both query
+// buffers and both staging tiles take 225 KB of the 227 KB a CTA may have) and
+// one TMA store writes them (a 3-D box [Q][G][128 keys] of the scores viewed
+// as [B*Q, Hq, ld]); fewer columns store straight from registers
 __host__ __device__ constexpr bool tma_store_for(int N) { return N == 32 || N == 64; }
 
 // kProbe: the pipeline waits are diagnostic probes bounded by p.max_polls
@@ -107,7 +109,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int S = stages_for(N);
     constexpr uint32_t kCols = tmem_cols_for(N);
     constexpr int kQBuf = N * 256;  // two 64-dim blocks of N rows x 128 B
-    constexpr int kOutBytes = tma_store_for(N) ? N * kTileKeys * 4 : 0;  // one tile of scores, [n][key]
+    constexpr int kOutBytes = tma_store_for(N) ? 2 * N * kTileKeys * 4 : 0;  // two tiles of scores, [n][key]
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *stages = base;
@@ -270,13 +272,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!mbar_wait(drain, 0, reinterpret_cast<volatile int *>(&no_abort))) ok = false;
         }
     } else if (tma_store_for(N)) {
-        // each tile: TMEM -> registers -> the shared-memory tile (column n at
-        // [n][key]); the 128 epilogue threads decide together whether to go
-        // on (a barrier that ANDs their waits: no thread is left behind at
-        // the barriers below), the accumulator is released as soon as it has
-        // been read, and one thread stores the tile with TMA once the previous
-        // store has finished reading the buffer.  Scores a causal query
-        // position cannot see are stored too: nothing reads them.
+        // each tile: TMEM -> registers (every column's load issued before
+        // one wait) -> one of two shared-memory tiles (column n at [n][key]);
+        // the 128 epilogue threads decide together whether to go on (a
+        // barrier that ANDs their waits: no thread is left behind at the
+        // barriers below), the accumulator is released as soon as it has been
+        // read, and one thread stores the tile with TMA.  A staging tile is
+        // rewritten two tiles later, once its store has read it.  Scores a
+        // causal query position cannot see are stored too: nothing reads them.
         const int quarter = warp & 3;  // TMEM lanes [32*quarter, +32)
         const uint32_t tlane = (uint32_t)(quarter * 32) << 16;
         const int kq = quarter * 32 + lane;
@@ -289,24 +292,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = named_bar_and(1, 128, ok);
             if (!ok) break;
             tc_fence_after();
-            if (issuer) bulk_wait_read_all();
-            named_bar_sync(1, 128);  // the buffer is free
+            float *stage = outbuf + (i & 1) * (N * kTileKeys);
+            uint32_t r[N / 16][16];
+#pragma unroll
+            for (int c = 0; c < N / 16; c++)
+                if (c * 16 < p.NQ) tmem_ld16(tmem + tlane + buf * N + c * 16, r[c]);
+            if (issuer) bulk_wait_read_but_one();  // the store of two tiles ago has read this stage
+            tmem_wait_ld();
+            named_bar_sync(1, 128);  // the stage is free
 #pragma unroll
             for (int c = 0; c < N / 16; c++) {
                 if (c * 16 >= p.NQ) break;
-                uint32_t r[16];
-                tmem_ld16(tmem + tlane + buf * N + c * 16, r);
-                tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 16; j++)
-                    if (c * 16 + j < p.NQ) outbuf[(c * 16 + j) * kTileKeys + kq] = __uint_as_float(r[j]) * scale;
+                    if (c * 16 + j < p.NQ) stage[(c * 16 + j) * kTileKeys + kq] = __uint_as_float(r[c][j]) * scale;
             }
             tc_fence_before();
             mbar_arrive(&tempty[buf]);
             fence_proxy_async_shared();
             named_bar_sync(1, 128);  // the tile is complete
             if (issuer) {
-                tma_store_3d(&smap, outbuf, w.t * kTileKeys, kvh * p.G, b * p.Q);
+                tma_store_3d(&smap, stage, w.t * kTileKeys, kvh * p.G, b * p.Q);
                 bulk_commit_group();
             }
             w.next(p);
@@ -382,7 +388,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int N>
 size_t smem_bytes() {
     constexpr int S = stages_for(N);
-    return 1024 + (size_t)S * kTileBytes + 2 * (size_t)N * 256 + (tma_store_for(N) ? (size_t)N * kTileKeys * 4 : 0) +
+    return 1024 + (size_t)S * kTileBytes + 2 * (size_t)N * 256 +
+           (tma_store_for(N) ? 2 * (size_t)N * kTileKeys * 4 : 0) +
            (2 * S + 9) * 8 + 64;
 }
 
