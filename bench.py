@@ -445,8 +445,13 @@ def run_ours(args, world, rank, local):
         flush_w.zero_()  # evicts everything the step left in L2 ...
         flush_r.amax()   # ... and leaves only clean lines behind
 
+    staged = not (block or certified or paged or hisa or indexer)
     for _ in range(args.warmup):
         step()
+        if staged:
+            # the stage-timed pass runs the three-kernel path, which a small
+            # problem's plain call (one launch) does not: load its kernels too
+            staged_step([None] * 4)
     torch.cuda.synchronize()
     if tka.topk_attn_device_status() != 0:
         raise RuntimeError("device status raised during warm-up")
@@ -459,7 +464,6 @@ def run_ours(args, world, rank, local):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    staged = not (block or certified or paged or hisa or indexer)
     sevs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)] if staged else []
     for e in (x for row in sevs for x in row):
         e.record()

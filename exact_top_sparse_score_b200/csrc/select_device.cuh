@@ -30,10 +30,12 @@
 //   emit    from the lists only: every kept entry (s > T, or s = T among the
 //           first ties) to its final ascending slot, with Z_k over the kept
 //           terms; Z_tail = sum_all - Z_k, the tail mass Z_tail / (Z_k + Z_tail).
-// If fewer than k scores reach lo_t, a warp's list overflows, or the sample
-// maximum lies too far below the row maximum for the sum against it, the row
-// falls back to three exact histogram passes and an ordered compaction pass
-// over the row.
+// A row the sample holds whole (at most 32 kS positions per warp) skips the
+// pass and the lists when the sample histogram settles the k-th score
+// (select_short).  If fewer than k scores reach lo_t, a warp's list
+// overflows, or the sample maximum lies too far below the row maximum for the
+// sum against it, the row falls back to three exact histogram passes and an
+// ordered compaction pass over the row.
 #pragma once
 
 #include <atomic>
@@ -322,6 +324,154 @@ __device__ __forceinline__ void st_shared_v2_if(bool p, void *a, uint32_t x, uin
                  : "memory");
 }
 
+// The select step of a row the sample holds whole (lane l of a warp holding
+// positions lo + l + 32 j of the warp's segment [lo, hi) in sv[j]): the sample
+// histogram's bin b* of the k-th score (scal[0], with scal[1] scores above it)
+// bounds it exactly, so the kept scores are those in bins above b* and, in b*,
+// either all of it (when that completes k) or, with at most 32 scores there,
+// those above the exact k-th key T plus the lowest-positioned ties at T.  They
+// are emitted straight from the registers: no second read of the row, no
+// lists.  Returns false, having written nothing, when b* holds more than 32
+// scores and is not kept whole (the caller takes the general route).
+template <int kThreads>
+__device__ __forceinline__ bool select_short(const SelectParams &p, int row, int lo, int hi, const float (&sv)[kS],
+                                             float min_s, float m_s, float scale_s, uint32_t *wstat,
+                                             const SelectSmem &sm) {
+    constexpr int kWarps = kThreads / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t lt = lanemask_lt();
+    const int k = p.k;
+    auto wword = [&](int f) { return lane < kWarps ? wstat[lane * 8 + f] : 0u; };
+    // the sample histogram's bin function, expression for expression
+    auto binv = [&](float x) { return (uint32_t)min(2047, (int)((x - min_s) * scale_s)); };
+    const uint32_t bstar = sm.scal[0], c_star = sm.hist[bstar], r = (uint32_t)k - sm.scal[1];  // 1 <= r <= c_star
+    const bool by_bin = r == c_star;
+    if (!by_bin && c_star > 32u) {
+        __syncthreads();  // every thread has read the histogram before the caller clears it
+        return false;
+    }
+    uint32_t T_key = 0u, r_eq = 0u;
+    if (!by_bin) {
+        uint32_t *cand = sm.tmp;  // [32]: free after the bin search
+        if (threadIdx.x == 0) sm.scal[4] = 0u;
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < kS; j++)
+            if (lo + 32 * j + lane < hi && binv(sv[j]) == bstar) cand[atomicAdd(&sm.scal[4], 1u)] = canon_key(sv[j]);
+        __syncthreads();
+        if (warp == 0) {
+            const uint32_t mine = lane < (int)c_star ? cand[lane] : 0u;
+            uint32_t g = 0u, e = 0u;
+            for (uint32_t j = 0; j < c_star; j++) {
+                const uint32_t o = cand[j];
+                g += o > mine;
+                e += o == mine;
+            }
+            const uint32_t hit = __ballot_sync(0xffffffffu, lane < (int)c_star && g < r && r <= g + e);
+            const int L = hit ? __ffs(hit) - 1 : 0;
+            const uint32_t tk = __shfl_sync(0xffffffffu, mine, L), tg = __shfl_sync(0xffffffffu, g, L);
+            if (lane == 0) {
+                sm.scal[5] = tk;
+                sm.scal[6] = r - tg;
+                if (!hit) raise_status(p.status, TKA_DEV_INTERNAL);
+            }
+        }
+        __syncthreads();
+        T_key = sm.scal[5];
+        r_eq = sm.scal[6];
+    }
+    auto above = [&](float x) { return by_bin ? binv(x) >= bstar : canon_key(x) > T_key; };
+    auto tie = [&](float x) { return !by_bin && canon_key(x) == T_key; };
+
+    // ---- per warp: kept scores above T and ties at T, then output offsets
+    {
+        uint32_t g = 0u, t = 0u;
+#pragma unroll
+        for (int j = 0; j < kS; j++) {
+            if (lo + 32 * j + lane < hi) {
+                g += above(sv[j]);
+                t += tie(sv[j]);
+            }
+        }
+        g = warp_sum(g);
+        t = warp_sum(t);
+        if (lane == 0) {
+            wstat[warp * 8 + 5] = g;
+            wstat[warp * 8 + 6] = t;
+        }
+    }
+    __syncthreads();
+    uint32_t out_run, tie_run, n_eq;
+    {
+        const uint32_t tie_l = wword(6);
+        const uint32_t tie_incl = warp_incl_scan(tie_l), tie_excl = tie_incl - tie_l;
+        const uint32_t kept_l = wword(5) + (r_eq > tie_excl ? min(tie_l, r_eq - tie_excl) : 0u);
+        const uint32_t out_incl = warp_incl_scan(kept_l);
+        out_run = __shfl_sync(0xffffffffu, out_incl - kept_l, warp);
+        tie_run = __shfl_sync(0xffffffffu, tie_excl, warp);
+        n_eq = __shfl_sync(0xffffffffu, tie_incl, 31);
+    }
+    const bool rank_ties = r_eq < n_eq;
+    const uint32_t out_begin = out_run;
+
+    // ---- emit in position order; Z_k over the kept, Z_tail over the rest
+    int32_t *idx = p.idx + (size_t)row * k;
+    float *wv = p.w + (size_t)row * k;
+    const float m = m_s;  // the sample is the whole row
+    const float m_l2e = m * kLog2e;
+    float zk = 0.f, zt = 0.f;
+#pragma unroll
+    for (int j = 0; j < kS; j++) {
+        const int pos = lo + 32 * j + lane;
+        const bool in = pos < hi;
+        const float xv = sv[j];
+        bool sel = in && above(xv);
+        if (rank_ties) {
+            const bool t = in && tie(xv);
+            const uint32_t tb = __ballot_sync(0xffffffffu, t);
+            sel = sel || (t && tie_run + __popc(tb & lt) < r_eq);
+            tie_run += __popc(tb);
+        } else {
+            sel = sel || (in && tie(xv));
+        }
+        const uint32_t sb = __ballot_sync(0xffffffffu, sel);
+        if (in) {
+            const float ew = exp2_approx(fmaf(xv, kLog2e, -m_l2e));
+            if (sel) {
+                const uint32_t o = out_run + __popc(sb & lt);
+                if (o < (uint32_t)k) {  // always true unless the counts above are wrong
+                    idx[o] = pos;
+                    wv[o] = ew;
+                }
+                zk += ew;
+            } else {
+                zt += ew;
+            }
+        }
+        out_run += __popc(sb);
+    }
+    zk = warp_sum(zk);
+    zt = warp_sum(zt);
+    if (lane == 0) {  // words 1-3: words 5 and 6 may still be read by a slower warp's scan
+        wstat[warp * 8 + 1] = __float_as_uint(zk);
+        wstat[warp * 8 + 2] = out_run - out_begin;
+        wstat[warp * 8 + 3] = __float_as_uint(zt);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const float zk_row = warp_sum(lane < kWarps ? __uint_as_float(wstat[lane * 8 + 1]) : 0.f);
+        const float zt_row = warp_sum(lane < kWarps ? __uint_as_float(wstat[lane * 8 + 3]) : 0.f);
+        const uint32_t written = warp_sum(wword(2));
+        if (lane == 0) {
+            if (written != (uint32_t)k) raise_status(p.status, TKA_DEV_INTERNAL);
+            p.stats[row] = make_float4(m, zk_row, zt_row, 0.f);
+            if (p.tail) p.tail[row] = zt_row / (zk_row + zt_row);
+            p.counters[row] = 0u;
+        }
+    }
+    return true;
+}
+
 // The select step of one row by the whole CTA (kThreads threads, the dynamic
 // shared memory select_smem_bytes(kThreads, p.k)); kEvictFirst as for
 // ld_score.
@@ -416,6 +566,8 @@ __device__ void select_row(const SelectParams &p, int row) {
         // one bin lower than the bin's bottom edge: below every sample score in it
         lo_t = b_lo > 0u ? min_s + (float)(b_lo - 1u) / scale_s : -INFINITY;
     }
+    // a row the sample holds whole: the bin search above bounds the k-th score exactly
+    if (!sampled && select_short<kThreads>(p, row, lo, hi, sv, min_s, m_s, scale_s, wstat, sm)) return;
     for (int i = threadIdx.x; i < 2048; i += kThreads) sm.hist[i] = 0u;  // for the list histogram
 
     // ---- the one pass over the row: its maximum, sum e^{s - m_s} against the
@@ -601,13 +753,15 @@ __device__ void select_row(const SelectParams &p, int row) {
     }
     zk = warp_sum(zk);
     if (lane == 0) {
-        wstat[warp * 8 + 6] = __float_as_uint(zk);
-        wstat[warp * 8 + 7] = out_run - out_begin;
+        // words 1 and 2 (the sample's, read long before): words 5 and 6 may
+        // still be read by a slower warp's offset scan above
+        wstat[warp * 8 + 1] = __float_as_uint(zk);
+        wstat[warp * 8 + 2] = out_run - out_begin;
     }
     __syncthreads();
     if (warp == 0) {
-        const float zk_row = warp_sum(lane < kWarps ? __uint_as_float(wstat[lane * 8 + 6]) : 0.f);
-        const uint32_t written = warp_sum(wword(7));
+        const float zk_row = warp_sum(lane < kWarps ? __uint_as_float(wstat[lane * 8 + 1]) : 0.f);
+        const uint32_t written = warp_sum(wword(2));
         if (lane == 0) {
             const float zt = fmaxf(z_all - zk_row, 0.f);  // formed as total - kept: >= 0
             if (written != (uint32_t)k) raise_status(p.status, TKA_DEV_INTERNAL);

@@ -118,6 +118,34 @@ def test_all_scores_equal(B, cuda_device):
     check_token(w, k, out, idx, tail, ref)
 
 
+@pytest.mark.parametrize("k", [100, 2047])
+def test_short_row_all_scores_equal(k, cuda_device):
+    # a row its select step samples whole (2048 keys) with every score equal:
+    # the k-th score's bin holds more than 32 scores, so the row leaves the
+    # register-resident route for the lists and the exact multi-pass route
+    w = workloads.make_workload(1, 1, 8, 2, 2048, dtype="bf16", seed=21)
+    w.k_cache[:] = w.k_cache[:, :, :1].expand_as(w.k_cache)
+    out, idx, tail = run_token(w, k)
+    ref = oracle.topk_attn(w, k)
+    assert np.array_equal(idx.cpu().numpy(), ref["idx"])
+    check_token(w, k, out, idx, tail, ref)
+
+
+def test_short_row_ties_inside_the_kth_bin(cuda_device):
+    # 40 distinct key rows repeated along 1024 positions: the k-th score's
+    # value occurs ~26 times, the register-resident route ranks the bin's
+    # scores and keeps the lowest-positioned ties
+    L = 1024
+    w = workloads.make_workload(2, 1, 8, 2, L, dtype="bf16", seed=22)
+    src = torch.arange(L) % 40
+    w.k_cache[:] = w.k_cache[:, :, src]
+    for k in (30, 333):
+        out, idx, tail = run_token(w, k)
+        ref = oracle.topk_attn(w, k)
+        assert np.array_equal(idx.cpu().numpy(), ref["idx"])
+        check_token(w, k, out, idx, tail, ref)
+
+
 def test_repeat_calls_are_bitwise_identical(cuda_device):
     w = workloads.make_workload(2, 1, 32, 8, 3000, dtype="bf16", seed=6)
     q, kc, vc, lens = to_device(w)
