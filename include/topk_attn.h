@@ -103,7 +103,11 @@ typedef struct {
 size_t topk_attn_workspace_size(const tka_shape *shape, int32_t k);
 
 /* Exact Top-k decode attention for all B*Q*Hq query rows (see top of file).
- * idx is required; tail_mass may be NULL. */
+ * idx is required; tail_mass may be NULL.  Three kernels (score, select,
+ * attention over the kept rows); a small problem -- at most 65536 cache rows
+ * in all (B*Hkv*L_max), no more query rows and kv-heads than the GPU has SMs,
+ * at most 64 query rows per kv-head -- runs as one cooperative launch with the
+ * same results up to the rounding of the fp32 scores. */
 tka_status topk_attn_decode(const tka_shape *shape, const void *q, const void *k_cache,
                             const void *v_cache, const int32_t *seq_lens, int32_t k, float *out,
                             int32_t *idx, float *tail_mass, void *workspace, size_t workspace_bytes,
@@ -115,8 +119,10 @@ tka_status topk_attn_decode(const tka_shape *shape, const void *q, const void *k
  * events[2] between select and gather (idx is final there: a caller may start
  * copying it out while the gather runs), events[3] after gather.  Any entry
  * may be null (not recorded).  Used to time each step, or to overlap the idx
- * read-back with the gather, without changing what runs; a kernel that follows
- * a recorded event does not start early behind the kernel before it. */
+ * read-back with the gather; a kernel that follows a recorded event does not
+ * start early behind the kernel before it.  This call always runs the three
+ * kernels (a small problem included), with the results topk_attn_decode gives
+ * up to the rounding of the fp32 scores. */
 typedef struct CUevent_st *tka_event_t;
 tka_status topk_attn_decode_staged(const tka_shape *shape, const void *q, const void *k_cache,
                                    const void *v_cache, const int32_t *seq_lens, int32_t k, float *out,
