@@ -77,3 +77,23 @@ def test_both_arms_describe_the_workload_with_one_config_object():
     w = workloads.config_workload(1, seed=1001)
     args = argparse.Namespace(certified_eps=None, paged=None, hisa=None, indexer=None)
     assert out[0]["config"] == bench.workload_config(w, w.k, 1, args)
+
+
+
+def test_launch_accounting_of_the_five_workloads():
+    # gpu_launches per step: the one-launch path takes workload 1 only (a
+    # 4096-row cache); the MoBA selection fits one cluster launch
+    import types
+
+    import bench
+    import workloads
+
+    def shape(c):
+        spec = dict(workloads.CONFIGS[c])
+        return types.SimpleNamespace(B=spec["B"], Q=spec["Q"], Hq=spec["Hq"], Hkv=spec["Hkv"], L_max=spec["L_max"])
+
+    one = {c: bench.one_launch(shape(c), 148) for c in (1, 2, 3, 5)}
+    assert one == {1: True, 2: False, 3: False, 5: False}
+    G4 = workloads.CONFIGS[4]["Hq"] // workloads.CONFIGS[4]["Hkv"]
+    assert bench.block_select_launches(G4, workloads.CONFIGS[4]["L_max"] // workloads.CONFIGS[4]["block_size"]) == 1
+    assert bench.block_select_launches(32, 131072 // 16) == 2
