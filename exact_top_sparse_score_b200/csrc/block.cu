@@ -351,8 +351,9 @@ __global__ void __launch_bounds__(kSelThreads) block_topk(BlockSelectParams p) {
 // gathers head g's scores of every chunk from the other CTAs' shared memory
 // (distributed shared memory) and keeps its top blocks.  A last cluster
 // barrier keeps every CTA's scores in place until all gathers are done.
+// (four CTAs per SM: 64 clusters of 8 fit in one wave on 148 SMs)
 template <typename T>
-__global__ void __launch_bounds__(kSelThreads) block_select_cluster(BlockSelectParams p) {
+__global__ void __launch_bounds__(kSelThreads, 4) block_select_cluster(BlockSelectParams p) {
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
     pdl_wait();  // inputs may come from the kernel before
@@ -381,27 +382,37 @@ __global__ void __launch_bounds__(kSelThreads) block_select_cluster(BlockSelectP
         const T *q = reinterpret_cast<const T *>(p.q) + ((size_t)b * p.Hq + (size_t)kvh * G) * kHeadDim;
         for (int e = threadIdx.x; e < G * 32; e += kSelThreads) qs[e] = load4(q + 4 * e);
         __syncthreads();
-        // eight lanes per block, lane c holding float4 columns c, c + 8, c + 16, c + 24
+        // eight lanes per block, lane c holding float4 columns c, c + 8, c + 16,
+        // c + 24; the loads of kRounds rounds of blocks are issued before any
+        // of them is scored (one memory round trip per kRounds rounds)
+        constexpr int kRounds = 2;
         const int c = threadIdx.x & 7;
         const float4 *bk = reinterpret_cast<const float4 *>(p.block_keys + (size_t)bh * p.nblk_max * kHeadDim);
         const int j_lo = rank * ch, j_hi = min(ncomp, j_lo + ch);
-        for (int j0 = j_lo; j0 < j_hi; j0 += kSelThreads / 8) {
-            const int j = j0 + (threadIdx.x >> 3);
-            float4 kv[4];
+        for (int j0 = j_lo; j0 < j_hi; j0 += kRounds * (kSelThreads / 8)) {
+            float4 kv[kRounds][4];
 #pragma unroll
-            for (int u = 0; u < 4; u++)
-                kv[u] = j < j_hi ? __ldg(bk + (size_t)j * 32 + c + 8 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int g = 0; g < G; g++) {
-                float s = 0.f;
+            for (int r = 0; r < kRounds; r++) {
+                const int j = j0 + r * (kSelThreads / 8) + (threadIdx.x >> 3);
 #pragma unroll
-                for (int u = 0; u < 4; u++) {
-                    const float4 qv = qs[g * 32 + c + 8 * u];
-                    s += qv.x * kv[u].x + qv.y * kv[u].y + qv.z * kv[u].z + qv.w * kv[u].w;
+                for (int u = 0; u < 4; u++)
+                    kv[r][u] = j < j_hi ? __ldg(bk + (size_t)j * 32 + c + 8 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int r = 0; r < kRounds; r++) {
+                const int j = j0 + r * (kSelThreads / 8) + (threadIdx.x >> 3);
+                for (int g = 0; g < G; g++) {
+                    float s = 0.f;
+#pragma unroll
+                    for (int u = 0; u < 4; u++) {
+                        const float4 qv = qs[g * 32 + c + 8 * u];
+                        s += qv.x * kv[r][u].x + qv.y * kv[r][u].y + qv.z * kv[r][u].z + qv.w * kv[r][u].w;
+                    }
+                    s += __shfl_xor_sync(0xffffffffu, s, 1);
+                    s += __shfl_xor_sync(0xffffffffu, s, 2);
+                    s += __shfl_xor_sync(0xffffffffu, s, 4);
+                    if (c == 0 && j < j_hi) sc[(size_t)g * chmax + (j - j_lo)] = s * p.scale;
                 }
-                s += __shfl_xor_sync(0xffffffffu, s, 1);
-                s += __shfl_xor_sync(0xffffffffu, s, 2);
-                s += __shfl_xor_sync(0xffffffffu, s, 4);
-                if (c == 0 && j < j_hi) sc[(size_t)g * chmax + (j - j_lo)] = s * p.scale;
             }
         }
     }
